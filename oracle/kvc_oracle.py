@@ -330,19 +330,24 @@ def decode_dense(q, K, V, scale):
 def decode_varrate(q, lat_k, lat_v, rank_k, rank_v, bk, bv, scale):
     """Per-token variable rank.  lat_* [B, Hkv, T, rmax] (entries beyond the
     token's rank are ignored), rank_* [B, T] (every rank >= 1), factors
-    [Hkv, rmax, d] truncated to the token's first r rows."""
+    [Hkv, rmax, d] truncated to the token's first r rows:
+    k_t = lat_t[:r_t] Bk[:r_t]."""
     bsz, hkv, T, _ = lat_k.shape
     d = bk.shape[-1]
     out = np.empty((bsz, q.shape[1], bv.shape[-1]))
     for b in range(bsz):
+        rk = np.asarray(rank_k)[b, :T].astype(np.int64)
+        rv = np.asarray(rank_v)[b, :T].astype(np.int64)
+        assert (rk >= 1).all() and (rv >= 1).all(), "a token is never at rank zero"
         K = np.empty((hkv, T, d))
         V = np.empty((hkv, T, bv.shape[-1]))
         for g in range(hkv):
-            for t in range(T):
-                rk, rv = int(rank_k[b, t]), int(rank_v[b, t])
-                assert rk >= 1 and rv >= 1, "a token is never at rank zero"
-                K[g, t] = lat_k[b, g, t, :rk] @ bk[g, :rk]
-                V[g, t] = lat_v[b, g, t, :rv] @ bv[g, :rv]
+            for r in np.unique(rk):
+                tok = np.nonzero(rk == r)[0]
+                K[g, tok] = lat_k[b, g][tok][:, :r] @ bk[g, :r]
+            for r in np.unique(rv):
+                tok = np.nonzero(rv == r)[0]
+                V[g, tok] = lat_v[b, g][tok][:, :r] @ bv[g, :r]
         out[b] = gqa_decode(q[b], K, V, scale)
     return out
 
@@ -383,35 +388,37 @@ def gather_pages(pool, page_table, n_tokens, page_size):
     physical page page_table[b, t // P])."""
     pool = np.asarray(pool)
     pt = np.asarray(page_table)
-    bsz = pt.shape[0]
-    hkv = pool.shape[1]
-    out = np.empty((bsz, hkv, n_tokens) + pool.shape[3:], dtype=pool.dtype)
-    for b in range(bsz):
-        for t in range(n_tokens):
-            out[b, :, t] = pool[pt[b, t // page_size], :, t % page_size]
-    return out
+    t = np.arange(n_tokens)
+    phys = pt[:, t // page_size]                       # [B, T]
+    g = pool[phys, :, t[None, :] % page_size]          # [B, T, Hkv, ...]
+    return np.moveaxis(g, 2, 1)
 
 
 def read_varrate_records(stream, offsets, ranks, n_kv_heads, n_tokens, rmax, g):
     """Ragged per-token records.  For batch row b and token t the record is
     stream[b, offsets[b, t] : offsets[b, t + 1]], holding for each KV head in
     turn: r/2 code bytes, then ceil(r/g) (scale, zero) fp16 pairs, r = ranks[b, t].
-    Returns dequantized latents [B, Hkv, T, rmax], zero beyond each token's rank."""
+    Returns dequantized latents [B, Hkv, T, rmax], zero beyond each token's rank.
+    (Tokens are handled in groups of equal rank; each group is read the same way.)"""
     stream = np.asarray(stream, dtype=np.uint8)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    ranks = np.asarray(ranks)[:, :n_tokens].astype(np.int64)
     bsz = stream.shape[0]
     out = np.zeros((bsz, n_kv_heads, n_tokens, rmax))
     for b in range(bsz):
-        for t in range(n_tokens):
-            r = int(ranks[b, t])
+        sizes = offsets[b, 1 : n_tokens + 1] - offsets[b, :n_tokens]
+        for r in np.unique(ranks[b]):
+            r = int(r)
             ng = n_groups(r, g)
-            pos = int(offsets[b, t])
+            per_head = r // 2 + 4 * ng
+            tok = np.nonzero(ranks[b] == r)[0]
+            assert (sizes[tok] == n_kv_heads * per_head).all(), "record length mismatch"
             for h in range(n_kv_heads):
-                codes = stream[b, pos : pos + r // 2]
-                pos += r // 2
-                sz = stream[b, pos : pos + 4 * ng].view(np.float16).reshape(ng, 2)
-                pos += 4 * ng
-                out[b, h, t, :r] = read_int4_latent(codes, sz, r, g)
-            assert pos == int(offsets[b, t + 1]), "record length mismatch"
+                start = offsets[b, tok] + h * per_head               # [n]
+                codes = stream[b][start[:, None] + np.arange(r // 2)]
+                szb = stream[b][start[:, None] + r // 2 + np.arange(4 * ng)]
+                sz = np.ascontiguousarray(szb).view(np.float16).reshape(len(tok), ng, 2)
+                out[b, h, tok, :r] = read_int4_latent(codes, sz, r, g)
     return out
 
 

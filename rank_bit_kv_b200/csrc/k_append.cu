@@ -1,0 +1,235 @@
+// Append: project each new token's pre-RoPE key / value onto the latent and
+// quantize it into its slot (contiguous row, page slot or ragged record).
+//
+//   l = x Bk^T                                     (fp32, summed over d in order)
+//   INT4 per group: z = fp16(min), s = fp16((max - min) / 15),
+//                   code = clamp(rint((l - z) / s), 0, 15)  (IEEE fp32 divide,
+//                   round half to even; code 0 when s == 0)
+//   residual:       e = x - l_hat Bk, y = H (diag(signs) e) / sqrt(128),
+//                   s = fp16(max|y| / 1.5), code = clamp(floor(y / s) + 2, 0, 3)
+//   block-shared:   s = fp16(max|x| / 7), code = clamp(rint(x / s), -7, 7) + 8
+// This is the min/max rule of the BellowsKV worked example ("Worked Example:
+// Why the Latent Quantizes Flat", qerr: s = (hi - lo) / 15,
+// round((v - lo) / s)) with the scale and zero stored in fp16.
+#include <math.h>
+
+#include "kvc_device.cuh"
+
+namespace kvc {
+namespace {
+
+constexpr int kThreads = 128;
+
+// Quantize lat[0..r) in groups of g into packed INT4 codes and (s, z) pairs.
+__device__ void quant_int4_asym(const float* lat, int r, int g, uint8_t* codes, __half* sz,
+                                float* lhat, int tid) {
+  __shared__ float gs[64], gz[64];
+  const int ng = (r + g - 1) / g;
+  if (tid < ng) {
+    const int a = tid * g, e = min(a + g, r);
+    float lo = lat[a], hi = lat[a];
+    for (int j = a + 1; j < e; ++j) lo = fminf(lo, lat[j]), hi = fmaxf(hi, lat[j]);
+    const __half z = __float2half_rn(lo);
+    const __half s = __float2half_rn((hi - lo) / 15.f);
+    gs[tid] = __half2float(s);
+    gz[tid] = __half2float(z);
+    sz[2 * tid] = s;
+    sz[2 * tid + 1] = z;
+  }
+  __syncthreads();
+  for (int i = tid; i < r / 2; i += kThreads) {
+    int c2[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int j = 2 * i + k, gi = j / g;
+      const float s = gs[gi], z = gz[gi];
+      int c = 0;
+      if (s > 0.f) c = (int)fminf(fmaxf(rintf((lat[j] - z) / s), 0.f), 15.f);
+      c2[k] = c;
+      if (lhat) lhat[j] = fmaf((float)c, s, z);
+    }
+    codes[i] = (uint8_t)(c2[0] | (c2[1] << 4));
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kThreads) append_lowrank_kernel(AppendParams a) {
+  const Params& p = a.p;
+  __shared__ float xs[128];
+  __shared__ float lat[128];
+  __shared__ float lhat[128];
+  __shared__ float ys[128];
+  __shared__ float red[kThreads / 32];
+  // grid: ((b * Hkv + h) * 2 + comp) * n_new + i
+  int idx = blockIdx.x;
+  const int i = idx % a.n_new;
+  idx /= a.n_new;
+  const int comp = idx % 2;
+  idx /= 2;
+  const int h = idx % p.Hkv;
+  const int b = idx / p.Hkv;
+  const int tid = threadIdx.x;
+  const int d = p.d;
+  const int tok = a.pos[b] + i;
+  const __nv_bfloat16* src = (comp == 0 ? a.k_new : a.v_new) + (((int64_t)b * p.Hkv + h) * a.n_new + i) * d;
+  for (int j = tid; j < d; j += kThreads) xs[j] = bf2f(src[j]);
+
+  int r;
+  const __half* fac;
+  if (p.kind == KVC_VARRATE) {
+    r = (comp == 0 ? p.rank_k : p.rank_v)[(int64_t)b * p.tmax + tok];
+    fac = (comp == 0 ? p.bk : p.bv) + (int64_t)h * 64 * d;
+  } else {
+    r = comp == 0 ? p.rk : p.rv;
+    fac = (comp == 0 ? p.bk : p.bv) + (int64_t)h * r * d;
+  }
+  __syncthreads();
+  for (int j = tid; j < r; j += kThreads) {
+    const __half* br = fac + (int64_t)j * d;
+    float acc = 0.f;
+    for (int k = 0; k < d; ++k) acc = fmaf(xs[k], h2f(br[k]), acc);
+    lat[j] = acc;
+  }
+  __syncthreads();
+
+  if (p.kind == KVC_VARRATE) {
+    const int* off = comp == 0 ? a.off_k_w : a.off_v_w;
+    uint8_t* stream = (comp == 0 ? a.lk_w : a.lv_w) + (size_t)b * p.stream_bytes;
+    uint8_t* rec = stream + off[(int64_t)b * (p.tmax + 1) + tok] + h * varrate_head_bytes(r);
+    quant_int4_asym(lat, r, 32, rec, reinterpret_cast<__half*>(rec + r / 2), nullptr, tid);
+    return;
+  }
+  const int64_t row = lowrank_row(p, b, h, tok);
+  if (p.bits == 16) {
+    __half* dst = reinterpret_cast<__half*>(comp == 0 ? a.lk_w : a.lv_w) + row * r;
+    for (int j = tid; j < r; j += kThreads) dst[j] = __float2half_rn(lat[j]);
+    return;
+  }
+  uint8_t* codes = (comp == 0 ? a.lk_w : a.lv_w) + row * (r / 2);
+  __half* sz = (comp == 0 ? a.lksz_w : a.lvsz_w) + row * 2 * ((r + p.g - 1) / p.g);
+  quant_int4_asym(lat, r, p.g, codes, sz, p.resid ? lhat : nullptr, tid);
+  if (!p.resid) return;
+
+  // residual against the dequantized latent, rotated into the Hadamard basis
+  const int8_t* sg = comp == 0 ? p.signs_k : p.signs_v;
+  for (int j = tid; j < d; j += kThreads) {
+    float e = xs[j];
+    for (int k = 0; k < r; ++k) e = fmaf(-lhat[k], h2f(fac[(int64_t)k * d + j]), e);
+    ys[j] = (float)sg[j] * e;
+  }
+  fwht_smem(ys, kResidDim, tid, kThreads);
+  const float inv = rsqrtf((float)kResidDim);
+  float amax = 0.f;
+  for (int j = tid; j < d; j += kThreads) {
+    ys[j] *= inv;
+    amax = fmaxf(amax, fabsf(ys[j]));
+  }
+  amax = warp_max(amax);
+  if ((tid & 31) == 0) red[tid >> 5] = amax;
+  __syncthreads();
+  float m = red[0];
+  for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+  const __half sh = __float2half_rn(m / 1.5f);
+  const float s = __half2float(sh);
+  if (tid == 0) (comp == 0 ? a.rks_w : a.rvs_w)[row] = sh;
+  uint8_t* rc = (comp == 0 ? a.rkc_w : a.rvc_w) + row * (kResidDim / 4);
+  for (int j = tid; j < kResidDim / 4; j += kThreads) {
+    int byte = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      int c = 2;
+      if (s > 0.f) c = (int)fminf(fmaxf(floorf(ys[4 * j + k] / s) + 2.f, 0.f), 3.f);
+      byte |= c << (2 * k);
+    }
+    rc[j] = (uint8_t)byte;
+  }
+}
+
+// VARRATE: offsets of the new records, offset[pos + i + 1] = offset[pos + i] + size.
+__global__ void varrate_offsets_kernel(AppendParams a) {
+  const Params& p = a.p;
+  const int comp = blockIdx.x % 2, b = blockIdx.x / 2;
+  if (threadIdx.x != 0) return;
+  int* off = (comp == 0 ? a.off_k_w : a.off_v_w) + (int64_t)b * (p.tmax + 1);
+  const uint8_t* rank = (comp == 0 ? p.rank_k : p.rank_v) + (int64_t)b * p.tmax;
+  int o = off[a.pos[b]];
+  for (int i = 0; i < a.n_new; ++i) {
+    o += p.Hkv * varrate_head_bytes(rank[a.pos[b] + i]);
+    off[a.pos[b] + i + 1] = o;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) append_block_kernel(AppendParams a) {
+  const Params& p = a.p;
+  const int i = blockIdx.x % a.n_new, b = blockIdx.x / a.n_new;
+  const int tok = a.pos[b] + i;
+  const int D = p.D, g = p.g, ng = D / g;
+  const __nv_bfloat16* src = a.k_new + ((int64_t)b * a.n_new + i) * D;
+  const int64_t mi = (int64_t)b * p.tmax + tok;
+  uint8_t* codes = a.lk_w + mi * (D / 2);
+  __half* sc = a.lksz_w + mi * ng;
+  __shared__ float gsc[64];
+  for (int gi = threadIdx.x; gi < ng; gi += kThreads) {
+    float m = 0.f;
+    for (int j = gi * g; j < (gi + 1) * g; ++j) m = fmaxf(m, fabsf(bf2f(src[j])));
+    const __half sh = __float2half_rn(m / 7.f);
+    sc[gi] = sh;
+    gsc[gi] = __half2float(sh);
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < D / 2; j += kThreads) {
+    int c2[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = 2 * j + k;
+      const float s = gsc[e / g];
+      int c = 8;
+      if (s > 0.f) c = (int)fminf(fmaxf(rintf(bf2f(src[e]) / s), -7.f), 7.f) + 8;
+      c2[k] = c;
+    }
+    codes[j] = (uint8_t)(c2[0] | (c2[1] << 4));
+  }
+}
+
+__global__ void append_dense_kernel(AppendParams a) {
+  const Params& p = a.p;
+  // grid: ((l * B + b) * Hkv + h) * n_new + i
+  int idx = blockIdx.x;
+  const int i = idx % a.n_new;
+  idx /= a.n_new;
+  const int h = idx % p.Hkv;
+  idx /= p.Hkv;
+  const int b = idx % p.B;
+  const int l = idx / p.B;
+  const int d = p.d;
+  const int64_t src = ((((int64_t)l * p.B + b) * p.Hkv + h) * a.n_new + i) * d;
+  const int64_t dst = ((((int64_t)l * p.B + b) * p.Hkv + h) * p.tmax + a.pos[b] + i) * d;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    a.kd_w[dst + j] = a.k_new[src + j];
+    a.vd_w[dst + j] = a.v_new[src + j];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendParams& a, cudaStream_t s) {
+  const Params& p = a.p;
+  switch (p.kind) {
+    case KVC_LOWRANK:
+      append_lowrank_kernel<<<p.B * p.Hkv * 2 * a.n_new, kThreads, 0, s>>>(a);
+      break;
+    case KVC_VARRATE:
+      varrate_offsets_kernel<<<p.B * 2, 32, 0, s>>>(a);
+      append_lowrank_kernel<<<p.B * p.Hkv * 2 * a.n_new, kThreads, 0, s>>>(a);
+      break;
+    case KVC_BLOCK_SHARED:
+      append_block_kernel<<<p.B * a.n_new, kThreads, 0, s>>>(a);
+      break;
+    default:
+      append_dense_kernel<<<p.L * p.B * p.Hkv * a.n_new, 128, 0, s>>>(a);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

@@ -1,0 +1,98 @@
+// Split combine and up-projection, once per query head.
+//
+// Merges the S split partials of a query row with the log-sum-exp rule
+// (w_s = 2^(m_s - m*), acc = sum w_s acc_s, l = sum w_s l_s), then maps the
+// value-space accumulator to the head dimension:
+//   LOWRANK / VARRATE : o = acc[:r] Bv (+ Q^T acc_res) / l
+//   BLOCK_SHARED      : o = acc W_v^l[:, head slice] / l
+//   DENSE             : o = acc / l
+// A row with no tokens (l = 0) produces zeros.
+#include <math.h>
+
+#include "kvc_device.cuh"
+
+namespace kvc {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kMaxS = 1024;
+
+__global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
+  extern __shared__ float sm[];
+  float* acc = sm;                       // [vdim]
+  float* ws = sm + p.vdim;               // [S] weights
+  __shared__ float lsum;
+  const int row = blockIdx.x;            // (l * B + b) * Hq + h
+  const int h = row % p.Hq;
+  const int l = row / (p.B * p.Hq);
+  const int kvh = h / p.G;
+  const int tid = threadIdx.x;
+  const size_t rows = (size_t)p.L * p.B * p.Hq;
+  const int pst = p.vdim + 2;
+  const float* part = p.part + (size_t)row * pst;
+
+  if (tid < 32) {
+    float mx = -INFINITY;
+    for (int s = tid; s < p.S; s += 32) mx = fmaxf(mx, part[(size_t)s * rows * pst + p.vdim]);
+    mx = warp_max(mx);
+    float lt = 0.f;
+    for (int s = tid; s < p.S; s += 32) {
+      const float* ps = part + (size_t)s * rows * pst;
+      const float w = (mx == -INFINITY) ? 0.f : exp2f(ps[p.vdim] - mx);
+      ws[s] = w;
+      lt += w * ps[p.vdim + 1];
+    }
+    lt = warp_sum(lt);
+    if (tid == 0) lsum = lt;
+  }
+  __syncthreads();
+  for (int j = tid; j < p.vdim; j += kThreads) {
+    float a = 0.f;
+    for (int s = 0; s < p.S; ++s) a = fmaf(ws[s], part[(size_t)s * rows * pst + j], a);
+    acc[j] = a;
+  }
+  __syncthreads();
+  const float L = lsum;
+  const float inv_l = L > 0.f ? 1.f / L : 0.f;
+  const int d = p.d;
+  float* outf = reinterpret_cast<float*>(p.out);
+  __nv_bfloat16* outb = reinterpret_cast<__nv_bfloat16*>(p.out);
+
+  if (p.kind == KVC_LOWRANK && p.resid) {
+    // Q^T acc_res = diag(signs_v) H acc_res / sqrt(128)
+    fwht_smem(acc + p.rv, kResidDim, tid, kThreads);
+  }
+  for (int i = tid; i < d; i += kThreads) {
+    float o = 0.f;
+    if (p.kind == KVC_LOWRANK || p.kind == KVC_VARRATE) {
+      const int r = p.kind == KVC_VARRATE ? 64 : p.rv;
+      const __half* bv = p.bv + (int64_t)kvh * r * d + i;
+      for (int j = 0; j < r; ++j) o = fmaf(acc[j], h2f(bv[(int64_t)j * d]), o);
+      if (p.kind == KVC_LOWRANK && p.resid)
+        o = fmaf((float)p.signs_v[i] * rsqrtf((float)kResidDim), acc[p.rv + i], o);
+    } else if (p.kind == KVC_BLOCK_SHARED) {
+      const __half* w = p.bv + (int64_t)l * p.D * p.Hkv * d + kvh * d + i;
+      for (int c = 0; c < p.D; ++c) o = fmaf(acc[c], h2f(w[(int64_t)c * p.Hkv * d]), o);
+    } else {
+      o = acc[i];
+    }
+    o *= inv_l;
+    if (p.out_bf16) outb[(int64_t)row * d + i] = __float2bfloat16_rn(o);
+    else outf[(int64_t)row * d + i] = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Params& p, cudaStream_t s) {
+  if (p.S > kMaxS) return cudaErrorInvalidValue;
+  const int rows = p.L * p.B * p.Hq;
+  const size_t bytes = ((size_t)p.vdim + p.S) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(combine_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  combine_kernel<<<rows, kThreads, bytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

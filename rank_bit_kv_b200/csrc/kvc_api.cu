@@ -1,0 +1,508 @@
+// Host layer of libkvc: layout validation, closed-form buffer sizes, split
+// planning and the C ABI entry points declared in include/kvc.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+#include <string>
+
+#include "kvc_internal.h"
+
+struct kvc_layout {
+  kvc_layout_desc d;
+  int G, L, ngk, ngv;
+  int lk_row, lv_row, lksz_row, lvsz_row;  // bytes per row
+  int64_t rows;                             // rows per low-rank component
+  int qdim, vdim;
+  int units;                                // independent (row, head) units of the split kernel
+  size_t sizes[KVC_NBUF];
+  float scale;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+kvc_status fail(kvc_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+kvc_status ok() {
+  g_err.clear();
+  return KVC_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Bytes of one VARRATE record per KV head at rank r (codes + (scale, zero) pairs).
+int varrate_head_bytes(int r) { return r / 2 + 4 * ceil_div(r, 32); }
+
+// Split planning: S splits per unit so that units * S covers about two waves
+// of the 148 SMs, each split a whole number of tiles.
+void plan(const kvc_layout* L, int n_tokens, int* S, int* split_len) {
+  const int tile = kvc::split_tile(L->d.kind, L->d.rope);
+  const int tiles = n_tokens > 0 ? ceil_div(n_tokens, tile) : 1;
+  int s = ceil_div(2 * kvc::kNumSMs, L->units > 0 ? L->units : 1);
+  if (s < 1) s = 1;
+  if (s > tiles) s = tiles;
+  int per = ceil_div(tiles, s);
+  *split_len = per * tile;
+  *S = ceil_div(tiles, per);
+}
+
+size_t ws_bytes(const kvc_layout* L, int n_tokens) {
+  int S, len;
+  plan(L, n_tokens, &S, &len);
+  const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
+  size_t b = round_up(rows * L->qdim * sizeof(float), 256);
+  b += round_up((size_t)S * rows * (L->vdim + 2) * sizeof(float), 256);
+  return b;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvc_last_error(void) { return g_err.c_str(); }
+
+const char* kvc_version(void) { return "kvc 0.1 (sm_100a)"; }
+
+kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out) {
+  if (!desc || !out) return fail(KVC_EINVAL, "kvc_create_layout: NULL argument");
+  *out = nullptr;
+  kvc_layout_desc d = *desc;
+  if (d.n_layers <= 0) d.n_layers = 1;
+  if (d.kind < KVC_DENSE_BF16 || d.kind > KVC_VARRATE)
+    return fail(KVC_EINVAL, "unknown kind %d", d.kind);
+  if (d.batch < 1 || d.batch > kvc::kMaxBatch)
+    return fail(KVC_EINVAL, "batch %d outside 1..%d", d.batch, kvc::kMaxBatch);
+  if (d.n_kv_heads < 1 || d.n_q_heads < 1 || d.n_q_heads % d.n_kv_heads)
+    return fail(KVC_EINVAL, "n_q_heads %d must be a positive multiple of n_kv_heads %d",
+                d.n_q_heads, d.n_kv_heads);
+  if (d.head_dim != 64 && d.head_dim != 128)
+    return fail(KVC_EUNSUPPORTED, "head_dim %d (64 or 128 supported)", d.head_dim);
+  if (d.max_tokens < 1) return fail(KVC_EINVAL, "max_tokens %d", d.max_tokens);
+  if (d.rope && d.kind != KVC_LOWRANK)
+    return fail(KVC_EUNSUPPORTED, "rope is a LOWRANK option");
+  if (d.rope && !(d.rope_theta > 1.0)) return fail(KVC_EINVAL, "rope_theta must be > 1");
+  if (d.resid_bits != 0 && d.resid_bits != 2)
+    return fail(KVC_EUNSUPPORTED, "resid_bits %d (0 or 2)", d.resid_bits);
+  if (d.resid_bits && (d.kind != KVC_LOWRANK || d.head_dim != kvc::kResidDim))
+    return fail(KVC_EUNSUPPORTED, "a rotated residual needs LOWRANK with head_dim 128");
+  if (d.page_size != 0 && d.page_size != 16)
+    return fail(KVC_EUNSUPPORTED, "page_size %d (0 or 16)", d.page_size);
+  if (d.page_size && d.kind != KVC_LOWRANK)
+    return fail(KVC_EUNSUPPORTED, "paging is a LOWRANK option");
+  if (d.page_size && (d.max_tokens % d.page_size || d.n_pages < 1))
+    return fail(KVC_EINVAL, "paged: max_tokens %% page_size must be 0 and n_pages >= 1");
+  if (d.n_layers > 1 && d.kind != KVC_BLOCK_SHARED && d.kind != KVC_DENSE_BF16)
+    return fail(KVC_EUNSUPPORTED, "n_layers > 1 only for BLOCK_SHARED and DENSE");
+
+  kvc_layout* L = new (std::nothrow) kvc_layout();
+  if (!L) return fail(KVC_EINVAL, "out of host memory");
+  L->d = d;
+  L->G = d.n_q_heads / d.n_kv_heads;
+  L->L = d.n_layers;
+  L->scale = d.softmax_scale > 0 ? d.softmax_scale : 1.0f / sqrtf((float)d.head_dim);
+  memset(L->sizes, 0, sizeof(L->sizes));
+  const size_t B = d.batch, Hkv = d.n_kv_heads, T = d.max_tokens, hd = d.head_dim;
+  kvc_status st = KVC_OK;
+  const char* why = "";
+
+  switch (d.kind) {
+    case KVC_LOWRANK: {
+      if (d.rank_k < 2 || d.rank_v < 2 || d.rank_k % 2 || d.rank_v % 2 || d.rank_k > 128 ||
+          d.rank_v > 128) {
+        st = KVC_EINVAL, why = "ranks must be even in 2..128";
+        break;
+      }
+      if (d.latent_bits != 16 && d.latent_bits != 4) {
+        st = KVC_EUNSUPPORTED, why = "latent_bits must be 16 or 4";
+        break;
+      }
+      if (d.latent_bits == 4 && (d.group_size < 2 || d.group_size % 2)) {
+        st = KVC_EINVAL, why = "group_size must be even and >= 2";
+        break;
+      }
+      if (d.latent_bits == 16 && d.resid_bits) {
+        st = KVC_EUNSUPPORTED, why = "a residual needs an INT4 latent";
+        break;
+      }
+      L->rows = d.page_size ? (int64_t)d.n_pages * Hkv * d.page_size : (int64_t)B * Hkv * T;
+      if (d.latent_bits == 4) {
+        L->ngk = ceil_div(d.rank_k, d.group_size);
+        L->ngv = ceil_div(d.rank_v, d.group_size);
+        L->lk_row = d.rank_k / 2;
+        L->lv_row = d.rank_v / 2;
+        L->lksz_row = 4 * L->ngk;
+        L->lvsz_row = 4 * L->ngv;
+      } else {
+        L->lk_row = 2 * d.rank_k;
+        L->lv_row = 2 * d.rank_v;
+      }
+      L->sizes[KVC_BUF_LK_CODES] = (size_t)L->rows * L->lk_row;
+      L->sizes[KVC_BUF_LV_CODES] = (size_t)L->rows * L->lv_row;
+      L->sizes[KVC_BUF_LK_SZ] = (size_t)L->rows * L->lksz_row;
+      L->sizes[KVC_BUF_LV_SZ] = (size_t)L->rows * L->lvsz_row;
+      if (d.resid_bits) {
+        L->sizes[KVC_BUF_RK_CODES] = L->sizes[KVC_BUF_RV_CODES] = (size_t)L->rows * hd / 4;
+        L->sizes[KVC_BUF_RK_SCALE] = L->sizes[KVC_BUF_RV_SCALE] = (size_t)L->rows * 2;
+        L->sizes[KVC_BUF_SIGNS_K] = L->sizes[KVC_BUF_SIGNS_V] = hd;
+      }
+      L->sizes[KVC_BUF_BK] = Hkv * d.rank_k * hd * 2;
+      L->sizes[KVC_BUF_BV] = Hkv * d.rank_v * hd * 2;
+      if (d.page_size) L->sizes[KVC_BUF_PAGE_TABLE] = B * (T / d.page_size) * 4;
+      const int res = d.resid_bits ? kvc::kResidDim : 0;
+      L->qdim = d.rope ? 0 : d.rank_k + res;
+      L->vdim = d.rank_v + res;
+      L->units = (int)(B * Hkv);
+      break;
+    }
+    case KVC_VARRATE: {
+      if (d.rank_k != 64 || d.rank_v != 64 || d.latent_bits != 4 || d.group_size != 32) {
+        st = KVC_EUNSUPPORTED, why = "VARRATE needs rank_k = rank_v = 64, latent_bits 4, group 32";
+        break;
+      }
+      const size_t per_tok = Hkv * varrate_head_bytes(64);
+      L->sizes[KVC_BUF_LK_CODES] = L->sizes[KVC_BUF_LV_CODES] = B * T * per_tok;
+      L->sizes[KVC_BUF_OFFSET_K] = L->sizes[KVC_BUF_OFFSET_V] = B * (T + 1) * 4;
+      L->sizes[KVC_BUF_RANK_K] = L->sizes[KVC_BUF_RANK_V] = B * T;
+      L->sizes[KVC_BUF_BK] = L->sizes[KVC_BUF_BV] = Hkv * 64 * hd * 2;
+      L->qdim = 64;
+      L->vdim = 64;
+      L->units = (int)(B * Hkv);
+      break;
+    }
+    case KVC_BLOCK_SHARED: {
+      if (d.latent_dim < 16 || d.latent_dim > 1024 || d.latent_dim % 16) {
+        st = KVC_EINVAL, why = "latent_dim must be a multiple of 16 in 16..1024";
+        break;
+      }
+      if (d.group_size < 2 || d.latent_dim % d.group_size || d.group_size % 2) {
+        st = KVC_EINVAL, why = "group_size must be even and divide latent_dim";
+        break;
+      }
+      if (d.latent_dim / d.group_size > 64) {
+        st = KVC_EUNSUPPORTED, why = "at most 64 scale groups per latent";
+        break;
+      }
+      if ((d.n_layers * d.n_q_heads) % kvc::kBlockQueries) {
+        st = KVC_EUNSUPPORTED, why = "n_layers * n_q_heads must be a multiple of 32";
+        break;
+      }
+      L->sizes[KVC_BUF_LK_CODES] = B * T * d.latent_dim / 2;
+      L->sizes[KVC_BUF_LK_SZ] = B * T * (d.latent_dim / d.group_size) * 2;
+      L->sizes[KVC_BUF_BK] = L->sizes[KVC_BUF_BV] =
+          (size_t)d.n_layers * d.latent_dim * Hkv * hd * 2;
+      L->qdim = d.latent_dim;
+      L->vdim = d.latent_dim;
+      L->units = (int)(B * d.n_layers * d.n_q_heads / kvc::kBlockQueries);
+      break;
+    }
+    case KVC_DENSE_BF16: {
+      L->sizes[KVC_BUF_K_DENSE] = L->sizes[KVC_BUF_V_DENSE] =
+          (size_t)d.n_layers * B * Hkv * T * hd * 2;
+      L->qdim = 0;
+      L->vdim = d.head_dim;
+      L->units = (int)(d.n_layers * B * Hkv);
+      break;
+    }
+  }
+  if (st != KVC_OK) {
+    delete L;
+    return fail(st, "kvc_create_layout: %s", why);
+  }
+  *out = L;
+  return ok();
+}
+
+void kvc_destroy_layout(kvc_layout* layout) { delete layout; }
+
+kvc_status kvc_buffer_sizes(const kvc_layout* L, size_t sizes[KVC_NBUF]) {
+  if (!L || !sizes) return fail(KVC_EINVAL, "kvc_buffer_sizes: NULL argument");
+  memcpy(sizes, L->sizes, sizeof(L->sizes));
+  return ok();
+}
+
+size_t kvc_step_bytes(const kvc_layout* L, int32_t n) {
+  if (!L || n <= 0) return 0;
+  const kvc_layout_desc& d = L->d;
+  const size_t rowsB = (size_t)d.batch * d.n_kv_heads * n;
+  switch (d.kind) {
+    case KVC_LOWRANK: {
+      size_t per = L->lk_row + L->lv_row + L->lksz_row + L->lvsz_row;
+      if (d.resid_bits) per += 2 * (d.head_dim / 4 + 2);
+      return rowsB * per;
+    }
+    case KVC_VARRATE: {
+      // expected record bytes under the rank mix {4,8,16,32,64} x {.4,.25,.2,.1,.05}
+      const double ef = 0.4 * 6 + 0.25 * 8 + 0.2 * 12 + 0.1 * 20 + 0.05 * 40;
+      return (size_t)((double)rowsB * 2 * ef) + (size_t)d.batch * n * 10;
+    }
+    case KVC_BLOCK_SHARED:
+      return (size_t)d.batch * n * (d.latent_dim / 2 + 2 * (d.latent_dim / d.group_size));
+    case KVC_DENSE_BF16:
+      return (size_t)d.n_layers * rowsB * d.head_dim * 2 * 2;
+  }
+  return 0;
+}
+
+size_t kvc_workspace_bytes(const kvc_layout* L, int32_t n_tokens) {
+  if (!L) return 0;
+  return ws_bytes(L, n_tokens < 0 ? 0 : n_tokens);
+}
+
+int32_t kvc_decode_launches(const kvc_layout* L, int32_t n_tokens) {
+  if (!L) return 0;
+  kvc::Params p;
+  p.kind = L->d.kind;
+  p.rope = L->d.rope;
+  return 2 + (kvc::needs_qproj(p) ? 1 : 0);
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------------
+// parameter assembly shared by append and decode
+// ----------------------------------------------------------------------------
+
+static kvc_status fill_params(const kvc_layout* L, const kvc_cache* c, kvc::Params* p) {
+  const kvc_layout_desc& d = L->d;
+  memset(p, 0, sizeof(*p));
+  p->kind = d.kind;
+  p->B = d.batch;
+  p->Hq = d.n_q_heads;
+  p->Hkv = d.n_kv_heads;
+  p->G = L->G;
+  p->d = d.head_dim;
+  p->L = L->L;
+  p->rk = d.rank_k;
+  p->rv = d.rank_v;
+  p->bits = d.latent_bits;
+  p->g = d.group_size;
+  p->ngk = L->ngk;
+  p->ngv = L->ngv;
+  p->resid = d.resid_bits;
+  p->rope = d.rope;
+  p->page = d.page_size;
+  p->tmax = d.max_tokens;
+  p->n_pages = d.n_pages;
+  p->D = d.latent_dim;
+  p->n_tokens = c->n_tokens;
+  p->seq_lens = c->seq_lens;
+  p->lk_row = L->lk_row;
+  p->lv_row = L->lv_row;
+  p->lksz_row = L->lksz_row;
+  p->lvsz_row = L->lvsz_row;
+  p->lk = (const uint8_t*)c->lk_codes;
+  p->lksz = (const __half*)c->lk_sz;
+  p->lv = (const uint8_t*)c->lv_codes;
+  p->lvsz = (const __half*)c->lv_sz;
+  p->rkc = (const uint8_t*)c->rk_codes;
+  p->rks = (const __half*)c->rk_scale;
+  p->rvc = (const uint8_t*)c->rv_codes;
+  p->rvs = (const __half*)c->rv_scale;
+  p->kd = (const __nv_bfloat16*)c->k_dense;
+  p->vd = (const __nv_bfloat16*)c->v_dense;
+  p->bk = (const __half*)c->bk;
+  p->bv = (const __half*)c->bv;
+  p->signs_k = c->signs_k;
+  p->signs_v = c->signs_v;
+  p->page_table = c->page_table;
+  p->off_k = c->offset_k;
+  p->off_v = c->offset_v;
+  p->rank_k = c->rank_k;
+  p->rank_v = c->rank_v;
+  p->stream_bytes = d.kind == KVC_VARRATE ? L->sizes[KVC_BUF_LK_CODES] / d.batch : 0;
+  p->scale = L->scale;
+  p->scale_log2 = L->scale * 1.4426950408889634f;
+  p->qdim = L->qdim;
+  p->vdim = L->vdim;
+  if (d.rope) {
+    for (int i = 0; i < d.head_dim / 2; ++i)
+      p->rope_f[i] = pow(d.rope_theta, -2.0 * i / d.head_dim) / (2.0 * M_PI);
+  }
+  // required buffers, by kind
+  struct Need { const void* ptr; const char* name; };
+  Need need[24];
+  int nn = 0;
+  switch (d.kind) {
+    case KVC_LOWRANK:
+      need[nn++] = {c->lk_codes, "lk_codes"};
+      need[nn++] = {c->lv_codes, "lv_codes"};
+      need[nn++] = {c->bk, "bk"};
+      need[nn++] = {c->bv, "bv"};
+      if (d.latent_bits == 4) {
+        need[nn++] = {c->lk_sz, "lk_sz"};
+        need[nn++] = {c->lv_sz, "lv_sz"};
+      }
+      if (d.resid_bits) {
+        need[nn++] = {c->rk_codes, "rk_codes"};
+        need[nn++] = {c->rv_codes, "rv_codes"};
+        need[nn++] = {c->rk_scale, "rk_scale"};
+        need[nn++] = {c->rv_scale, "rv_scale"};
+        need[nn++] = {c->signs_k, "signs_k"};
+        need[nn++] = {c->signs_v, "signs_v"};
+      }
+      if (d.page_size) need[nn++] = {c->page_table, "page_table"};
+      break;
+    case KVC_VARRATE:
+      need[nn++] = {c->lk_codes, "lk_codes"};
+      need[nn++] = {c->lv_codes, "lv_codes"};
+      need[nn++] = {c->offset_k, "offset_k"};
+      need[nn++] = {c->offset_v, "offset_v"};
+      need[nn++] = {c->rank_k, "rank_k"};
+      need[nn++] = {c->rank_v, "rank_v"};
+      need[nn++] = {c->bk, "bk"};
+      need[nn++] = {c->bv, "bv"};
+      break;
+    case KVC_BLOCK_SHARED:
+      need[nn++] = {c->lk_codes, "lk_codes"};
+      need[nn++] = {c->lk_sz, "lk_sz"};
+      need[nn++] = {c->bk, "bk (W_k)"};
+      need[nn++] = {c->bv, "bv (W_v)"};
+      break;
+    case KVC_DENSE_BF16:
+      need[nn++] = {c->k_dense, "k_dense"};
+      need[nn++] = {c->v_dense, "v_dense"};
+      break;
+  }
+  for (int i = 0; i < nn; ++i) {
+    if (!need[i].ptr) return fail(KVC_EINVAL, "cache.%s is NULL", need[i].name);
+    if (!aligned16(need[i].ptr))
+      return fail(KVC_EALIGN, "cache.%s is not 16-byte aligned", need[i].name);
+  }
+  if (c->seq_lens && !aligned16(c->seq_lens))
+    return fail(KVC_EALIGN, "cache.seq_lens is not 16-byte aligned");
+  return KVC_OK;
+}
+
+static kvc_status launch_status(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(KVC_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+  return KVC_OK;
+}
+
+extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache* c,
+                                            const void* q, void* out, void* workspace,
+                                            size_t ws_size, void* stream, void* ev_begin,
+                                            void* ev_end) {
+  if (!L || !c || !q || !out) return fail(KVC_EINVAL, "kvc_decode_attn: NULL argument");
+  if (c->n_tokens < 0) return fail(KVC_EINVAL, "n_tokens %d < 0", c->n_tokens);
+  if (c->n_tokens > L->d.max_tokens)
+    return fail(KVC_ECAPACITY, "n_tokens %d > max_tokens %d", c->n_tokens, L->d.max_tokens);
+  if (!aligned16(q) || !aligned16(out))
+    return fail(KVC_EALIGN, "q / out must be 16-byte aligned");
+  const size_t need = ws_bytes(L, c->n_tokens);
+  if (!workspace || ws_size < need)
+    return fail(KVC_EWORKSPACE, "workspace %zu bytes < %zu needed", ws_size, need);
+  if (!aligned16(workspace)) return fail(KVC_EALIGN, "workspace must be 16-byte aligned");
+  kvc::Params p;
+  kvc_status st = fill_params(L, c, &p);
+  if (st != KVC_OK) return st;
+  p.q = (const __nv_bfloat16*)q;
+  p.out = out;
+  p.out_bf16 = L->d.out_bf16;
+  plan(L, c->n_tokens, &p.S, &p.split_len);
+  const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
+  char* ws = (char*)workspace;
+  p.qt = (float*)ws;
+  p.part = (float*)(ws + round_up(rows * L->qdim * sizeof(float), 256));
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaGetLastError();  // clear a stale error so it is not reported as ours
+  if (kvc::needs_qproj(p)) {
+    st = launch_status(kvc::launch_qproj(p, s), "qproj launch");
+    if (st != KVC_OK) return st;
+  }
+  if (ev_begin) cudaEventRecord((cudaEvent_t)ev_begin, s);
+  st = launch_status(kvc::launch_split(p, s), "split-T decode launch");
+  if (st != KVC_OK) return st;
+  if (ev_end) cudaEventRecord((cudaEvent_t)ev_end, s);
+  st = launch_status(kvc::launch_combine(p, s), "combine launch");
+  if (st != KVC_OK) return st;
+  return ok();
+}
+
+extern "C" kvc_status kvc_decode_attn(const kvc_layout* L, const kvc_cache* c, const void* q,
+                                      void* out, void* workspace, size_t ws_size,
+                                      void* stream) {
+  return kvc_decode_attn_timed(L, c, q, out, workspace, ws_size, stream, nullptr, nullptr);
+}
+
+extern "C" kvc_status kvc_append(const kvc_layout* L, const kvc_cache* c, const void* k_new,
+                                 const void* v_new, const int32_t* pos, int32_t n_new,
+                                 const uint8_t* new_ranks, void* stream) {
+  if (!L || !c || !pos) return fail(KVC_EINVAL, "kvc_append: NULL argument");
+  const kvc_layout_desc& d = L->d;
+  if (n_new < 1) return fail(KVC_EINVAL, "n_new %d < 1", n_new);
+  if (!k_new || (d.kind != KVC_BLOCK_SHARED && !v_new))
+    return fail(KVC_EINVAL, "kvc_append: k_new / v_new is NULL");
+  if (!aligned16(k_new) || (v_new && !aligned16(v_new)))
+    return fail(KVC_EALIGN, "k_new / v_new must be 16-byte aligned");
+  for (int b = 0; b < d.batch; ++b) {
+    if (pos[b] < 0 || (int64_t)pos[b] + n_new > d.max_tokens)
+      return fail(KVC_ECAPACITY, "row %d: slots %d..%d beyond max_tokens %d", b, pos[b],
+                  pos[b] + n_new - 1, d.max_tokens);
+  }
+  if (d.kind == KVC_VARRATE) {
+    if (!new_ranks) return fail(KVC_EINVAL, "VARRATE append needs new_ranks");
+    for (int64_t i = 0; i < 2LL * d.batch * n_new; ++i) {
+      const int r = new_ranks[i];
+      if (r != 4 && r != 8 && r != 16 && r != 32 && r != 64)
+        return fail(KVC_EINVAL, "rank %d not in {4, 8, 16, 32, 64}", r);
+    }
+  }
+  kvc::AppendParams* a = new (std::nothrow) kvc::AppendParams();
+  if (!a) return fail(KVC_EINVAL, "out of host memory");
+  kvc_status st = fill_params(L, c, &a->p);
+  if (d.kind == KVC_VARRATE && st == KVC_OK && (!c->offset_k || !c->offset_v))
+    st = fail(KVC_EINVAL, "cache offsets are NULL");
+  if (st != KVC_OK) {
+    delete a;
+    return st;
+  }
+  a->k_new = (const __nv_bfloat16*)k_new;
+  a->v_new = (const __nv_bfloat16*)v_new;
+  a->n_new = n_new;
+  for (int b = 0; b < d.batch; ++b) a->pos[b] = pos[b];
+  a->lk_w = (uint8_t*)c->lk_codes;
+  a->lksz_w = (__half*)c->lk_sz;
+  a->lv_w = (uint8_t*)c->lv_codes;
+  a->lvsz_w = (__half*)c->lv_sz;
+  a->rkc_w = (uint8_t*)c->rk_codes;
+  a->rks_w = (__half*)c->rk_scale;
+  a->rvc_w = (uint8_t*)c->rv_codes;
+  a->rvs_w = (__half*)c->rv_scale;
+  a->kd_w = (__nv_bfloat16*)c->k_dense;
+  a->vd_w = (__nv_bfloat16*)c->v_dense;
+  a->off_k_w = c->offset_k;
+  a->off_v_w = c->offset_v;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaGetLastError();
+  if (d.kind == KVC_VARRATE) {
+    for (int comp = 0; comp < 2 && st == KVC_OK; ++comp) {
+      uint8_t* dst = comp == 0 ? c->rank_k : c->rank_v;
+      for (int b = 0; b < d.batch && st == KVC_OK; ++b) {
+        cudaError_t e = cudaMemcpyAsync(dst + (size_t)b * d.max_tokens + pos[b],
+                                        new_ranks + ((size_t)comp * d.batch + b) * n_new,
+                                        n_new, cudaMemcpyHostToDevice, s);
+        st = launch_status(e, "rank copy");
+      }
+    }
+  }
+  if (st == KVC_OK) st = launch_status(kvc::launch_append(*a, s), "append launch");
+  delete a;
+  if (st != KVC_OK) return st;
+  return ok();
+}

@@ -1,0 +1,73 @@
+// Device helpers shared by the kernels of libkvc.
+#pragma once
+
+#include "kvc_internal.h"
+
+namespace kvc {
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float h2f(__half x) { return __half2float(x); }
+
+// Tokens attended by batch row b: seq_lens[b] clamped to [0, n_tokens].
+__device__ __forceinline__ int row_len(const Params& p, int b) {
+  int n = p.n_tokens;
+  if (p.seq_lens) {
+    int s = p.seq_lens[b];
+    n = s < 0 ? 0 : (s < n ? s : n);
+  }
+  return n;
+}
+
+// Row index of (batch row b, KV head h, token t) in a low-rank component.
+__device__ __forceinline__ int64_t lowrank_row(const Params& p, int b, int h, int t) {
+  if (p.page) {
+    const int pp = p.page_table[(int64_t)b * (p.tmax / p.page) + t / p.page];
+    return ((int64_t)pp * p.Hkv + h) * p.page + (t % p.page);
+  }
+  return ((int64_t)b * p.Hkv + h) * p.tmax + t;
+}
+
+// INT4 element r of a row: element 2i in the low nibble of byte i.
+__device__ __forceinline__ int int4_at(const uint8_t* row, int r) {
+  const int byte = row[r >> 1];
+  return (r & 1) ? (byte >> 4) : (byte & 15);
+}
+
+// 2-bit element i of a row: element 4j+k in bits 2k..2k+1 of byte j.
+__device__ __forceinline__ int int2_at(const uint8_t* row, int i) {
+  return (row[i >> 2] >> (2 * (i & 3))) & 3;
+}
+
+// Bytes of one VARRATE record per KV head at rank r.
+__device__ __forceinline__ int varrate_head_bytes(int r) { return r / 2 + 4 * ((r + 31) / 32); }
+
+// In-place unnormalised Walsh-Hadamard transform (Sylvester order) of n
+// values in shared memory, computed by nthreads cooperating threads.
+// Butterflies (a, b) -> (a + b, a - b) over blocks of doubling size give H x.
+__device__ __forceinline__ void fwht_smem(float* x, int n, int tid, int nthreads) {
+  for (int len = 1; len < n; len <<= 1) {
+    __syncthreads();
+    for (int k = tid; k < n / 2; k += nthreads) {
+      const int blk = k / len, off = k % len;
+      const int i = blk * 2 * len + off, j = i + len;
+      const float a = x[i], b = x[j];
+      x[i] = a + b;
+      x[j] = a - b;
+    }
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace kvc

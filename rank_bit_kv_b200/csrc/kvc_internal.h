@@ -1,0 +1,108 @@
+// Internal declarations shared by the host layer and the kernels of libkvc.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kvc.h"
+
+namespace kvc {
+
+constexpr int kMaxBatch = 256;
+constexpr int kNumSMs = 148;          // B200
+constexpr int kResidDim = 128;        // rotated-residual width (Hadamard size)
+
+// Everything a kernel needs about the layout, the cache and the call, passed
+// by value (kernel parameter space).  Pointers are device pointers.
+struct Params {
+  // shape
+  int kind, B, Hq, Hkv, G, d, L;
+  int rk, rv, bits, g, ngk, ngv;
+  int resid, rope, page, tmax, n_pages;
+  int D;                 // block-shared latent width
+  int n_tokens;
+  const int* seq_lens;
+  // compressed rows (bytes per row of each component)
+  int lk_row, lv_row, lksz_row, lvsz_row;
+  // buffers
+  const uint8_t* lk;     // codes (INT4) / fp16 latent / varrate K stream / block latent
+  const __half* lksz;    // (scale, zero) pairs / block scales
+  const uint8_t* lv;
+  const __half* lvsz;
+  const uint8_t* rkc;
+  const __half* rks;
+  const uint8_t* rvc;
+  const __half* rvs;
+  const __nv_bfloat16* kd;
+  const __nv_bfloat16* vd;
+  const __half* bk;
+  const __half* bv;
+  const int8_t* signs_k;
+  const int8_t* signs_v;
+  const int* page_table;
+  const int* off_k;
+  const int* off_v;
+  const uint8_t* rank_k;
+  const uint8_t* rank_v;
+  size_t stream_bytes;   // varrate stream bytes per batch row
+  // call
+  const __nv_bfloat16* q;
+  void* out;
+  int out_bf16;
+  float scale;           // softmax scale
+  float scale_log2;      // softmax scale * log2(e)
+  // workspace
+  float* qt;             // projected queries [L*B*Hq, qdim]
+  float* part;           // split partials [S, L*B*Hq, vdim + 2]
+  int qdim, vdim;
+  int S, split_len;      // splits per unit, tokens per split (multiple of the tile)
+  // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
+  double rope_f[64];
+};
+
+// Tokens per tile of the split kernel, per layout kind (a split is a whole
+// number of tiles).
+__host__ __device__ inline int split_tile(int kind, int rope) {
+  if (kind == KVC_BLOCK_SHARED) return 16;
+  return 64;
+}
+
+// Queries handled by one CTA of the block-shared split kernel.
+constexpr int kBlockQueries = 32;
+
+// Append-specific parameters.
+struct AppendParams {
+  Params p;
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  int n_new;
+  int pos[kMaxBatch];
+  uint8_t* lk_w;
+  __half* lksz_w;
+  uint8_t* lv_w;
+  __half* lvsz_w;
+  uint8_t* rkc_w;
+  __half* rks_w;
+  uint8_t* rvc_w;
+  __half* rvs_w;
+  __nv_bfloat16* kd_w;
+  __nv_bfloat16* vd_w;
+  int* off_k_w;
+  int* off_v_w;
+};
+
+// kernel launchers (return the cudaGetLastError of the launch)
+cudaError_t launch_qproj(const Params& p, cudaStream_t s);
+cudaError_t launch_split(const Params& p, cudaStream_t s);
+cudaError_t launch_combine(const Params& p, cudaStream_t s);
+cudaError_t launch_append(const AppendParams& a, cudaStream_t s);
+
+// Whether the decode of this layout runs a query projection first.
+__host__ __device__ inline bool needs_qproj(const Params& p) {
+  return p.kind == KVC_VARRATE || p.kind == KVC_BLOCK_SHARED ||
+         (p.kind == KVC_LOWRANK && !p.rope);
+}
+
+}  // namespace kvc

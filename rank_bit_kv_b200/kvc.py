@@ -1,0 +1,232 @@
+"""ctypes binding of libkvc (include/kvc.h): argument marshalling only.
+
+Every step of the decode runs in the library's CUDA kernels; this module only
+builds the C structs, owns device buffers as torch tensors (PyTorch is used
+for device memory and streams) and forwards calls.  There is no fallback: if
+libkvc.so is missing or fails to load, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvc.so")
+
+KVC_DENSE_BF16, KVC_LOWRANK, KVC_BLOCK_SHARED, KVC_VARRATE = 0, 1, 2, 3
+STATUS = {0: "KVC_OK", 1: "KVC_EINVAL", 2: "KVC_EUNSUPPORTED", 3: "KVC_ECAPACITY",
+          4: "KVC_EALIGN", 5: "KVC_EWORKSPACE", 6: "KVC_ECUDA"}
+BUFS = ["lk_codes", "lk_sz", "lv_codes", "lv_sz", "rk_codes", "rk_scale", "rv_codes",
+        "rv_scale", "k_dense", "v_dense", "bk", "bv", "signs_k", "signs_v", "page_table",
+        "offset_k", "offset_v", "rank_k", "rank_v"]
+NBUF = len(BUFS)
+
+
+class LayoutDesc(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in (
+        "kind", "batch", "n_q_heads", "n_kv_heads", "head_dim", "max_tokens", "n_layers",
+        "rank_k", "rank_v", "latent_bits", "group_size", "latent_dim", "rope", "resid_bits",
+        "page_size", "n_pages", "out_bf16")] + [("softmax_scale", C.c_float),
+                                                 ("rope_theta", C.c_double)]
+
+
+class CacheDesc(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in BUFS[:15]] + [
+        ("offset_k", C.c_void_p), ("offset_v", C.c_void_p), ("rank_k", C.c_void_p),
+        ("rank_v", C.c_void_p), ("seq_lens", C.c_void_p), ("n_tokens", C.c_int32),
+        ("_reserved", C.c_int32)]
+
+
+class KvcError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """Load libkvc.so (raises if it is missing: there is no CPU fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run `python -m rank_bit_kv_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        vp, i32, sz = C.c_void_p, C.c_int32, C.c_size_t
+        L.kvc_create_layout.argtypes = [C.POINTER(LayoutDesc), C.POINTER(vp)]
+        L.kvc_create_layout.restype = C.c_int
+        L.kvc_destroy_layout.argtypes = [vp]
+        L.kvc_destroy_layout.restype = None
+        L.kvc_buffer_sizes.argtypes = [vp, C.POINTER(sz)]
+        L.kvc_buffer_sizes.restype = C.c_int
+        L.kvc_step_bytes.argtypes = [vp, i32]
+        L.kvc_step_bytes.restype = sz
+        L.kvc_workspace_bytes.argtypes = [vp, i32]
+        L.kvc_workspace_bytes.restype = sz
+        L.kvc_decode_launches.argtypes = [vp, i32]
+        L.kvc_decode_launches.restype = i32
+        L.kvc_append.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, C.POINTER(i32), i32,
+                                 C.POINTER(C.c_uint8), vp]
+        L.kvc_append.restype = C.c_int
+        L.kvc_decode_attn.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, vp, sz, vp]
+        L.kvc_decode_attn.restype = C.c_int
+        L.kvc_decode_attn_timed.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, vp, sz, vp, vp, vp]
+        L.kvc_decode_attn_timed.restype = C.c_int
+        L.kvc_last_error.argtypes = []
+        L.kvc_last_error.restype = C.c_char_p
+        L.kvc_version.argtypes = []
+        L.kvc_version.restype = C.c_char_p
+        _lib = L
+    return _lib
+
+
+def check(status):
+    if status != 0:
+        raise KvcError(status, lib().kvc_last_error().decode())
+
+
+def make_desc(kind, **kw):
+    d = LayoutDesc()
+    d.kind = {"dense": KVC_DENSE_BF16, "lowrank": KVC_LOWRANK, "block_shared": KVC_BLOCK_SHARED,
+              "varrate": KVC_VARRATE}.get(kind, kind)
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def desc_from_config(c, capacity=None, out_bf16=0):
+    """Layout description for a synthetic-workload config dict (see synth.CONFIGS)."""
+    cap = capacity or c["T"]
+    kind = c["kind"]
+    if kind == "lowrank":
+        P = c["page"]
+        if P:
+            cap = -(-cap // P) * P
+        return make_desc("lowrank", batch=c["B"], n_q_heads=c["Hq"], n_kv_heads=c["Hkv"],
+                         head_dim=c["d"], max_tokens=cap, rank_k=c["rk"], rank_v=c["rv"],
+                         latent_bits=c["bits"], group_size=c["g"], rope=c.get("rope", 0),
+                         rope_theta=c.get("theta", 0.0), resid_bits=c["resid"], page_size=P,
+                         n_pages=(c["B"] * cap // P) if P else 0, out_bf16=out_bf16)
+    if kind == "varrate":
+        return make_desc("varrate", batch=c["B"], n_q_heads=c["Hq"], n_kv_heads=c["Hkv"],
+                         head_dim=c["d"], max_tokens=cap, rank_k=64, rank_v=64, latent_bits=4,
+                         group_size=32, out_bf16=out_bf16)
+    if kind == "block_shared":
+        return make_desc("block_shared", batch=c["B"], n_q_heads=c["Hq"], n_kv_heads=c["Hkv"],
+                         head_dim=c["d"], max_tokens=cap, n_layers=c["L"], latent_dim=c["D"],
+                         group_size=c["g"], out_bf16=out_bf16)
+    if kind == "dense":
+        return make_desc("dense", batch=c["B"], n_q_heads=c["Hq"], n_kv_heads=c["Hkv"],
+                         head_dim=c["d"], max_tokens=cap, n_layers=c.get("L", 1),
+                         out_bf16=out_bf16)
+    raise ValueError(kind)
+
+
+class Layout:
+    """Owns a kvc_layout handle."""
+
+    def __init__(self, desc: LayoutDesc):
+        h = C.c_void_p()
+        check(lib().kvc_create_layout(C.byref(desc), C.byref(h)))
+        self.h = h
+        self.desc = desc
+
+    def __del__(self):
+        if getattr(self, "h", None) and _lib is not None:
+            _lib.kvc_destroy_layout(self.h)
+            self.h = None
+
+    def buffer_sizes(self):
+        arr = (C.c_size_t * NBUF)()
+        check(lib().kvc_buffer_sizes(self.h, arr))
+        return dict(zip(BUFS, list(arr)))
+
+    def workspace_bytes(self, n_tokens):
+        return int(lib().kvc_workspace_bytes(self.h, n_tokens))
+
+    def step_bytes(self, n_tokens):
+        return int(lib().kvc_step_bytes(self.h, n_tokens))
+
+    def decode_launches(self, n_tokens):
+        return int(lib().kvc_decode_launches(self.h, n_tokens))
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+class Cache:
+    """Device buffers of a cache (torch uint8 tensors sized by kvc_buffer_sizes)."""
+
+    def __init__(self, layout: Layout, device="cuda", fill=None):
+        import torch
+
+        self.layout = layout
+        self.bufs = {}
+        for name, nbytes in layout.buffer_sizes().items():
+            if nbytes:
+                self.bufs[name] = torch.zeros(int(nbytes), dtype=torch.uint8, device=device)
+        self.n_tokens = 0
+        self.seq_lens = None
+        if fill:
+            self.upload(fill)
+
+    def upload(self, arrays):
+        """Copy numpy arrays (storage layout) into the matching buffers."""
+        import torch
+
+        for name, t in self.bufs.items():
+            key = {"lk_codes": ("lk_codes", "kstream"), "lv_codes": ("lv_codes", "vstream"),
+                   "bk": ("bk", "wk"), "bv": ("bv", "wv")}.get(name, (name,))
+            a = next((arrays[k] for k in key if k in arrays), None)
+            if a is None:
+                continue
+            raw = np.ascontiguousarray(a).view(np.uint8).reshape(-1)
+            if raw.size > t.numel():
+                raise ValueError(f"{name}: {raw.size} bytes > buffer {t.numel()}")
+            t[: raw.size].copy_(torch.from_numpy(raw.copy()))
+
+    def struct(self):
+        c = CacheDesc()
+        for name, t in self.bufs.items():
+            setattr(c, name, t.data_ptr())
+        c.seq_lens = None if self.seq_lens is None else self.seq_lens.data_ptr()
+        c.n_tokens = int(self.n_tokens)
+        return c
+
+
+def current_stream_ptr():
+    import torch
+
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def decode(layout: Layout, cache: Cache, q, out, ws, stream=None, events=None):
+    """kvc_decode_attn on torch tensors (q bf16, out fp32/bf16, ws uint8)."""
+    cs = cache.struct()
+    st = stream if stream is not None else current_stream_ptr()
+    if events is None:
+        check(lib().kvc_decode_attn(layout.h, C.byref(cs), _ptr(q), _ptr(out), _ptr(ws),
+                                    ws.numel(), st))
+    else:
+        check(lib().kvc_decode_attn_timed(layout.h, C.byref(cs), _ptr(q), _ptr(out), _ptr(ws),
+                                          ws.numel(), st, C.c_void_p(events[0].cuda_event),
+                                          C.c_void_p(events[1].cuda_event)))
+
+
+def append(layout: Layout, cache: Cache, k_new, v_new, pos, n_new, new_ranks=None,
+           stream=None):
+    """kvc_append: k_new / v_new torch bf16 device tensors, pos host ints [B]."""
+    cs = cache.struct()
+    posa = (C.c_int32 * len(pos))(*[int(x) for x in pos])
+    rk = None
+    if new_ranks is not None:
+        nr = np.ascontiguousarray(np.asarray(new_ranks, dtype=np.uint8))
+        rk = nr.ctypes.data_as(C.POINTER(C.c_uint8))
+    st = stream if stream is not None else current_stream_ptr()
+    check(lib().kvc_append(layout.h, C.byref(cs), _ptr(k_new), _ptr(v_new), posa, int(n_new),
+                           rk, st))

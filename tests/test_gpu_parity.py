@@ -1,0 +1,204 @@
+"""GPU decode parity: the CUDA path through the C ABI against the fp64 oracle on
+identical seeded integer codes.  Small cases compare every output; the
+full-size workloads (the launch configuration the benchmark times) compare
+sampled rows that the oracle recomputes on their own."""
+
+import numpy as np
+import pytest
+
+from oracle import kvc_oracle as O
+from rank_bit_kv_b200 import synth
+from tests.gpu_util import assert_close, run_decode
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle(cfg, arrays, n):
+    return O.decode_from_storage(cfg, arrays, n)
+
+
+def sub_batch(arrays, rows, keys):
+    out = dict(arrays)
+    for k in keys:
+        if k in out:
+            out[k] = arrays[k][rows]
+    return out
+
+
+# ------------------------------------------------------------------ tiny / small
+
+
+@pytest.mark.parametrize("T", [1, 100, 512])
+def test_c1_tiny_single_head(T):
+    c = synth.config("c1")
+    a = synth.lowrank_cache(c)                  # 512 slots, attend to the first T
+    got = run_decode(c, a, T, capacity=512)
+    assert_close(got, oracle(c, a, T), what=f"c1 T={T}")
+
+
+@pytest.mark.parametrize("rope", [0, 1])
+@pytest.mark.parametrize("T", [1000, 4161])
+def test_c2_shape_small_context(rope, T):
+    c = synth.config("c2", B=2, T=T, rope=rope)
+    a = synth.lowrank_cache(c)
+    got = run_decode(c, a, T)
+    assert_close(got, oracle(c, a, T), what=f"c2 rope={rope} T={T}")
+
+
+def test_c2_quantized_gaussian_latents():
+    """Codes produced from N(0,1) latents by the reference quantizer."""
+    c = synth.config("c2", B=1, T=777)
+    a = synth.lowrank_cache(c)
+    lk, lv = synth.gaussian_latents(c, 777)
+    for name, lat in (("lk", lk), ("lv", lv)):
+        codes, s, z = O.quantize_int4_asym(lat, 32)
+        a[f"{name}_codes"] = O.pack_int4(codes)
+        a[f"{name}_sz"] = np.stack([s, z], -1).astype(np.float16)
+    assert_close(run_decode(c, a, 777), oracle(c, a, 777), what="c2 gaussian")
+
+
+@pytest.mark.parametrize("mode", ["q_x8", "needle"])
+def test_c2_peaked_softmax(mode):
+    """The configured scores are nearly uniform; these keep the shapes but
+    make the softmax peaked (q scaled by 8, or one planted needle token)."""
+    c = synth.config("c2", B=2, T=2048, rope=0)
+    a = synth.lowrank_cache(c)
+    if mode == "q_x8":
+        a["q"] = synth.to_bf16_bits(synth.bf16_bits_to_f32(a["q"]) * 8)
+    else:
+        q = O.bf16_bits_to_f64(a["q"])
+        bk = a["bk"].astype(np.float64)
+        for b in range(c["B"]):
+            for h in range(c["Hkv"]):
+                qt = bk[h] @ q[b, h * 4]                       # first head of the group
+                lat = 3 * np.sqrt(32) * qt / np.linalg.norm(qt)
+                codes, s_, z_ = O.quantize_int4_asym(lat[None], 32)
+                a["lk_codes"][b, h, 1234] = O.pack_int4(codes)[0]
+                a["lk_sz"][b, h, 1234] = np.stack([s_, z_], -1).astype(np.float16)[0]
+    ref = oracle(c, a, 2048)
+    assert_close(run_decode(c, a, 2048), ref, what=mode)
+
+
+@pytest.mark.parametrize("rope", [0, 1])
+def test_c5_shape_small_paged_residual(rope):
+    c = synth.config("c5", B=2, T=400, rope=rope, theta=500000.0)
+    a = synth.lowrank_cache(c)
+    assert_close(run_decode(c, a, 400), oracle(c, a, 400), what=f"c5 rope={rope}")
+    assert_close(run_decode(c, a, 333), oracle(c, a, 333), what="c5 ragged")
+
+
+def test_paging_shuffled_equals_identity_table():
+    c = synth.config("c5", B=2, T=256)
+    a = synth.lowrank_cache(c)
+    ident = dict(a)
+    perm = a["page_table"].reshape(-1)
+    comps = ("lk_codes", "lk_sz", "lv_codes", "lv_sz", "rk_codes", "rk_scale", "rv_codes",
+             "rv_scale")
+    for k in comps:
+        ident[k] = a[k][perm]            # logical page j now stored at physical j
+    ident["page_table"] = np.arange(perm.size, dtype=np.int32).reshape(a["page_table"].shape)
+    g1 = run_decode(c, a, 256)
+    g2 = run_decode(c, ident, 256)
+    np.testing.assert_allclose(g1, g2, rtol=0, atol=1e-6)
+
+
+@pytest.mark.parametrize("T", [1, 300, 2000])
+def test_c4_shape_small_varrate(T):
+    c = synth.config("c4", T=T)
+    a = synth.varrate_cache(c)
+    assert_close(run_decode(c, a, T), oracle(c, a, T), what=f"c4 T={T}")
+
+
+def test_c3_shape_small_block_shared():
+    c = synth.config("c3", B=2, T=300)
+    a = synth.block_shared_cache(c)
+    assert_close(run_decode(c, a, 300), oracle(c, a, 300), what="c3 small")
+
+
+def test_dense_bf16_small():
+    cfg = dict(kind="dense", B=2, Hq=32, Hkv=8, d=128, T=700)
+    a = synth.dense_cache(2, 32, 8, 128, 700, seed=5)
+    assert_close(run_decode(cfg, a, 700), oracle(cfg, a, 700), what="dense")
+
+
+def test_dense_layered():
+    cfg = dict(kind="dense", B=1, Hq=8, Hkv=2, d=128, T=129, L=2)
+    a = synth.dense_cache(1, 8, 2, 128, 129, seed=6, n_layers=2)
+    assert_close(run_decode(cfg, a, 129), oracle(cfg, a, 129), what="dense layered")
+
+
+# ------------------------------------------------------------------ edge cases
+
+
+def test_empty_context_gives_zero():
+    c = synth.config("c2", B=2, T=64)
+    a = synth.lowrank_cache(c)
+    got = run_decode(c, a, 0, capacity=64)
+    assert (got == 0).all()
+
+
+def test_per_row_lengths():
+    c = synth.config("c2", B=3, T=900)
+    a = synth.lowrank_cache(c)
+    lens = [900, 0, 257]
+    got = run_decode(c, a, 900, seq_lens=lens)
+    for b, n in enumerate(lens):
+        sub = sub_batch(a, [b], ("q", "lk_codes", "lk_sz", "lv_codes", "lv_sz"))
+        cb = dict(c, B=1)
+        if n == 0:
+            assert (got[b] == 0).all()
+        else:
+            assert_close(got[b:b + 1], oracle(cb, sub, n), what=f"row {b} len {n}")
+
+
+def test_bf16_output():
+    c = synth.config("c2", B=1, T=500)
+    a = synth.lowrank_cache(c)
+    got = run_decode(c, a, 500, out_bf16=1)
+    ref = oracle(c, a, 500)
+    # bf16 output rounding adds up to 2^-9 relative per element
+    assert_close(got, ref, max_abs=1e-2, rel_l2=5e-3, what="bf16 out")
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+
+def test_c2_full_size_sampled():
+    c = synth.config("c2")
+    a = synth.lowrank_cache(c)
+    got = run_decode(c, a, c["T"])
+    for b in (0, 5):
+        sub = sub_batch(a, [b], ("q", "lk_codes", "lk_sz", "lv_codes", "lv_sz"))
+        assert_close(got[b:b + 1], oracle(dict(c, B=1), sub, c["T"]), what=f"c2 full b={b}")
+
+
+def test_c5_full_size_sampled():
+    c = synth.config("c5")
+    a = synth.lowrank_cache(c)
+    got = run_decode(c, a, c["T"])
+    for b in (3,):
+        sub = dict(a)
+        sub["q"] = a["q"][[b]]
+        sub["page_table"] = a["page_table"][[b]]
+        assert_close(got[b:b + 1], oracle(dict(c, B=1), sub, c["T"]), what=f"c5 full b={b}")
+
+
+def test_c4_full_size():
+    c = synth.config("c4")
+    a = synth.varrate_cache(c)
+    assert_close(run_decode(c, a, c["T"]), oracle(c, a, c["T"]), what="c4 full")
+
+
+def test_c3_full_size_sampled():
+    c = synth.config("c3")
+    a = synth.block_shared_cache(c)
+    got = run_decode(c, a, c["T"])
+    T, d = c["T"], c["d"]
+    codes = O.unpack_int4(a["lk_codes"][[1], :T], c["D"])
+    lat = O.dequant_int4_sym(codes, a["lk_sz"][[1], :T].astype(np.float64), c["g"])
+    for kvh in (0, 7):
+        sl = slice(kvh * d, (kvh + 1) * d)
+        q = O.bf16_bits_to_f64(a["q"][:, [1], kvh * 4:(kvh + 1) * 4])     # [L, 1, 4, d]
+        ref = O.decode_block_shared(q, lat, a["wk"][:, :, sl].astype(np.float64),
+                                    a["wv"][:, :, sl].astype(np.float64), 1, 1 / np.sqrt(d))
+        assert_close(got[:, 1:2, kvh * 4:(kvh + 1) * 4], ref, what=f"c3 full kvh={kvh}")
