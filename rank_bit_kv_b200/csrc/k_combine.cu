@@ -31,12 +31,20 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
   const int pst = p.vdim + 2;
   const float* part = p.part + (size_t)row * pst;
 
+  // partial slots of this row: all S splits, or the CTA ranges of the
+  // persistent partition that cover this row's unit
+  int nS = p.S;
+  if (p.seg_W > 0) {
+    const int u = (row / p.Hq) * p.Hkv + kvh;   // L == 1 on this path
+    const long long a = (long long)u * p.seg_tpu, e = (long long)(u + 1) * p.seg_tpu - 1;
+    nS = (int)(e / p.seg_W - a / p.seg_W + 1);
+  }
   if (tid < 32) {
     float mx = -INFINITY;
-    for (int s = tid; s < p.S; s += 32) mx = fmaxf(mx, part[(size_t)s * rows * pst + p.vdim]);
+    for (int s = tid; s < nS; s += 32) mx = fmaxf(mx, part[(size_t)s * rows * pst + p.vdim]);
     mx = warp_max(mx);
     float lt = 0.f;
-    for (int s = tid; s < p.S; s += 32) {
+    for (int s = tid; s < nS; s += 32) {
       const float* ps = part + (size_t)s * rows * pst;
       const float w = (mx == -INFINITY) ? 0.f : exp2f(ps[p.vdim] - mx);
       ws[s] = w;
@@ -48,7 +56,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
   __syncthreads();
   for (int j = tid; j < p.vdim; j += kThreads) {
     float a = 0.f;
-    for (int s = 0; s < p.S; ++s) a = fmaf(ws[s], part[(size_t)s * rows * pst + j], a);
+    for (int s = 0; s < nS; ++s) a = fmaf(ws[s], part[(size_t)s * rows * pst + j], a);
     acc[j] = a;
   }
   __syncthreads();

@@ -62,11 +62,26 @@ void plan(const kvc_layout* L, int n_tokens, int* S, int* split_len) {
   *S = ceil_div(tiles, per);
 }
 
+// Workspace: a 256-byte header (error word), the projected queries, then the
+// split partials; sized for the larger of the two split plans.
+constexpr size_t kWsHeader = 256;
+
+int fast_slots(const kvc_layout* L, int n_tokens) {
+  if (n_tokens <= 0) return 1;
+  const int tpu = ceil_div(n_tokens, 128);
+  const int total = L->d.batch * L->d.n_kv_heads * tpu;
+  int g = total < kvc::kNumSMs ? total : kvc::kNumSMs;
+  const int w = ceil_div(total, g);
+  return ceil_div(tpu, w) + 1;
+}
+
 size_t ws_bytes(const kvc_layout* L, int n_tokens) {
   int S, len;
   plan(L, n_tokens, &S, &len);
+  const int Sf = fast_slots(L, n_tokens);
+  if (Sf > S) S = Sf;
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
-  size_t b = round_up(rows * L->qdim * sizeof(float), 256);
+  size_t b = kWsHeader + round_up(rows * L->qdim * sizeof(float), 256);
   b += round_up((size_t)S * rows * (L->vdim + 2) * sizeof(float), 256);
   return b;
 }
@@ -415,10 +430,18 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
   p.out = out;
   p.out_bf16 = L->d.out_bf16;
   plan(L, c->n_tokens, &p.S, &p.split_len);
+  if (kvc::rope_tc_supported(p)) {
+    int grid, W, tpu, slots;
+    kvc::rope_tc_plan(p, &grid, &W, &tpu, &slots);
+    p.S = slots;
+    p.seg_W = W;
+    p.seg_tpu = tpu;
+  }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   char* ws = (char*)workspace;
-  p.qt = (float*)ws;
-  p.part = (float*)(ws + round_up(rows * L->qdim * sizeof(float), 256));
+  p.err = (uint32_t*)ws;
+  p.qt = (float*)(ws + kWsHeader);
+  p.part = (float*)(ws + kWsHeader + round_up(rows * L->qdim * sizeof(float), 256));
   cudaStream_t s = (cudaStream_t)stream;
   cudaGetLastError();  // clear a stale error so it is not reported as ours
   if (kvc::needs_qproj(p)) {

@@ -58,6 +58,10 @@ struct Params {
   float* part;           // split partials [S, L*B*Hq, vdim + 2]
   int qdim, vdim;
   int S, split_len;      // splits per unit, tokens per split (multiple of the tile)
+  // persistent tensor-core path: contiguous ranges of seg_W tiles per CTA over
+  // units of seg_tpu tiles (0 = split partials indexed by split)
+  int seg_W, seg_tpu;
+  uint32_t* err;         // error word of the workspace (bounded waits that gave up)
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
   double rope_f[64];
 };
@@ -92,6 +96,11 @@ struct AppendParams {
   int* off_k_w;
   int* off_v_w;
 };
+
+// tensor-core decode of pre-RoPE INT4 low-rank caches
+bool rope_tc_supported(const Params& p);
+void rope_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
+cudaError_t launch_rope_tc(const Params& p, uint32_t* err, cudaStream_t s);
 
 // kernel launchers (return the cudaGetLastError of the launch)
 cudaError_t launch_qproj(const Params& p, cudaStream_t s);

@@ -202,3 +202,35 @@ def test_c3_full_size_sampled():
         ref = O.decode_block_shared(q, lat, a["wk"][:, :, sl].astype(np.float64),
                                     a["wv"][:, :, sl].astype(np.float64), 1, 1 / np.sqrt(d))
         assert_close(got[:, 1:2, kvh * 4:(kvh + 1) * 4], ref, what=f"c3 full kvh={kvh}")
+
+
+# ------------------------------------------------------------------ tensor-core path
+
+
+@pytest.mark.parametrize("B,T", [(1, 1), (2, 127), (2, 128), (1, 129), (2, 3000), (3, 8191)])
+def test_rope_tensor_core_path_against_oracle_and_generic(B, T):
+    """Pre-RoPE INT4 keys run on the tcgen05 kernel; per-row lengths force the
+    generic CUDA-core kernel.  Both must match the oracle, and the tensor-core
+    kernel must report no aborted wait in the workspace error word."""
+    import torch
+
+    from rank_bit_kv_b200 import kvc
+
+    c = synth.config("c2", B=B, T=T)
+    a = synth.lowrank_cache(c)
+    ref = oracle(c, a, T)
+    lay = kvc.Layout(kvc.desc_from_config(c))
+    cache = kvc.Cache(lay, fill=a)
+    cache.n_tokens = T
+    q = torch.from_numpy(a["q"].view(np.int16)).cuda().view(torch.bfloat16)
+    out = torch.empty(q.shape, device="cuda")
+    ws = torch.zeros(lay.workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    kvc.decode(lay, cache, q, out, ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0, "a bounded wait gave up"
+    fast = out.cpu().numpy()
+    assert_close(fast, ref, what=f"tcgen05 B={B} T={T}")
+    cache.seq_lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    kvc.decode(lay, cache, q, out, ws)
+    torch.cuda.synchronize()
+    assert_close(out.cpu().numpy(), ref, what=f"generic B={B} T={T}")
