@@ -31,8 +31,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
   const int pst = p.vdim + 2;
   const float* part = p.part + (size_t)row * pst;
 
-  // partial slots of this row: all S splits, or the CTA ranges of the
-  // persistent partition that cover this row's unit
+  // partial slots of this row: all S splits, or -- on the persistent
+  // tensor-core path -- one partial for every CTA whose tile range covers
+  // this row's unit
   int nS = p.S;
   if (p.seg_W > 0) {
     const int u = (row / p.Hq) * p.Hkv + kvh;   // L == 1 on this path
@@ -48,7 +49,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
       const float* ps = part + (size_t)s * rows * pst;
       const float w = (mx == -INFINITY) ? 0.f : exp2f(ps[p.vdim] - mx);
       ws[s] = w;
-      lt += w * ps[p.vdim + 1];
+      if (w != 0.f) lt += w * ps[p.vdim + 1];
     }
     lt = warp_sum(lt);
     if (tid == 0) lsum = lt;
@@ -56,7 +57,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
   __syncthreads();
   for (int j = tid; j < p.vdim; j += kThreads) {
     float a = 0.f;
-    for (int s = 0; s < nS; ++s) a = fmaf(ws[s], part[(size_t)s * rows * pst + j], a);
+    for (int s = 0; s < nS; ++s)
+      if (ws[s] != 0.f) a = fmaf(ws[s], part[(size_t)s * rows * pst + j], a);
     acc[j] = a;
   }
   __syncthreads();

@@ -9,9 +9,10 @@
 //   1. stages the compressed rows with 1-D bulk copies (no multicast),
 //   2. dequantizes L_k into TMEM (the A operand) and L_v into shared memory,
 //   3. reconstructs K_hat = L_k Bk on the tensor cores (M = 128 tokens,
-//      N = 128 dims, K = rk) into TMEM,
-//   4. applies RoPE as R_t = R_t0 R_delta (delta = row in the tile): each
-//      epilogue thread owns one row, so R_delta is a per-thread constant
+//      N = 128 dims, K = rk) into TMEM (fp32),
+//   4. applies RoPE as R_t = R_t0 R_delta (delta = row in the tile), writing
+//      K'' as packed fp16 back to TMEM (the A operand of the score MMA):
+//      each epilogue thread owns one row, so R_delta is a per-thread constant
 //      rotation, and R_t0 is folded into the queries (q_rot = R_t0^T q, so
 //      q . R_t k = q_rot . R_delta k) -- no per-token sin/cos,
 //   5. scores S = K'' q_rot^T on the tensor cores with K'' read from TMEM,
@@ -26,13 +27,18 @@
 // into equal contiguous ranges, one per CTA, so every SM streams the same
 // number of bytes; a range may cross a unit boundary (two partials).
 //
-// Warp roles (320 threads, one CTA per SM):
-//   warp 0     bulk-copy producer (6-stage ring of compressed tiles)
-//   warp 1     TMEM allocation + MMA issue (one elected lane)
-//   warps 2-5  epilogue: RoPE, scores, softmax, P, partials (thread = row)
-//   warps 6-9  dequantization (thread = row)
-// Every wait is bounded; on a timeout the CTA sets an error bit in the
-// workspace, drains its own bulk copies, frees TMEM and exits.
+// Warp roles (448 threads, one CTA per SM):
+//   warp 0      bulk-copy producer (6-stage ring of compressed tiles)
+//   warp 1      TMEM allocation + MMA issue (one lane, non-blocking scheduler)
+//   warps 2-9   epilogue: two groups of four warps work on the same tile;
+//               group h rotates RoPE pairs 32h..32h+31 and owns query heads
+//               2h, 2h+1 (their scores, softmax state, P columns, partials).
+//               Software-pipelined: RoPE of tile t, then softmax of tile t-1.
+//   warps 10-13 dequantization (thread = row)
+// Buffer rings: compressed stages (6), dequantized operands (4), reconstructed
+// keys and rotated keys in TMEM (2 each), scores (2), P and q_rot (2).  Every wait is bounded; on a
+// timeout the CTA sets an error bit in the workspace, drains its own bulk
+// copies and MMAs, frees TMEM and exits.
 #include <math.h>
 
 #include "kvc_device.cuh"
@@ -45,43 +51,49 @@ using namespace tc;
 
 constexpr int kTile = 128;
 constexpr int kStages = 6;
-constexpr int kThreads = 320;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpEpi = 2, kWarpDeq = 6;
+constexpr int kThreads = 448;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpEpi = 2, kWarpDeq = 10;
 constexpr int kD = 128;            // head dim
 constexpr int kHalf = 64;          // RoPE pairs
 constexpr int kG = 4;              // query heads per KV head
 constexpr int kVM = 64;            // M of the value MMA (rank_v + 1 <= 64)
 constexpr int kN = 16;             // N of score / value MMAs (4 heads padded)
+constexpr int kNB = 4;             // dequantized operand buffers (tile jj uses jj % kNB)
 
-// TMEM columns (512 allocated)
-constexpr uint32_t kColALk = 0;    // 2 x 16  recon A (128 x rk fp16, rk <= 32)
-constexpr uint32_t kColS = 32;     // 2 x 16  scores (fp32)
-constexpr uint32_t kColAcc = 64;   // 16      value accumulator (M = 64 layout)
-constexpr uint32_t kColDr = 128;   // 2 x 128 reconstructed keys (fp32)
-constexpr uint32_t kColAK = 384;   // 2 x 64  rotated keys (fp16, A of the score MMA)
+// TMEM columns (512 allocated); a 16-bit accumulator would still take one
+// column per value, while a TMEM A operand packs two fp16 per column, so the
+// reconstruction stays fp32 and the rotated keys get their own packed buffer
+constexpr uint32_t kColALk = 0;    // kNB x 16   recon A (128 x rk fp16, rk <= 32)
+constexpr uint32_t kColS = 64;     // 2 x 16     scores (fp32)
+constexpr uint32_t kColAcc = 96;   // 16         value accumulator (M = 64 layout)
+constexpr uint32_t kColDr = 128;   // 2 x 128    reconstructed keys K_hat (fp32)
+constexpr uint32_t kColAK = 384;   // 2 x 64     rotated keys K'' (packed fp16)
 constexpr uint32_t kTmemCols = 512;
 
 // Shared memory carve-up (bytes, from a 1024-aligned base)
-constexpr int kSmStage = 0;                           // kStages x stage bytes
+constexpr int kSmStage = 0;                            // kStages x stage bytes
 constexpr int kStageMax = 8192;
-constexpr int kSmBk = kSmStage + kStages * kStageMax;  // 8 KB  B of recon (128 x 32)
-constexpr int kSmQ = kSmBk + 8192;                    // 2 x 4 KB  B of score (16 x 128)
-constexpr int kSmLV = kSmQ + 2 * 4096;                // 2 x 16 KB A of value (64 x 128)
-constexpr int kSmP = kSmLV + 2 * 16384;               // 2 x 4 KB  B of value (128 x 16)
-constexpr int kSmBar = kSmP + 2 * 4096;               // barriers + scratch
+constexpr int kSmBk = kSmStage + kStages * kStageMax;   // 8 KB   B of recon (128 x 32)
+constexpr int kSmQ = kSmBk + 8192;                     // 2 x 4 KB   B of score (16 x 128)
+constexpr int kSmLV = kSmQ + 2 * 4096;                 // kNB x 16 KB A of value (64 x 128)
+constexpr int kSmP = kSmLV + kNB * 16384;              // 2 x 4 KB   B of value (128 x 16)
+constexpr int kSmBar = kSmP + 2 * 4096;                // barriers + scratch
 constexpr int kSmTotal = kSmBar + 1024;
-constexpr int kSmAlloc = 120 * 1024 + 1024;           // forces one CTA per SM
+constexpr int kSmAlloc = kSmTotal + 2048;              // > half the SM: one CTA per SM
 
 struct Bars {
   uint64_t full[kStages], empty[kStages];
-  uint64_t tile_in[2], recon_done[2], kq_full[2], score_done[2], p_full[2], v_done[2];
-  uint64_t acc_free;
-  uint64_t epi_sync;     // bounded barrier among the 128 epilogue threads
-  uint64_t mma_drain;    // last MMAs of the CTA completed
+  uint64_t tile_in[kNB], v_done[kNB];       // per dequantized operand buffer
+  uint64_t alk_free[kNB];                   // recon of the buffer's last tile completed
+  uint64_t recon_done[2], kq_full[2];       // per reconstructed / rotated key buffer
+  uint64_t score_done[2], p_full[2];        // per score / P buffer
+  uint64_t acc_free;                        // the accumulator was read at a unit end
+  uint64_t epi_sync[2];                     // bounded barrier among a group's 128 threads
+  uint64_t mma_drain;                       // last MMAs of the CTA completed
   uint32_t tmem_base;
   int abort;
-  int flag[3];
-  float wmax[4][kG];
+  int flag[2][3];
+  float wmax[2][4][2];
 };
 
 struct Work {
@@ -143,19 +155,22 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 4);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kNB; ++b) {
       mbar_init(&bars.tile_in[b], 4);
-      mbar_init(&bars.recon_done[b], 1);
-      mbar_init(&bars.kq_full[b], 128);
-      mbar_init(&bars.score_done[b], 1);
-      mbar_init(&bars.p_full[b], 128);
       mbar_init(&bars.v_done[b], 1);
+      mbar_init(&bars.alk_free[b], 1);
     }
-    mbar_init(&bars.acc_free, 128);
-    mbar_init(&bars.epi_sync, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.recon_done[b], 1);
+      mbar_init(&bars.kq_full[b], 256);
+      mbar_init(&bars.score_done[b], 1);
+      mbar_init(&bars.p_full[b], 256);
+      mbar_init(&bars.epi_sync[b], 128);
+      for (int k = 0; k < 3; ++k) bars.flag[b][k] = 0;
+    }
+    mbar_init(&bars.acc_free, 256);
     mbar_init(&bars.mma_drain, 1);
     bars.abort = 0;
-    bars.flag[0] = bars.flag[1] = bars.flag[2] = 0;
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
@@ -163,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     tmem_relinquish();
   }
   // static zeros of the operand buffers (padding heads / rows)
-  for (int i = threadIdx.x; i < (2 * 4096 + 2 * 16384 + 2 * 4096) / 16; i += kThreads)
+  for (int i = threadIdx.x; i < (2 * 4096 + kNB * 16384 + 2 * 4096) / 16; i += kThreads)
     reinterpret_cast<uint4*>(sm + kSmQ)[i] = make_uint4(0, 0, 0, 0);
   tc_fence_before();
   __syncthreads();
@@ -180,8 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       unit_of(p, wk, t_first + jj, &u, &jt, &nt);
       const size_t row0 = (size_t)u * p.tmax + (size_t)jt * kTile;
       uint8_t* st = sm + kSmStage + s * kStageMax;
-      const uint8_t* src[4] = {p.lk + row0 * lk_row, reinterpret_cast<const uint8_t*>(p.lksz) + row0 * lksz_row,
-                               p.lv + row0 * lv_row, reinterpret_cast<const uint8_t*>(p.lvsz) + row0 * lvsz_row};
+      const uint8_t* src[4] = {p.lk + row0 * lk_row,
+                               reinterpret_cast<const uint8_t*>(p.lksz) + row0 * lksz_row,
+                               p.lv + row0 * lv_row,
+                               reinterpret_cast<const uint8_t*>(p.lvsz) + row0 * lvsz_row};
       const int rowb[4] = {lk_row, lksz_row, lv_row, lvsz_row};
       // bulk copies need 16-byte aligned sources: a unit base u * max_tokens * row
       // is aligned only when max_tokens * row is a multiple of 16
@@ -219,60 +236,75 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issue
+    // Non-blocking scheduler: issue whichever of (value nv, score ns,
+    // reconstruction nr) is ready, in tile order within each kind.  recon(nr)
+    // overwrites the K_hat buffer of tile nr - 2, which the epilogue has read
+    // once score(nr - 2) could be issued.
     if (lane == 0) {
       const uint32_t id_recon = idesc_f16(kTile, kD, 0, 0);
       const uint32_t id_score = idesc_f16(kTile, kN, 0, 0);
       const uint32_t id_val = idesc_f16(kVM, kN, 1, 1);
       const int ksteps_recon = p.rk / 16;
-      int unit_idx = -1, cur_u = -1;
-      auto recon = [&](int jj) -> bool {
-        const int b = jj & 1;
-        if (!mbar_wait(&bars.tile_in[b], (jj >> 1) & 1, abort, err)) return false;
-        tc_fence_after();
-        for (int kk = 0; kk < ksteps_recon; ++kk)
-          mma_ts(tmem + kColDr + b * 128, tmem + kColALk + b * 16 + kk * 8,
-                 smem_desc(sm + kSmBk + kk * 256, 128, 512), id_recon, kk > 0);
-        tc_commit(&bars.recon_done[b]);
-        return true;
-      };
-      auto score = [&](int jj) -> bool {
-        const int b = jj & 1;
-        if (!mbar_wait(&bars.kq_full[b], (jj >> 1) & 1, abort, err)) return false;
-        tc_fence_after();
-        for (int kk = 0; kk < kD / 16; ++kk)
-          mma_ts(tmem + kColS + b * 16, tmem + kColAK + b * 64 + kk * 8,
-                 smem_desc(sm + kSmQ + b * 4096 + kk * 256, 128, 2048), id_score, kk > 0);
-        tc_commit(&bars.score_done[b]);
-        return true;
-      };
-      auto value = [&](int jj) -> bool {
-        const int b = jj & 1;
-        if (!mbar_wait(&bars.p_full[b], (jj >> 1) & 1, abort, err)) return false;
-        int u, jt, nt;
-        unit_of(p, wk, t_first + jj, &u, &jt, &nt);
-        bool first = false;
-        if (u != cur_u) {
-          first = true;
-          cur_u = u;
-          ++unit_idx;
-          if (unit_idx > 0 && !mbar_wait(&bars.acc_free, (unit_idx - 1) & 1, abort, err))
-            return false;
+      int nr = 0, ns = 0, nv = 0;
+      int v_unit = -1, v_started = 0;
+      uint64_t idle_since = 0;
+      uint32_t idle = 0;
+      while (nv < n_tiles) {
+        bool prog = false;
+        if (nv < ns && mbar_test(&bars.p_full[nv & 1], (nv >> 1) & 1)) {
+          int u, jt, nt;
+          unit_of(p, wk, t_first + nv, &u, &jt, &nt);
+          const bool first = u != v_unit;
+          bool ready = true;
+          if (first && v_started > 0) ready = mbar_test(&bars.acc_free, (v_started - 1) & 1);
+          if (ready) {
+            if (first) v_unit = u, ++v_started;
+            const int bd = nv % kNB, pb = nv & 1;
+            tc_fence_after();
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ss(tmem + kColAcc, smem_desc(sm + kSmLV + bd * 16384 + kk * 256, 128, 2048),
+                     smem_desc(sm + kSmP + pb * 4096 + kk * 256, 128, 2048), id_val,
+                     (first && kk == 0) ? 0u : 1u);
+            tc_commit(&bars.v_done[bd]);
+            ++nv;
+            prog = true;
+          }
         }
-        tc_fence_after();
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ss(tmem + kColAcc, smem_desc(sm + kSmLV + b * 16384 + kk * 256, 128, 2048),
-                 smem_desc(sm + kSmP + b * 4096 + kk * 256, 128, 2048), id_val,
-                 (first && kk == 0) ? 0u : 1u);
-        tc_commit(&bars.v_done[b]);
-        return true;
-      };
-      bool ok = n_tiles > 0 ? recon(0) : true;
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        if (j >= 1) ok = value(j - 1);
-        if (ok && j + 1 < n_tiles) ok = recon(j + 1);
-        if (ok) ok = score(j);
+        if (ns < nr && mbar_test(&bars.kq_full[ns & 1], (ns >> 1) & 1)) {
+          const int sb = ns & 1;
+          tc_fence_after();
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ts(tmem + kColS + sb * 16, tmem + kColAK + sb * 64 + kk * 8,
+                   smem_desc(sm + kSmQ + sb * 4096 + kk * 256, 128, 2048), id_score, kk > 0);
+          tc_commit(&bars.score_done[sb]);
+          ++ns;
+          prog = true;
+        }
+        if (nr < n_tiles && nr - ns < 2 &&
+            mbar_test(&bars.tile_in[nr % kNB], (nr / kNB) & 1)) {
+          const int kb = nr & 1, bd = nr % kNB;
+          tc_fence_after();
+          for (int kk = 0; kk < ksteps_recon; ++kk)
+            mma_ts(tmem + kColDr + kb * 128, tmem + kColALk + bd * 16 + kk * 8,
+                   smem_desc(sm + kSmBk + kk * 256, 128, 512), id_recon, kk > 0);
+          tc_commit(&bars.recon_done[kb]);
+          tc_commit(&bars.alk_free[bd]);
+          ++nr;
+          prog = true;
+        }
+        if (prog) {
+          idle = 0;
+        } else if ((++idle & 255u) == 0) {
+          if (*abort) break;
+          const uint64_t now = globaltimer();
+          if (idle == 256) idle_since = now;
+          else if (now - idle_since > kWaitLimitNs) {
+            *abort = 1;
+            atomicOr(err, kErrTimeout);
+            break;
+          }
+        }
       }
-      if (ok && n_tiles > 0) value(n_tiles - 1);
       // every MMA this thread issued must complete before TMEM is released
       tc_commit(&bars.mma_drain);
       volatile int no_abort = 0;
@@ -288,9 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     for (int jj = 0; jj < n_tiles; ++jj) {
       int u, jt, nt;
       unit_of(p, wk, t_first + jj, &u, &jt, &nt);
-      const int b = jj & 1, s = jj % kStages;
+      const int bd = jj % kNB, s = jj % kStages;
       if (u != cur_u) {
-        if (jj > 0 && !mbar_wait(&bars.recon_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort, err))
+        if (jj > 0 && !mbar_wait(&bars.alk_free[(jj - 1) % kNB], ((jj - 1) / kNB) & 1, abort, err))
           break;
         // B operand of the reconstruction: N = 128 dims x K = rk (logical ranks),
         // K-major core matrices, logical k holds Bk row perm_rank(k)
@@ -306,9 +338,10 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
         cur_u = u;
       }
       if (!mbar_wait(&bars.full[s], (jj / kStages) & 1, abort, err)) break;
-      if (jj >= 2) {
-        if (!mbar_wait(&bars.recon_done[b], ((jj - 2) >> 1) & 1, abort, err)) break;
-        if (!mbar_wait(&bars.v_done[b], ((jj - 2) >> 1) & 1, abort, err)) break;
+      if (jj >= kNB) {
+        // recon(jj - kNB) read this A buffer, value(jj - kNB) this L_v buffer
+        if (!mbar_wait(&bars.alk_free[bd], ((jj - kNB) / kNB) & 1, abort, err)) break;
+        if (!mbar_wait(&bars.v_done[bd], ((jj - kNB) / kNB) & 1, abort, err)) break;
       }
       tc_fence_after();
       const bool valid = row < nt;
@@ -322,26 +355,26 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
         const __half2 s2 = __low2half2(sz0), z2 = __high2half2(sz0);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if (j < p.rk / 8) {
-            dequant_word(valid ? codes[j] : 0u, s2, z2, ka + 4 * j);
-            if (!valid) ka[4 * j] = ka[4 * j + 1] = ka[4 * j + 2] = ka[4 * j + 3] = 0u;
+          if (j < p.rk / 8 && valid) {
+            dequant_word(codes[j], s2, z2, ka + 4 * j);
           } else {
             ka[4 * j] = ka[4 * j + 1] = ka[4 * j + 2] = ka[4 * j + 3] = 0u;
           }
         }
       }
-      tmem_st16(tmem + ((uint32_t)(32 * q4) << 16) + kColALk + b * 16, ka);
+      tmem_st16(tmem + ((uint32_t)(32 * q4) << 16) + kColALk + bd * 16, ka);
       // ---- values: rv/8 words -> shared memory (A of the value MMA, MN-major)
       {
         const uint8_t* vbase = st + kTile * (lk_row + lksz_row);
         const uint32_t* codes = reinterpret_cast<const uint32_t*>(vbase + row * lv_row);
         const __half2* sz = reinterpret_cast<const __half2*>(vbase + kTile * lv_row + row * lvsz_row);
-        uint8_t* lv = sm + kSmLV + b * 16384 + (row >> 3) * 128 + (row & 7) * 16;
+        uint8_t* lv = sm + kSmLV + bd * 16384 + (row >> 3) * 128 + (row & 7) * 16;
         for (int j = 0; j < rv / 8; ++j) {
-          const __half2 szg = sz[j / 4];          // group of 32 ranks = 4 words
-          uint32_t r[4];
-          dequant_word(valid ? codes[j] : 0u, __low2half2(szg), __high2half2(szg), r);
-          if (!valid) r[0] = r[1] = r[2] = r[3] = 0u;
+          uint32_t r[4] = {0u, 0u, 0u, 0u};
+          if (valid) {
+            const __half2 szg = sz[j / 4];          // group of 32 ranks = 4 words
+            dequant_word(codes[j], __low2half2(szg), __high2half2(szg), r);
+          }
           *reinterpret_cast<uint4*>(lv + j * 2048) = make_uint4(r[0], r[1], r[2], r[3]);
         }
         // the constant-one row (logical rank rv) sums P into the softmax denominator
@@ -355,52 +388,63 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bars.empty[s]);
-        mbar_arrive(&bars.tile_in[b]);
+        mbar_arrive(&bars.tile_in[bd]);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    const int h = (warp - kWarpEpi) >> 2;    // group: RoPE pairs 32h.., heads 2h, 2h+1
+    const int ew = (warp - kWarpEpi) & 3;    // warp index within the group
     const int q4 = warp & 3;
     const int row = 32 * q4 + lane;
-    const int ew = warp - kWarpEpi;           // 0..3 epilogue warp index
+    const int gtid = ew * 32 + lane;         // 0..127 within the group
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-    // RoPE rotation of this row (delta = row) for every pair, as f16x2 over
-    // consecutive frequencies (i, i + 1)
-    uint32_t cs[32], sn[32];
+    // RoPE rotation of this row (delta = row) for the group's pairs, as f16x2
+    // over consecutive frequencies (i, i + 1), i = 32h + 2k
+    uint32_t cs[16], sn[16];
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
+    for (int k = 0; k < 16; ++k) {
       float c0, s0, c1, s1;
-      const double t0 = (double)row * p.rope_f[2 * k], t1 = (double)row * p.rope_f[2 * k + 1];
+      const int i = 32 * h + 2 * k;
+      const double t0 = (double)row * p.rope_f[i], t1 = (double)row * p.rope_f[i + 1];
       sincospif(2.f * (float)(t0 - rint(t0)), &s0, &c0);
       sincospif(2.f * (float)(t1 - rint(t1)), &s1, &c1);
       cs[k] = pack_h2(c0, c1);
       sn[k] = pack_h2(s0, s1);
     }
-    // queries of the current unit for the q-side rotation: this thread rotates
-    // pair i = row % 64 of heads 2 * (row / 64) and 2 * (row / 64) + 1
-    const int qi = row & (kHalf - 1), qh0 = 2 * (row >> 6);
-    float qlo[2], qhi[2];
-    float m_ref[kG];
-    int cur_u = -1, unit_idx = -1, cur_b = 0, cur_kvh = 0, cur_slot = 0;
+    // q-side rotation: this thread rotates pair qi of head qh
+    const int qi = 32 * h + (gtid & 31), qh = gtid >> 5;
+    float qlo = 0.f, qhi = 0.f;
+    int rope_u = -1;
+    // softmax state of the group's two heads
+    float m_ref[2] = {-INFINITY, -INFINITY};
+    int sm_u = -1, sm_b = 0, sm_kvh = 0, sm_slot = 0, sm_last = -1;
     const size_t rows_q = (size_t)p.B * p.Hq;
     const int pst = p.vdim + 2;
-
+    uint32_t epi_phase = 0;
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(&bars.epi_sync[h]);
+      const bool r = mbar_wait(&bars.epi_sync[h], epi_phase & 1, abort, err);
+      ++epi_phase;
+      return r;
+    };
+    // the accumulator of the finished unit -> partials of the group's heads
     auto finish_unit = [&](int jj_last) -> bool {
-      if (!mbar_wait(&bars.v_done[jj_last & 1], (jj_last >> 1) & 1, abort, err)) return false;
+      if (!mbar_wait(&bars.v_done[jj_last % kNB], (jj_last / kNB) & 1, abort, err)) return false;
       tc_fence_after();
-      uint32_t r[16];
-      tmem_ld16(tmem + lane_base + kColAcc, r);
+      uint32_t r[2];
+      tmem_ld2(tmem + lane_base + kColAcc + 2 * h, r);
       tmem_wait_ld();
       reg_fence(r);
       if (lane < 16) {
         const int m = 16 * q4 + lane;          // logical value row
-        for (int h = 0; h < kG; ++h) {
-          const size_t qr = (size_t)cur_b * p.Hq + cur_kvh * kG + h;
-          float* dst = p.part + ((size_t)cur_slot * rows_q + qr) * pst;
-          const float v = __uint_as_float(r[h]);
+        for (int e = 0; e < 2; ++e) {
+          const size_t qr = (size_t)sm_b * p.Hq + sm_kvh * kG + 2 * h + e;
+          float* dst = p.part + ((size_t)sm_slot * rows_q + qr) * pst;
+          const float v = __uint_as_float(r[e]);
           if (m < rv) dst[perm_rank(m)] = v;
           else if (m == rv) {
-            dst[p.vdim] = m_ref[h];
+            dst[p.vdim] = m_ref[e];
             dst[p.vdim + 1] = v;
           }
         }
@@ -410,160 +454,158 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       return true;
     };
 
-    uint32_t epi_phase = 0;
-    auto epi_sync = [&]() -> bool {
-      mbar_arrive(&bars.epi_sync);
-      const bool r = mbar_wait(&bars.epi_sync, epi_phase & 1, abort, err);
-      ++epi_phase;
-      return r;
-    };
-
-    bool ok = true;
-    int jj = 0;
-    for (; jj < n_tiles && ok; ++jj) {
+    // ---- stage 1: q_rot and RoPE of the reconstructed keys (in place)
+    auto rope_stage = [&](int jj) -> bool {
       int u, jt, nt;
       unit_of(p, wk, t_first + jj, &u, &jt, &nt);
-      const int b = jj & 1;
-      if (u != cur_u) {
-        if (cur_u >= 0 && !(ok = finish_unit(jj - 1))) break;
-        cur_u = u;
-        ++unit_idx;
-        cur_b = u / p.Hkv;
-        cur_kvh = u % p.Hkv;
-        cur_slot = cta - (int)(((long long)u * wk.tpu) / wk.W);
-        const __nv_bfloat16* qq = p.q + ((size_t)cur_b * p.Hq + cur_kvh * kG) * kD;
-        for (int h = 0; h < 2; ++h) {
-          qlo[h] = bf2f(qq[(qh0 + h) * kD + qi]);
-          qhi[h] = bf2f(qq[(qh0 + h) * kD + qi + kHalf]);
-        }
-#pragma unroll
-        for (int h = 0; h < kG; ++h) m_ref[h] = -INFINITY;
+      if (u != rope_u) {
+        rope_u = u;
+        const __nv_bfloat16* qq =
+            p.q + ((size_t)(u / p.Hkv) * p.Hq + (u % p.Hkv) * kG + qh) * kD;
+        qlo = bf2f(qq[qi]);
+        qhi = bf2f(qq[qi + kHalf]);
       }
-      // ---- q_rot = R_t0^T q for this tile (B operand of the score MMA)
       {
+        // q_rot = R_t0^T q (B operand of the score MMA); this buffer was last
+        // read by score(jj - 2), whose completion the softmax stage of jj - 2 saw
         const double turns = (double)(jt * kTile) * p.rope_f[qi];
         float sa, ca;
         sincospif(2.f * (float)(turns - rint(turns)), &sa, &ca);
-        __half* qd = reinterpret_cast<__half*>(sm + kSmQ + b * 4096);
-        for (int h = 0; h < 2; ++h) {
-          const int hh = qh0 + h;
-          const float rl = ca * qlo[h] + sa * qhi[h];
-          const float rh = ca * qhi[h] - sa * qlo[h];
-          qd[((hh >> 3) * 2048 + (qi >> 3) * 128 + (hh & 7) * 16 + (qi & 7) * 2) / 2] =
-              __float2half_rn(rl);
-          const int qj = qi + kHalf;
-          qd[((hh >> 3) * 2048 + (qj >> 3) * 128 + (hh & 7) * 16 + (qj & 7) * 2) / 2] =
-              __float2half_rn(rh);
-        }
+        __half* qd = reinterpret_cast<__half*>(sm + kSmQ + (jj & 1) * 4096);
+        const float rl = ca * qlo + sa * qhi;
+        const float rh = ca * qhi - sa * qlo;
+        qd[((qh >> 3) * 2048 + (qi >> 3) * 128 + (qh & 7) * 16 + (qi & 7) * 2) / 2] =
+            __float2half_rn(rl);
+        const int qj = qi + kHalf;
+        qd[((qh >> 3) * 2048 + (qj >> 3) * 128 + (qh & 7) * 16 + (qj & 7) * 2) / 2] =
+            __float2half_rn(rh);
       }
-      // ---- RoPE of the reconstructed keys: K'' = R_delta K_hat, into TMEM (fp16)
-      if (!(ok = mbar_wait(&bars.recon_done[b], (jj >> 1) & 1, abort, err))) break;
+      if (!mbar_wait(&bars.recon_done[jj & 1], (jj >> 1) & 1, abort, err)) return false;
       tc_fence_after();
+      // K_hat (fp32, column = dim) -> K'' (f16x2, column c = dims 2c, 2c+1).
+      // This group rotates the low dims 32h..32h+31 against 64+32h..64+32h+31,
+      // in two halves of 16 pairs.
+      const uint32_t dr = tmem + lane_base + kColDr + (jj & 1) * 128;
+      const uint32_t ak = tmem + lane_base + kColAK + (jj & 1) * 64;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        // dims 8c..8c+7 (low half) and 64+8c..64+8c+7 (high half): 4 f16x2 each,
-        // stored at columns 4c.. and 32+4c.. (column k holds dims 2k, 2k+1)
-        uint32_t lo[8], hi[8];
-        tmem_ld8(tmem + lane_base + kColDr + b * 128 + 8 * c, lo);
-        tmem_ld8(tmem + lane_base + kColDr + b * 128 + kHalf + 8 * c, hi);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t lo[16], hi[16];
+        tmem_ld16(dr + 32 * h + 16 * half, lo);
+        tmem_ld16(dr + kHalf + 32 * h + 16 * half, hi);
         tmem_wait_ld();
         reg_fence(lo);
         reg_fence(hi);
-        uint32_t xo[4], yo[4];
+        uint32_t xo[8], yo[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 8; ++k) {
           const __half2 x = __floats2half2_rn(__uint_as_float(lo[2 * k]), __uint_as_float(lo[2 * k + 1]));
           const __half2 y = __floats2half2_rn(__uint_as_float(hi[2 * k]), __uint_as_float(hi[2 * k + 1]));
-          const __half2 C = *reinterpret_cast<const __half2*>(&cs[4 * c + k]);
-          const __half2 S = *reinterpret_cast<const __half2*>(&sn[4 * c + k]);
+          const __half2 C = *reinterpret_cast<const __half2*>(&cs[8 * half + k]);
+          const __half2 S = *reinterpret_cast<const __half2*>(&sn[8 * half + k]);
           const __half2 xr = __hfma2(C, x, __hneg2(__hmul2(S, y)));   // k_i cos - k_{i+64} sin
           const __half2 yr = __hfma2(C, y, __hmul2(S, x));            // k_{i+64} cos + k_i sin
           xo[k] = *reinterpret_cast<const uint32_t*>(&xr);
           yo[k] = *reinterpret_cast<const uint32_t*>(&yr);
         }
-        tmem_st4(tmem + lane_base + kColAK + b * 64 + 4 * c, xo);
-        tmem_st4(tmem + lane_base + kColAK + b * 64 + 32 + 4 * c, yo);
+        tmem_st8(ak + 16 * h + 8 * half, xo);
+        tmem_st8(ak + 32 + 16 * h + 8 * half, yo);
       }
       tmem_wait_st();
       tc_fence_before();
       fence_proxy_async_smem();
-      mbar_arrive(&bars.kq_full[b]);
+      mbar_arrive(&bars.kq_full[jj & 1]);
+      return true;
+    };
 
-      // ---- scores and the online softmax
-      if (!(ok = mbar_wait(&bars.score_done[b], (jj >> 1) & 1, abort, err))) break;
+    // ---- stage 2: scores, online softmax, P
+    auto softmax_stage = [&](int jj) -> bool {
+      int u, jt, nt;
+      unit_of(p, wk, t_first + jj, &u, &jt, &nt);
+      if (u != sm_u) {
+        if (sm_u >= 0 && !finish_unit(sm_last)) return false;
+        sm_u = u;
+        sm_b = u / p.Hkv;
+        sm_kvh = u % p.Hkv;
+        sm_slot = cta - (int)(((long long)u * wk.tpu) / wk.W);
+        m_ref[0] = m_ref[1] = -INFINITY;
+      }
+      const int sb = jj & 1;
+      if (!mbar_wait(&bars.score_done[sb], (jj >> 1) & 1, abort, err)) return false;
       tc_fence_after();
-      uint32_t sr[4];
-      tmem_ld4(tmem + lane_base + kColS + b * 16, sr);
+      uint32_t sr[2];
+      tmem_ld2(tmem + lane_base + kColS + sb * 16 + 2 * h, sr);
       tmem_wait_ld();
       reg_fence(sr);
       const bool valid = row < nt;
-      float s2[kG];
+      float s2[2];
       bool need = false;
 #pragma unroll
-      for (int h = 0; h < kG; ++h) {
-        s2[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
-        need |= s2[h] > m_ref[h] + 8.f;
+      for (int e = 0; e < 2; ++e) {
+        s2[e] = valid ? __uint_as_float(sr[e]) * p.scale_log2 : -INFINITY;
+        need |= s2[e] > m_ref[e] + 8.f;
       }
-      // a flag is reset two tiles after its last read (every thread has passed
-      // the synchronisation of the tile in between)
+      // P buffer sb was read by value(jj - 2)
+      if (jj >= 2 && !mbar_wait(&bars.v_done[(jj - 2) % kNB], ((jj - 2) / kNB) & 1, abort, err))
+        return false;
+      // a flag is reset two tiles after its last read (every thread of the
+      // group has passed the synchronisation in between)
       const int fl = jj % 3;
-      if (threadIdx.x == 32 * kWarpEpi) bars.flag[(jj + 1) % 3] = 0;
-      if (__any_sync(0xffffffffu, need) && lane == 0) atomicOr(&bars.flag[fl], 1);
-      if (!(ok = epi_sync())) break;
-      if (bars.flag[fl]) {
+      if (gtid == 0) bars.flag[h][(jj + 1) % 3] = 0;
+      if (__any_sync(0xffffffffu, need) && lane == 0) atomicOr(&bars.flag[h][fl], 1);
+      if (!epi_sync()) return false;
+      if (bars.flag[h][fl]) {
         // raise the reference maximum to the tile maximum, rescale acc
 #pragma unroll
-        for (int h = 0; h < kG; ++h) {
-          const float tm = warp_max(s2[h]);
-          if (lane == 0) bars.wmax[ew][h] = tm;
+        for (int e = 0; e < 2; ++e) {
+          const float tm = warp_max(s2[e]);
+          if (lane == 0) bars.wmax[h][ew][e] = tm;
         }
-        if (!(ok = epi_sync())) break;
-        float alpha[kG];
+        if (!epi_sync()) return false;
+        float alpha[2];
         bool any_scale = false;
 #pragma unroll
-        for (int h = 0; h < kG; ++h) {
-          const float mt = fmaxf(fmaxf(bars.wmax[0][h], bars.wmax[1][h]),
-                                 fmaxf(bars.wmax[2][h], bars.wmax[3][h]));
-          const float mn = fmaxf(m_ref[h], mt);
-          alpha[h] = (m_ref[h] == -INFINITY) ? 1.f : exp2f(m_ref[h] - mn);
-          any_scale |= (m_ref[h] != -INFINITY) && (mn > m_ref[h]);
-          m_ref[h] = mn;
+        for (int e = 0; e < 2; ++e) {
+          const float mt = fmaxf(fmaxf(bars.wmax[h][0][e], bars.wmax[h][1][e]),
+                                 fmaxf(bars.wmax[h][2][e], bars.wmax[h][3][e]));
+          const float mn = fmaxf(m_ref[e], mt);
+          alpha[e] = (m_ref[e] == -INFINITY) ? 1.f : exp2f(m_ref[e] - mn);
+          any_scale |= (m_ref[e] != -INFINITY) && (mn > m_ref[e]);
+          m_ref[e] = mn;
         }
-        // no earlier value MMA of this unit exists while m_ref was -inf; any_scale
-        // is the same in every thread (same wmax, same m_ref)
+        // while m_ref was -inf there is no earlier value MMA of this unit;
+        // any_scale is the same in every thread of the group
         if (any_scale) {
-          ok = mbar_wait(&bars.v_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort, err);
-          if (ok) {
-            tc_fence_after();
-            uint32_t r[16];
-            tmem_ld16(tmem + lane_base + kColAcc, r);
-            tmem_wait_ld();
-            reg_fence(r);
-#pragma unroll
-            for (int h = 0; h < kG; ++h) r[h] = __float_as_uint(__uint_as_float(r[h]) * alpha[h]);
-            tmem_st16(tmem + lane_base + kColAcc, r);
-            tmem_wait_st();
-            tc_fence_before();
-          }
+          if (!mbar_wait(&bars.v_done[(jj - 1) % kNB], ((jj - 1) / kNB) & 1, abort, err))
+            return false;
+          tc_fence_after();
+          uint32_t r[2];
+          tmem_ld2(tmem + lane_base + kColAcc + 2 * h, r);
+          tmem_wait_ld();
+          reg_fence(r);
+          r[0] = __float_as_uint(__uint_as_float(r[0]) * alpha[0]);
+          r[1] = __float_as_uint(__uint_as_float(r[1]) * alpha[1]);
+          tmem_st2(tmem + lane_base + kColAcc + 2 * h, r);
+          tmem_wait_st();
+          tc_fence_before();
         }
-        if (!epi_sync() || !ok) {   // wmax is read by everyone before it is reused
-          ok = false;
-          break;
-        }
+        if (!epi_sync()) return false;   // wmax is read by everyone before it is reused
       }
-      // ---- P (fp16) into the B operand of the value MMA: row -> 8 bytes
-      if (jj >= 2 && !(ok = mbar_wait(&bars.v_done[b], ((jj - 2) >> 1) & 1, abort, err))) break;
-      {
-        float pv[kG];
-#pragma unroll
-        for (int h = 0; h < kG; ++h) pv[h] = valid ? exp2f(s2[h] - m_ref[h]) : 0.f;
-        uint2 w2 = make_uint2(pack_h2(pv[0], pv[1]), pack_h2(pv[2], pv[3]));
-        *reinterpret_cast<uint2*>(sm + kSmP + b * 4096 + (row >> 3) * 128 + (row & 7) * 16) = w2;
-      }
+      const float p0 = valid ? exp2f(s2[0] - m_ref[0]) : 0.f;
+      const float p1 = valid ? exp2f(s2[1] - m_ref[1]) : 0.f;
+      *reinterpret_cast<uint32_t*>(sm + kSmP + sb * 4096 + (row >> 3) * 128 + (row & 7) * 16 +
+                                   4 * h) = pack_h2(p0, p1);
       fence_proxy_async_smem();
-      mbar_arrive(&bars.p_full[b]);
+      mbar_arrive(&bars.p_full[sb]);
+      sm_last = jj;
+      return true;
+    };
+
+    bool ok = true;
+    for (int jj = 0; jj <= n_tiles && ok; ++jj) {
+      if (jj < n_tiles) ok = rope_stage(jj);
+      if (ok && jj >= 1) ok = softmax_stage(jj - 1);
     }
-    if (ok && n_tiles > 0 && cur_u >= 0) finish_unit(n_tiles - 1);
+    if (ok && sm_u >= 0) finish_unit(sm_last);
   }
 
   tc_fence_before();
@@ -583,15 +625,16 @@ bool rope_tc_supported(const Params& p) {
          kTile * (p.lk_row + p.lksz_row + p.lv_row + p.lvsz_row) <= kStageMax;
 }
 
-// Partial slots a unit spans under the persistent partition.
+// Persistent partition: grid CTAs of W tiles each; a unit of tpu tiles spans
+// at most ceil(tpu / W) + 1 CTAs, each with one partial per unit.
 void rope_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots) {
   const int t = (p.n_tokens + kTile - 1) / kTile;
   const int units = p.B * p.Hkv;
   const int total = units * t;
-  int g = total < kNumSMs ? total : kNumSMs;
-  const int w = (total + g - 1) / g;
-  g = (total + w - 1) / w;
-  *grid = g;
+  int gr = total < kNumSMs ? total : kNumSMs;
+  const int w = (total + gr - 1) / gr;
+  gr = (total + w - 1) / w;
+  *grid = gr;
   *W = w;
   *tpu = t;
   *slots = (t + w - 1) / w + 1;
@@ -605,6 +648,7 @@ cudaError_t launch_rope_tc(const Params& p, uint32_t* err, cudaStream_t s) {
                                        kSmAlloc);
   if (e != cudaSuccess) return e;
   static_assert(kSmTotal + 1024 <= kSmAlloc, "shared memory carve-up exceeds the allocation");
+  static_assert(sizeof(Bars) <= 1024, "barrier block exceeds its slot");
   rope_tc_kernel<<<grid, kThreads, kSmAlloc, s>>>(p, wk, err);
   return cudaGetLastError();
 }
