@@ -199,6 +199,44 @@ class Cache:
         return c
 
 
+class RawEvent:
+    """A CUDA event created through the CUDA runtime that libkvc links, so that
+    the library can record it (kvc_decode_attn_timed) and the caller can read
+    the elapsed time."""
+
+    _rt = None
+
+    @classmethod
+    def rt(cls):
+        if cls._rt is None:
+            lib()  # libkvc pulls in the CUDA runtime
+            rt = C.CDLL("libcudart.so.12")
+            rt.cudaEventCreate.argtypes = [C.POINTER(C.c_void_p)]
+            rt.cudaEventElapsedTime.argtypes = [C.POINTER(C.c_float), C.c_void_p, C.c_void_p]
+            rt.cudaEventDestroy.argtypes = [C.c_void_p]
+            cls._rt = rt
+        return cls._rt
+
+    def __init__(self):
+        self.cuda_event = C.c_void_p()
+        err = self.rt().cudaEventCreate(C.byref(self.cuda_event))
+        if err != 0:
+            raise RuntimeError(f"cudaEventCreate failed ({err})")
+        self.cuda_event = self.cuda_event.value
+
+    def elapsed_ms(self, end):
+        ms = C.c_float()
+        err = self.rt().cudaEventElapsedTime(C.byref(ms), C.c_void_p(self.cuda_event),
+                                             C.c_void_p(end.cuda_event))
+        if err != 0:
+            raise RuntimeError(f"cudaEventElapsedTime failed ({err})")
+        return ms.value
+
+    def __del__(self):
+        if self._rt is not None and getattr(self, "cuda_event", None):
+            self._rt.cudaEventDestroy(C.c_void_p(self.cuda_event))
+
+
 def current_stream_ptr():
     import torch
 
