@@ -242,6 +242,30 @@ kvc_status kvc_decode_attn_timed(const kvc_layout* layout, const kvc_cache* cach
                                  size_t ws_bytes, void* stream,
                                  void* ev_begin, void* ev_end);
 
+/* Bytes of the library's built-in decode scratch area (see below). */
+#define KVC_STATIC_SCRATCH_BYTES (4u << 20)
+
+/* Decode without a caller-provided workspace.  This entry point has no
+ * counterpart on the pages; it exists for callers that cannot allocate device
+ * memory themselves -- code embedded in a host framework that owns every
+ * device allocation and does not expose an allocator, or a latency-critical
+ * serving loop that must not call cudaMalloc (which can synchronize the
+ * device).  It allocates nothing: its scratch is a file-scope device array of
+ * KVC_STATIC_SCRATCH_BYTES bytes that every GPU loading the library keeps
+ * until the process exits.  The caller still passes the cache, q and out, as
+ * for kvc_decode_attn, which this call runs with that array as the workspace.
+ *   - Layouts whose kvc_workspace_bytes(layout, cache->n_tokens) exceeds
+ *     KVC_STATIC_SCRATCH_BYTES are rejected with KVC_EWORKSPACE (nothing runs).
+ *   - The first call on a device looks up the array's device address on the
+ *     current device (once per device, with that device current); make that
+ *     first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; the call clears what must start at zero (the error word) on the
+ *     stream before the kernels run.  Calls that overlap on the GPU (other
+ *     streams, other threads) race on the array: serialize them. */
+kvc_status kvc_decode_attn_static(const kvc_layout* layout, const kvc_cache* cache,
+                                  const void* q, void* out, void* stream);
+
 /* Thread-local description of the last error on this thread ("" if none). */
 const char* kvc_last_error(void);
 

@@ -88,6 +88,16 @@ size_t ws_bytes(const kvc_layout* L, int n_tokens) {
 
 }  // namespace
 
+kvc_status kvc::report_error(kvc_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
 extern "C" {
 
 const char* kvc_last_error(void) { return g_err.c_str(); }

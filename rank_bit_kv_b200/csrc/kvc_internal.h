@@ -102,6 +102,9 @@ bool rope_tc_supported(const Params& p);
 void rope_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
 cudaError_t launch_rope_tc(const Params& p, uint32_t* err, cudaStream_t s);
 
+// Record a status and message for kvc_last_error(); returns st.
+kvc_status report_error(kvc_status st, const char* fmt, ...);
+
 // kernel launchers (return the cudaGetLastError of the launch)
 cudaError_t launch_qproj(const Params& p, cudaStream_t s);
 cudaError_t launch_split(const Params& p, cudaStream_t s);

@@ -76,6 +76,8 @@ def lib():
         L.kvc_decode_attn.restype = C.c_int
         L.kvc_decode_attn_timed.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, vp, sz, vp, vp, vp]
         L.kvc_decode_attn_timed.restype = C.c_int
+        L.kvc_decode_attn_static.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, vp]
+        L.kvc_decode_attn_static.restype = C.c_int
         L.kvc_last_error.argtypes = []
         L.kvc_last_error.restype = C.c_char_p
         L.kvc_version.argtypes = []
@@ -254,6 +256,17 @@ def decode(layout: Layout, cache: Cache, q, out, ws, stream=None, events=None):
         check(lib().kvc_decode_attn_timed(layout.h, C.byref(cs), _ptr(q), _ptr(out), _ptr(ws),
                                           ws.numel(), st, C.c_void_p(events[0].cuda_event),
                                           C.c_void_p(events[1].cuda_event)))
+
+
+STATIC_SCRATCH_BYTES = 4 << 20   # KVC_STATIC_SCRATCH_BYTES
+
+
+def decode_static(layout: Layout, cache: Cache, q, out, stream=None):
+    """kvc_decode_attn_static: decode with the library's built-in scratch area
+    (for callers that cannot allocate a workspace)."""
+    cs = cache.struct()
+    st = stream if stream is not None else current_stream_ptr()
+    check(lib().kvc_decode_attn_static(layout.h, C.byref(cs), _ptr(q), _ptr(out), st))
 
 
 def append(layout: Layout, cache: Cache, k_new, v_new, pos, n_new, new_ranks=None,
