@@ -33,12 +33,12 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
 
   // partial slots of this row: all S splits, or -- on the persistent
   // tensor-core path -- one partial for every CTA whose tile range covers
-  // this row's unit
+  // this row's unit (seg_parts partials per CTA)
   int nS = p.S;
   if (p.seg_W > 0) {
     const int u = (row / p.Hq) * p.Hkv + kvh;   // L == 1 on this path
     const long long a = (long long)u * p.seg_tpu, e = (long long)(u + 1) * p.seg_tpu - 1;
-    nS = (int)(e / p.seg_W - a / p.seg_W + 1);
+    nS = (int)(e / p.seg_W - a / p.seg_W + 1) * p.seg_parts;
   }
   if (tid < 32) {
     float mx = -INFINITY;

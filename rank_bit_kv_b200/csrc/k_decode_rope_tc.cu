@@ -1,5 +1,4 @@
-// Split-T fused decode for low-rank INT4 caches with keys stored before RoPE,
-// on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
+// Split-T fused decode for low-rank INT4 caches with keys stored before RoPE.
 //
 // Per KV head the cache holds INT4 latents L_k (T x rk) and L_v (T x rv) with
 // per-group fp16 (scale, zero); keys are k_t = l_t Bk rotated by RoPE at slot
@@ -7,38 +6,41 @@
 // pre-RoPE; the FlashJoLT decode "attends directly on the stored core,
 // factors and residual").  For a tile of 128 tokens starting at t0 the kernel
 //   1. stages the compressed rows with 1-D bulk copies (no multicast),
-//   2. dequantizes L_k into TMEM (the A operand) and L_v into shared memory,
-//   3. reconstructs K_hat = L_k Bk on the tensor cores (M = 128 tokens,
-//      N = 128 dims, K = rk) into TMEM (fp32),
-//   4. applies RoPE as R_t = R_t0 R_delta (delta = row in the tile), writing
-//      K'' as packed fp16 back to TMEM (the A operand of the score MMA):
-//      each epilogue thread owns one row, so R_delta is a per-thread constant
-//      rotation, and R_t0 is folded into the queries (q_rot = R_t0^T q, so
+//   2. dequantizes L_k into TMEM and L_v into shared memory,
+//   3. reconstructs K_hat = L_k Bk with one tcgen05 MMA per 16 ranks
+//      (M = 128 tokens, N = 128 dims, f16 accumulator in TMEM),
+//   4. applies RoPE as R_t = R_t0 R_delta (delta = row in the tile): R_delta is
+//      a per-thread constant rotation (each thread always owns the same rows),
+//      R_t0 is folded into the queries (q_rot = R_t0^T q, so
 //      q . R_t k = q_rot . R_delta k) -- no per-token sin/cos,
-//   5. scores S = K'' q_rot^T on the tensor cores with K'' read from TMEM,
-//   6. runs an online softmax with a lazily raised reference maximum,
-//   7. accumulates acc^T += L_v^T P in latent space on the tensor cores, with
-//      a constant-one row so that the same MMA also sums P (the softmax
-//      denominator),
-// and writes per-(segment, query head) partials (acc, m, l) that the split
-// combine merges and up-projects by Bv once per head.
+//   5. scores S = K'' q_rot^T and accumulates acc^T += L_v^T P with warp-level
+//      mma.sync (m16n8k16): these products have N = 4 query heads, and a
+//      tcgen05 MMA costs the same ~135 SM cycles per K = 16 step whatever its
+//      N, so only the N = 128 reconstruction runs on tcgen05,
+//   6. keeps an online softmax per warp with a lazily raised reference
+//      maximum (rescaling only when a score exceeds it by 2^8),
+// and writes one partial (acc, m, l) per warp and unit that the split combine
+// merges and up-projects by Bv once per head.
+//
+// TMEM -> registers uses the 16x256b shape with 16-bit packing: each warp gets
+// its 16 rows of K_hat with four consecutive f16 columns per thread and row,
+// which become the A fragments of the score MMA once the k order inside every
+// 16-wide step is permuted the same way on the query side (the query
+// fragments are stored in that order).
 //
 // The grid is persistent: the tiles of all (batch row, KV head) units are cut
 // into equal contiguous ranges, one per CTA, so every SM streams the same
-// number of bytes; a range may cross a unit boundary (two partials).
+// number of bytes; a range may cross a unit boundary (a partial per part).
 //
 // Warp roles (448 threads, one CTA per SM):
 //   warp 0      bulk-copy producer (6-stage ring of compressed tiles)
-//   warp 1      TMEM allocation + MMA issue (one lane, non-blocking scheduler)
-//   warps 2-9   epilogue: two groups of four warps work on the same tile;
-//               group h rotates RoPE pairs 32h..32h+31 and owns query heads
-//               2h, 2h+1 (their scores, softmax state, P columns, partials).
-//               Software-pipelined: RoPE of tile t, then softmax of tile t-1.
-//   warps 10-13 dequantization (thread = row)
-// Buffer rings: compressed stages (6), dequantized operands (4), reconstructed
-// keys and rotated keys in TMEM (2 each), scores (2), P and q_rot (2).  Every wait is bounded; on a
-// timeout the CTA sets an error bit in the workspace, drains its own bulk
-// copies and MMAs, frees TMEM and exits.
+//   warp 1      TMEM allocation + tcgen05 reconstruction MMAs (one lane)
+//   warps 2-5   dequantization (thread = token row); warp 2 also rotates the
+//               queries of each tile
+//   warps 6-13  epilogue: each owns 16 rows of every tile, in its TMEM lane
+//               quadrant
+// Every wait is bounded; on a timeout the CTA sets an error bit in the
+// workspace, drains its own bulk copies and MMAs, frees TMEM and exits.
 #include <math.h>
 
 #include "kvc_device.cuh"
@@ -50,54 +52,70 @@ namespace {
 using namespace tc;
 
 constexpr int kTile = 128;
-constexpr int kStages = 6;
+constexpr int kStagesLog2 = 3, kStages = 1 << kStagesLog2;
 constexpr int kThreads = 448;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpEpi = 2, kWarpDeq = 10;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpDeq = 2, kWarpEpi = 6, kEpiWarps = kRopeTcParts;
 constexpr int kD = 128;            // head dim
 constexpr int kHalf = 64;          // RoPE pairs
 constexpr int kG = 4;              // query heads per KV head
-constexpr int kVM = 64;            // M of the value MMA (rank_v + 1 <= 64)
-constexpr int kN = 16;             // N of score / value MMAs (4 heads padded)
-constexpr int kNB = 4;             // dequantized operand buffers (tile jj uses jj % kNB)
+constexpr int kRvMax = 48;         // value rank handled (3 m16 tiles)
+constexpr int kLvStride = 56;      // halves per L_v row in shared memory (48 + pad)
+constexpr int kNBLog2 = 2, kNB = 1 << kNBLog2;   // dequantized operand buffers (tile jj uses jj % kNB)
 
-// TMEM columns (512 allocated); a 16-bit accumulator would still take one
-// column per value, while a TMEM A operand packs two fp16 per column, so the
-// reconstruction stays fp32 and the rotated keys get their own packed buffer
+// TMEM columns (512 allocated)
 constexpr uint32_t kColALk = 0;    // kNB x 16   recon A (128 x rk fp16, rk <= 32)
-constexpr uint32_t kColS = 64;     // 2 x 16     scores (fp32)
-constexpr uint32_t kColAcc = 96;   // 16         value accumulator (M = 64 layout)
-constexpr uint32_t kColDr = 128;   // 2 x 128    reconstructed keys K_hat (fp32)
-constexpr uint32_t kColAK = 384;   // 2 x 64     rotated keys K'' (packed fp16)
+constexpr int kNDr = 3;            // K_hat buffers (tile jj uses jj % kNDr)
+constexpr uint32_t kColDr = 128;   // kNDr x 128 reconstructed keys K_hat (f16, one per column)
 constexpr uint32_t kTmemCols = 512;
 
 // Shared memory carve-up (bytes, from a 1024-aligned base)
-constexpr int kSmStage = 0;                            // kStages x stage bytes
+constexpr int kSmStage = 0;                              // kStages x stage bytes
 constexpr int kStageMax = 8192;
-constexpr int kSmBk = kSmStage + kStages * kStageMax;   // 8 KB   B of recon (128 x 32)
-constexpr int kSmQ = kSmBk + 8192;                     // 2 x 4 KB   B of score (16 x 128)
-constexpr int kSmLV = kSmQ + 2 * 4096;                 // kNB x 16 KB A of value (64 x 128)
-constexpr int kSmP = kSmLV + kNB * 16384;              // 2 x 4 KB   B of value (128 x 16)
-constexpr int kSmBar = kSmP + 2 * 4096;                // barriers + scratch
+constexpr int kSmBk = kSmStage + kStages * kStageMax;     // 8 KB  B of recon (128 x 32)
+constexpr int kLvBytes = kTile * kLvStride * 2;           // 14 KB per buffer
+constexpr int kSmLV = kSmBk + 8192;                      // kNB x L_v tile [128][56] fp16
+constexpr int kQfBytes = 2048;                           // q_rot fragments of a tile (8 heads, 4..7 zero)
+constexpr int kSmQF = kSmLV + kNB * kLvBytes;            // kNB x 2 KB
+constexpr int kSmBar = kSmQF + kNB * kQfBytes;           // barriers
 constexpr int kSmTotal = kSmBar + 1024;
-constexpr int kSmAlloc = kSmTotal + 2048;              // > half the SM: one CTA per SM
+constexpr int kSmAlloc = kSmTotal + 2048 > 120 * 1024 ? kSmTotal + 2048 : 120 * 1024;
 
 struct Bars {
   uint64_t full[kStages], empty[kStages];
-  uint64_t tile_in[kNB], v_done[kNB];       // per dequantized operand buffer
-  uint64_t alk_free[kNB];                   // recon of the buffer's last tile completed
-  uint64_t recon_done[2], kq_full[2];       // per reconstructed / rotated key buffer
-  uint64_t score_done[2], p_full[2];        // per score / P buffer
-  uint64_t acc_free;                        // the accumulator was read at a unit end
-  uint64_t epi_sync[2];                     // bounded barrier among a group's 128 threads
-  uint64_t mma_drain;                       // last MMAs of the CTA completed
+  uint64_t tile_in[kNB];     // L_k in TMEM, L_v and q_rot in shared memory (4 dequant warps)
+  uint64_t alk_free[kNB];    // recon of the buffer's last tile completed (tcgen05.commit)
+  uint64_t lv_free[kNB];     // every epilogue warp is done with L_v / q_rot of the buffer
+  uint64_t recon_done[kNDr]; // K_hat buffer written
+  uint64_t dr_free[kNDr];    // every epilogue warp has loaded the K_hat buffer
+  uint64_t mma_drain;        // last MMAs of the CTA completed
   uint32_t tmem_base;
   int abort;
-  int flag[2][3];
-  float wmax[2][4][2];
 };
+
+// slot and phase parity of tile j in a ring of 2^lg buffers
+template <int lg>
+__device__ __forceinline__ int slot_of(int j) { return j & ((1 << lg) - 1); }
+template <int lg>
+__device__ __forceinline__ uint32_t phase_of(int j) { return ((uint32_t)j >> lg) & 1u; }
+__device__ __forceinline__ int dr_slot(int j) { return (int)((uint32_t)j % kNDr); }
+__device__ __forceinline__ uint32_t dr_phase(int j) { return ((uint32_t)j / kNDr) & 1u; }
 
 struct Work {
   int W, tpu, total;     // tiles per CTA, tiles per unit, all tiles
+};
+
+// Position of a CTA's tile in its unit, advanced one tile at a time.
+struct TileCursor {
+  int u, jt, tpu;
+  __device__ TileCursor(int t, int tiles_per_unit)
+      : u(t / tiles_per_unit), jt(t % tiles_per_unit), tpu(tiles_per_unit) {}
+  __device__ void next() {
+    if (++jt == tpu) {
+      jt = 0;
+      ++u;
+    }
+  }
+  __device__ int valid_rows(int n_tokens) const { return min(kTile, n_tokens - jt * kTile); }
 };
 
 // rank permutation of the nibble extraction: logical k = 8j + 2a + h holds
@@ -129,13 +147,19 @@ __device__ __forceinline__ void dequant_word(uint32_t w, __half2 s2, __half2 z2,
   }
 }
 
-__device__ __forceinline__ void unit_of(const Params& p, const Work& w, int T, int* u, int* jt,
-                                        int* nt) {
-  *u = T / w.tpu;
-  *jt = T % w.tpu;
-  *nt = min(kTile, p.n_tokens - *jt * kTile);
+// Byte offset of the f16 pair q_rot[h][d], q_rot[h][d + 1] (d even) in a
+// tile's query-fragment buffer.  Epilogue thread (g = head, c4) reads 64
+// contiguous bytes: for every 16-wide k step kk the dims kk*16 + 4*c4 + 0..3
+// (b0 = first two, b1 = last two), 16-byte chunks XOR-swizzled so that the
+// 8 threads of a load phase hit distinct banks.
+__device__ __forceinline__ int qf_offset(int h, int d) {
+  const int kk = d >> 4, w = d & 15, c4 = w >> 2, e = w & 3;
+  const int blk = h * 4 + c4;
+  const int sw = (blk >> 1) & 3;
+  return blk * 64 + (((kk >> 1) ^ sw) << 4) + (kk & 1) * 8 + e * 2;
 }
 
+template <int RK>
 __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk, uint32_t* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -157,18 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     }
     for (int b = 0; b < kNB; ++b) {
       mbar_init(&bars.tile_in[b], 4);
-      mbar_init(&bars.v_done[b], 1);
       mbar_init(&bars.alk_free[b], 1);
+      mbar_init(&bars.lv_free[b], kEpiWarps);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kNDr; ++b) {
       mbar_init(&bars.recon_done[b], 1);
-      mbar_init(&bars.kq_full[b], 256);
-      mbar_init(&bars.score_done[b], 1);
-      mbar_init(&bars.p_full[b], 256);
-      mbar_init(&bars.epi_sync[b], 128);
-      for (int k = 0; k < 3; ++k) bars.flag[b][k] = 0;
+      mbar_init(&bars.dr_free[b], kEpiWarps);
     }
-    mbar_init(&bars.acc_free, 256);
     mbar_init(&bars.mma_drain, 1);
     bars.abort = 0;
     fence_mbar_init();
@@ -177,9 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // static zeros of the operand buffers (padding heads / rows)
-  for (int i = threadIdx.x; i < (2 * 4096 + kNB * 16384 + 2 * 4096) / 16; i += kThreads)
-    reinterpret_cast<uint4*>(sm + kSmQ)[i] = make_uint4(0, 0, 0, 0);
+  // zero the L_v tiles and query fragments once: the pad columns, ranks >= rv
+  // and the padding heads 4..7 stay zero (L_v and the fragments are adjacent)
+  static_assert(kSmQF == kSmLV + kNB * kLvBytes, "L_v and query fragments must be adjacent");
+  for (int i = threadIdx.x; i < (kNB * kLvBytes + kNB * kQfBytes) / 16; i += kThreads)
+    reinterpret_cast<uint4*>(sm + kSmLV)[i] = make_uint4(0, 0, 0, 0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -188,12 +209,12 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
   if (warp == kWarpProd) {
     // ------------------------------------------------------------ producer
     int issued_upto = 0;  // tiles issued
-    for (int jj = 0; jj < n_tiles && !*abort; ++jj) {
-      const int s = jj % kStages;
-      if (!mbar_wait(&bars.empty[s], ((jj / kStages) & 1) ^ 1, abort, err)) break;
-      int u, jt, nt;
-      unit_of(p, wk, t_first + jj, &u, &jt, &nt);
-      const size_t row0 = (size_t)u * p.tmax + (size_t)jt * kTile;
+    TileCursor cur(t_first, wk.tpu);
+    for (int jj = 0; jj < n_tiles && !*abort; ++jj, cur.next()) {
+      const int s = slot_of<kStagesLog2>(jj);
+      if (!mbar_wait(&bars.empty[s], phase_of<kStagesLog2>(jj) ^ 1, abort, err)) break;
+      const int nt = cur.valid_rows(p.n_tokens);
+      const size_t row0 = (size_t)cur.u * p.tmax + (size_t)cur.jt * kTile;
       uint8_t* st = sm + kSmStage + s * kStageMax;
       const uint8_t* src[4] = {p.lk + row0 * lk_row,
                                reinterpret_cast<const uint8_t*>(p.lksz) + row0 * lksz_row,
@@ -231,79 +252,25 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     if (*abort && lane == 0) {
       for (int jj = max(0, issued_upto - kStages); jj < issued_upto; ++jj) {
         volatile int no_abort = 0;
-        mbar_wait(&bars.full[jj % kStages], (jj / kStages) & 1, &no_abort, nullptr);
+        mbar_wait(&bars.full[slot_of<kStagesLog2>(jj)], phase_of<kStagesLog2>(jj), &no_abort, nullptr);
       }
     }
   } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issue
-    // Non-blocking scheduler: issue whichever of (value nv, score ns,
-    // reconstruction nr) is ready, in tile order within each kind.  recon(nr)
-    // overwrites the K_hat buffer of tile nr - 2, which the epilogue has read
-    // once score(nr - 2) could be issued.
+    // ------------------------------------------------------------ reconstruction MMAs
     if (lane == 0) {
-      const uint32_t id_recon = idesc_f16(kTile, kD, 0, 0);
-      const uint32_t id_score = idesc_f16(kTile, kN, 0, 0);
-      const uint32_t id_val = idesc_f16(kVM, kN, 1, 1);
-      const int ksteps_recon = p.rk / 16;
-      int nr = 0, ns = 0, nv = 0;
-      int v_unit = -1, v_started = 0;
-      uint64_t idle_since = 0;
-      uint32_t idle = 0;
-      while (nv < n_tiles) {
-        bool prog = false;
-        if (nv < ns && mbar_test(&bars.p_full[nv & 1], (nv >> 1) & 1)) {
-          int u, jt, nt;
-          unit_of(p, wk, t_first + nv, &u, &jt, &nt);
-          const bool first = u != v_unit;
-          bool ready = true;
-          if (first && v_started > 0) ready = mbar_test(&bars.acc_free, (v_started - 1) & 1);
-          if (ready) {
-            if (first) v_unit = u, ++v_started;
-            const int bd = nv % kNB, pb = nv & 1;
-            tc_fence_after();
-            for (int kk = 0; kk < kTile / 16; ++kk)
-              mma_ss(tmem + kColAcc, smem_desc(sm + kSmLV + bd * 16384 + kk * 256, 128, 2048),
-                     smem_desc(sm + kSmP + pb * 4096 + kk * 256, 128, 2048), id_val,
-                     (first && kk == 0) ? 0u : 1u);
-            tc_commit(&bars.v_done[bd]);
-            ++nv;
-            prog = true;
-          }
-        }
-        if (ns < nr && mbar_test(&bars.kq_full[ns & 1], (ns >> 1) & 1)) {
-          const int sb = ns & 1;
-          tc_fence_after();
-          for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ts(tmem + kColS + sb * 16, tmem + kColAK + sb * 64 + kk * 8,
-                   smem_desc(sm + kSmQ + sb * 4096 + kk * 256, 128, 2048), id_score, kk > 0);
-          tc_commit(&bars.score_done[sb]);
-          ++ns;
-          prog = true;
-        }
-        if (nr < n_tiles && nr - ns < 2 &&
-            mbar_test(&bars.tile_in[nr % kNB], (nr / kNB) & 1)) {
-          const int kb = nr & 1, bd = nr % kNB;
-          tc_fence_after();
-          for (int kk = 0; kk < ksteps_recon; ++kk)
-            mma_ts(tmem + kColDr + kb * 128, tmem + kColALk + bd * 16 + kk * 8,
-                   smem_desc(sm + kSmBk + kk * 256, 128, 512), id_recon, kk > 0);
-          tc_commit(&bars.recon_done[kb]);
-          tc_commit(&bars.alk_free[bd]);
-          ++nr;
-          prog = true;
-        }
-        if (prog) {
-          idle = 0;
-        } else if ((++idle & 255u) == 0) {
-          if (*abort) break;
-          const uint64_t now = globaltimer();
-          if (idle == 256) idle_since = now;
-          else if (now - idle_since > kWaitLimitNs) {
-            *abort = 1;
-            atomicOr(err, kErrTimeout);
-            break;
-          }
-        }
+      const uint32_t id_recon = idesc_f16(kTile, kD, 0, 0, /*d_f16=*/1);
+      for (int nr = 0; nr < n_tiles; ++nr) {
+        const int kb = dr_slot(nr), bd = slot_of<kNBLog2>(nr);
+        if (!mbar_wait(&bars.tile_in[bd], phase_of<kNBLog2>(nr), abort, err)) break;
+        // the K_hat buffer of tile nr - kNDr has been read by every epilogue warp
+        if (nr >= kNDr && !mbar_wait(&bars.dr_free[kb], dr_phase(nr - kNDr), abort, err)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < RK / 16; ++kk)
+          mma_ts(tmem + kColDr + kb * 128, tmem + kColALk + bd * 16 + kk * 8,
+                 smem_desc(sm + kSmBk + kk * 256, 128, 512), id_recon, kk > 0);
+        tc_commit(&bars.recon_done[kb]);
+        tc_commit(&bars.alk_free[bd]);
       }
       // every MMA this thread issued must complete before TMEM is released
       tc_commit(&bars.mma_drain);
@@ -311,80 +278,136 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       mbar_wait(&bars.mma_drain, 0, &no_abort, nullptr);
     }
     __syncwarp();
-  } else if (warp >= kWarpDeq) {
-    // ------------------------------------------------------------ dequantization
+  } else if (warp < kWarpEpi) {
+    // ------------------------------------------------------------ dequantization + q_rot
     const int q4 = warp & 3;                 // TMEM lane quadrant
     const int row = 32 * q4 + lane;          // token row in the tile
-    int cur_u = -1;
-    const __half2 one_h2 = __floats2half2_rn(1.f, 0.f);
-    for (int jj = 0; jj < n_tiles; ++jj) {
-      int u, jt, nt;
-      unit_of(p, wk, t_first + jj, &u, &jt, &nt);
-      const int bd = jj % kNB, s = jj % kStages;
-      if (u != cur_u) {
-        if (jj > 0 && !mbar_wait(&bars.alk_free[(jj - 1) % kNB], ((jj - 1) / kNB) & 1, abort, err))
+    const int dt = threadIdx.x - 32 * kWarpDeq;   // 0..127
+    const bool qrot_warp = warp == kWarpDeq;
+    // q_rot: lane m of the first dequant warp rotates pairs 2m, 2m + 1.  The
+    // angle of pair i at t0 = 128 jt is jt * frac(128 f_i) turns; frac(128 f_i)
+    // is held in 32-bit fixed point so that jt * F mod 2^32 is exact.
+    uint32_t Fq[2];
+    float qv[kG][4];                         // q[h][2m], [2m+1], [2m+64], [2m+65] * scale
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      double x = 128.0 * p.rope_f[(2 * lane + e) & (kHalf - 1)];
+      x -= floor(x);
+      Fq[e] = (uint32_t)(unsigned long long)llrint(x * 4294967296.0);
+    }
+#pragma unroll
+    for (int h = 0; h < kG; ++h) qv[h][0] = qv[h][1] = qv[h][2] = qv[h][3] = 0.f;
+    TileCursor cur(t_first, wk.tpu);
+    for (int jj = 0; jj < n_tiles; ++jj, cur.next()) {
+      const int nt = cur.valid_rows(p.n_tokens);
+      const int bd = slot_of<kNBLog2>(jj), s = slot_of<kStagesLog2>(jj);
+      if (jj == 0 || cur.jt == 0) {
+        // new unit: Bk is rewritten once the previous tile's recon is done
+        if (jj > 0 && !mbar_wait(&bars.alk_free[slot_of<kNBLog2>(jj - 1)], phase_of<kNBLog2>(jj - 1),
+                                 abort, err))
           break;
+        const int kvh = cur.u % p.Hkv, b = cur.u / p.Hkv;
         // B operand of the reconstruction: N = 128 dims x K = rk (logical ranks),
         // K-major core matrices, logical k holds Bk row perm_rank(k)
-        const int kvh = u % p.Hkv;
-        const __half* bk = p.bk + (size_t)kvh * p.rk * kD;
+        const __half* bk = p.bk + (size_t)kvh * RK * kD;
         __half* dst = reinterpret_cast<__half*>(sm + kSmBk);
-        for (int e = threadIdx.x - 32 * kWarpDeq; e < p.rk * kD; e += 128) {
+        for (int e = dt; e < RK * kD; e += 128) {
           const int k = e / kD, n = e % kD;
           dst[((n >> 3) * 512 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) / 2] =
               bk[(size_t)perm_rank(k) * kD + n];
         }
         fence_proxy_async_smem();
-        cur_u = u;
-      }
-      if (!mbar_wait(&bars.full[s], (jj / kStages) & 1, abort, err)) break;
-      if (jj >= kNB) {
-        // recon(jj - kNB) read this A buffer, value(jj - kNB) this L_v buffer
-        if (!mbar_wait(&bars.alk_free[bd], ((jj - kNB) / kNB) & 1, abort, err)) break;
-        if (!mbar_wait(&bars.v_done[bd], ((jj - kNB) / kNB) & 1, abort, err)) break;
-      }
-      tc_fence_after();
-      const bool valid = row < nt;
-      const uint8_t* st = sm + kSmStage + s * kStageMax;
-      // ---- keys: rk/8 words -> TMEM columns (A operand of the reconstruction)
-      uint32_t ka[16];
-      {
-        const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + row * lk_row);
-        const __half2* sz = reinterpret_cast<const __half2*>(st + kTile * lk_row + row * lksz_row);
-        const __half2 sz0 = sz[0];
-        const __half2 s2 = __low2half2(sz0), z2 = __high2half2(sz0);
+        if (qrot_warp) {
+          const __nv_bfloat16* qq = p.q + ((size_t)b * p.Hq + kvh * kG) * kD;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (j < p.rk / 8 && valid) {
-            dequant_word(codes[j], s2, z2, ka + 4 * j);
-          } else {
-            ka[4 * j] = ka[4 * j + 1] = ka[4 * j + 2] = ka[4 * j + 3] = 0u;
+          for (int h = 0; h < kG; ++h) {
+            qv[h][0] = bf2f(qq[h * kD + 2 * lane]) * p.scale_log2;
+            qv[h][1] = bf2f(qq[h * kD + 2 * lane + 1]) * p.scale_log2;
+            qv[h][2] = bf2f(qq[h * kD + 2 * lane + kHalf]) * p.scale_log2;
+            qv[h][3] = bf2f(qq[h * kD + 2 * lane + kHalf + 1]) * p.scale_log2;
           }
         }
       }
-      tmem_st16(tmem + ((uint32_t)(32 * q4) << 16) + kColALk + bd * 16, ka);
-      // ---- values: rv/8 words -> shared memory (A of the value MMA, MN-major)
+      if (!mbar_wait(&bars.full[s], phase_of<kStagesLog2>(jj), abort, err)) break;
+      if (jj >= kNB) {
+        // recon(jj - kNB) read this A buffer; the epilogue warps are done with
+        // this L_v / q_rot buffer
+        if (!mbar_wait(&bars.alk_free[bd], phase_of<kNBLog2>(jj - kNB), abort, err)) break;
+        if (!mbar_wait(&bars.lv_free[bd], phase_of<kNBLog2>(jj - kNB), abort, err)) break;
+      }
+      tc_fence_after();
+      // rows past the end get scale = zero = 0 (bitwise: the stage bytes of
+      // such rows are stale and may hold any fp16 pattern), hence zero latents
+      const uint32_t vmask = row < nt ? 0xFFFFFFFFu : 0u;
+      const uint8_t* st = sm + kSmStage + s * kStageMax;
+      // ---- keys: rk/8 words -> TMEM columns (A operand of the reconstruction)
+      {
+        uint32_t cw[RK / 8];
+        if constexpr (RK == 32) {
+          const uint4 v = *reinterpret_cast<const uint4*>(st + row * (RK / 2));
+          cw[0] = v.x;
+          cw[1] = v.y;
+          cw[2] = v.z;
+          cw[3] = v.w;
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2*>(st + row * (RK / 2));
+          cw[0] = v.x;
+          cw[1] = v.y;
+        }
+        const uint32_t szw =
+            *reinterpret_cast<const uint32_t*>(st + kTile * (RK / 2) + row * lksz_row) & vmask;
+        const __half2 sz0 = *reinterpret_cast<const __half2*>(&szw);
+        const __half2 s2 = __low2half2(sz0), z2 = __high2half2(sz0);
+        uint32_t ka[RK / 2];
+#pragma unroll
+        for (int j = 0; j < RK / 8; ++j) dequant_word(cw[j], s2, z2, ka + 4 * j);
+        const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + kColALk + bd * 16;
+        if constexpr (RK == 32) tmem_st16(ta, ka);
+        else tmem_st8(ta, ka);
+      }
+      // ---- values: rv/8 words -> shared memory rows [token][logical rank]
       {
         const uint8_t* vbase = st + kTile * (lk_row + lksz_row);
         const uint32_t* codes = reinterpret_cast<const uint32_t*>(vbase + row * lv_row);
-        const __half2* sz = reinterpret_cast<const __half2*>(vbase + kTile * lv_row + row * lvsz_row);
-        uint8_t* lv = sm + kSmLV + bd * 16384 + (row >> 3) * 128 + (row & 7) * 16;
-        for (int j = 0; j < rv / 8; ++j) {
-          uint32_t r[4] = {0u, 0u, 0u, 0u};
-          if (valid) {
-            const __half2 szg = sz[j / 4];          // group of 32 ranks = 4 words
-            dequant_word(codes[j], __low2half2(szg), __high2half2(szg), r);
+        const uint32_t* sz = reinterpret_cast<const uint32_t*>(vbase + kTile * lv_row + row * lvsz_row);
+        uint8_t* lv = sm + kSmLV + bd * kLvBytes + row * (kLvStride * 2);
+        // all loads first (words past rv read neighbouring bytes of the stage
+        // and are dropped), then branch-free dequantization
+        uint32_t vw[kRvMax / 8];
+#pragma unroll
+        for (int j = 0; j < kRvMax / 8; ++j) vw[j] = codes[j];
+        const uint32_t gw[2] = {sz[0] & vmask, sz[1] & vmask};   // groups of 32 ranks
+#pragma unroll
+        for (int j = 0; j < kRvMax / 8; ++j) {
+          if (j < rv / 8) {
+            const __half2 szg = *reinterpret_cast<const __half2*>(&gw[j < 4 ? 0 : 1]);
+            uint32_t r[4];
+            dequant_word(vw[j], __low2half2(szg), __high2half2(szg), r);
+            *reinterpret_cast<uint4*>(lv + j * 16) = make_uint4(r[0], r[1], r[2], r[3]);
           }
-          *reinterpret_cast<uint4*>(lv + j * 2048) = make_uint4(r[0], r[1], r[2], r[3]);
         }
-        // the constant-one row (logical rank rv) sums P into the softmax denominator
-        const __half2 on = valid ? one_h2 : __floats2half2_rn(0.f, 0.f);
-        *reinterpret_cast<uint4*>(lv + (rv / 8) * 2048) =
-            make_uint4(*reinterpret_cast<const uint32_t*>(&on), 0u, 0u, 0u);
+      }
+      // ---- q_rot = R_t0^T q (times the softmax scale) as score-MMA B fragments
+      if (qrot_warp) {
+        float ca[2], sa[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int turns = (int)((uint32_t)cur.jt * Fq[e]);      // in 2^-32 turns
+          __sincosf((float)turns * 1.4629180792671596e-09f, &sa[e], &ca[e]);   // 2 pi / 2^32
+        }
+        uint8_t* qf = sm + kSmQF + bd * kQfBytes;
+#pragma unroll
+        for (int h = 0; h < kG; ++h) {
+          const float lo0 = ca[0] * qv[h][0] + sa[0] * qv[h][2];
+          const float lo1 = ca[1] * qv[h][1] + sa[1] * qv[h][3];
+          const float hi0 = ca[0] * qv[h][2] - sa[0] * qv[h][0];
+          const float hi1 = ca[1] * qv[h][3] - sa[1] * qv[h][1];
+          *reinterpret_cast<uint32_t*>(qf + qf_offset(h, 2 * lane)) = pack_h2(lo0, lo1);
+          *reinterpret_cast<uint32_t*>(qf + qf_offset(h, 2 * lane + kHalf)) = pack_h2(hi0, hi1);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
-      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bars.empty[s]);
@@ -392,220 +415,224 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue
-    const int h = (warp - kWarpEpi) >> 2;    // group: RoPE pairs 32h.., heads 2h, 2h+1
-    const int ew = (warp - kWarpEpi) & 3;    // warp index within the group
-    const int q4 = warp & 3;
-    const int row = 32 * q4 + lane;
-    const int gtid = ew * 32 + lane;         // 0..127 within the group
-    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-    // RoPE rotation of this row (delta = row) for the group's pairs, as f16x2
-    // over consecutive frequencies (i, i + 1), i = 32h + 2k
-    uint32_t cs[16], sn[16];
+    // ------------------------------------------------------------ epilogue warps
+    const int ew = warp - kWarpEpi;          // partial index of this warp
+    const int q4 = warp & 3;                 // this warp's TMEM lane quadrant
+    const int m_base = 32 * q4 + 16 * (ew >> 2);   // inside the warp's lane quadrant
+    const int g = lane >> 2, c4 = lane & 3;  // fragment row / column group
+    const int r0 = m_base + g, r1 = r0 + 8;  // the two rows this thread holds
+    const uint32_t taddr0 = tmem + ((uint32_t)m_base << 16);
+    // RoPE rotation R_delta of rows r0 and r1 for the pairs this thread holds:
+    // dims i = 16 kk + 4 c4 + {0,1} (hf 0) and {2,3} (hf 1), kk = 0..3, against
+    // i + 64, as f16x2 over the two dims
+    uint32_t cs[4][2][2], sn[4][2][2];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      float c0, s0, c1, s1;
-      const int i = 32 * h + 2 * k;
-      const double t0 = (double)row * p.rope_f[i], t1 = (double)row * p.rope_f[i + 1];
-      sincospif(2.f * (float)(t0 - rint(t0)), &s0, &c0);
-      sincospif(2.f * (float)(t1 - rint(t1)), &s1, &c1);
-      cs[k] = pack_h2(c0, c1);
-      sn[k] = pack_h2(s0, s1);
-    }
-    // q-side rotation: this thread rotates pair qi of head qh
-    const int qi = 32 * h + (gtid & 31), qh = gtid >> 5;
-    float qlo = 0.f, qhi = 0.f;
-    int rope_u = -1;
-    // softmax state of the group's two heads
-    float m_ref[2] = {-INFINITY, -INFINITY};
-    int sm_u = -1, sm_b = 0, sm_kvh = 0, sm_slot = 0, sm_last = -1;
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int i = 16 * kk + 4 * c4 + 2 * hf;
+          const int delta = rr ? r1 : r0;
+          float c0, s0, c1, s1;
+          double t0 = (double)delta * p.rope_f[i], t1 = (double)delta * p.rope_f[i + 1];
+          t0 -= rint(t0);
+          t1 -= rint(t1);
+          __sincosf(6.283185307179586f * (float)t0, &s0, &c0);
+          __sincosf(6.283185307179586f * (float)t1, &s1, &c1);
+          cs[kk][hf][rr] = pack_h2(c0, c1);
+          sn[kk][hf][rr] = pack_h2(s0, s1);
+        }
+    // query-fragment block of this thread (g = head; heads 4..7 are zero)
+    const int qblk = g * 4 + c4;
+    const int qsw = (qblk >> 1) & 3;
+    // ldmatrix row address of this lane in an L_v buffer
+    const int lv_off = (m_base + (lane & 7) + ((lane >> 4) << 3)) * (kLvStride * 2) +
+                       ((lane >> 3) & 1) * 16;
+    // per-warp softmax state for heads 2*c4, 2*c4 + 1 (real heads when c4 < 2)
+    float m_ref[2], m_thr[2], l_sum[2];
+    float acc[3][4];
+    int cur_b = 0, cur_kvh = 0, cur_slot = 0;
     const size_t rows_q = (size_t)p.B * p.Hq;
     const int pst = p.vdim + 2;
-    uint32_t epi_phase = 0;
-    auto epi_sync = [&]() -> bool {
-      mbar_arrive(&bars.epi_sync[h]);
-      const bool r = mbar_wait(&bars.epi_sync[h], epi_phase & 1, abort, err);
-      ++epi_phase;
-      return r;
+    auto reset = [&]() {
+      m_ref[0] = m_ref[1] = -INFINITY;
+      m_thr[0] = m_thr[1] = -INFINITY;
+      l_sum[0] = l_sum[1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 3; ++mt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[mt][k] = 0.f;
     };
-    // the accumulator of the finished unit -> partials of the group's heads
-    auto finish_unit = [&](int jj_last) -> bool {
-      if (!mbar_wait(&bars.v_done[jj_last % kNB], (jj_last / kNB) & 1, abort, err)) return false;
-      tc_fence_after();
-      uint32_t r[2];
-      tmem_ld2(tmem + lane_base + kColAcc + 2 * h, r);
-      tmem_wait_ld();
-      reg_fence(r);
-      if (lane < 16) {
-        const int m = 16 * q4 + lane;          // logical value row
+    // partial of this warp for the finished unit
+    auto write_partial = [&]() {
+      float l0 = l_sum[0], l1 = l_sum[1];
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      }
+      if (c4 < 2) {
+        const int slot = cur_slot * kEpiWarps + ew;
+#pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const size_t qr = (size_t)sm_b * p.Hq + sm_kvh * kG + 2 * h + e;
-          float* dst = p.part + ((size_t)sm_slot * rows_q + qr) * pst;
-          const float v = __uint_as_float(r[e]);
-          if (m < rv) dst[perm_rank(m)] = v;
-          else if (m == rv) {
+          const size_t qr = (size_t)cur_b * p.Hq + cur_kvh * kG + 2 * c4 + e;
+          float* dst = p.part + ((size_t)slot * rows_q + qr) * pst;
+#pragma unroll
+          for (int mt = 0; mt < 3; ++mt) {
+            const int m0 = 16 * mt + g;
+            if (m0 < rv) dst[perm_rank(m0)] = acc[mt][e];
+            if (m0 + 8 < rv) dst[perm_rank(m0 + 8)] = acc[mt][2 + e];
+          }
+          if (g == 0) {
             dst[p.vdim] = m_ref[e];
-            dst[p.vdim + 1] = v;
+            dst[p.vdim + 1] = e ? l1 : l0;
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bars.acc_free);
+    };
+
+    // K_hat of this warp's 16 rows of tile jj (f16, four 32-column loads),
+    // issued one tile ahead so that the TMEM latency hides behind softmax + V
+    uint32_t klo[2][8], khi[2][8];
+    auto issue_k = [&](int jj) -> bool {
+      const int kb = dr_slot(jj);
+      if (!mbar_wait(&bars.recon_done[kb], dr_phase(jj), abort, err)) return false;
+      tc_fence_after();
+      const uint32_t dr = taddr0 + kColDr + kb * 128;
+      tmem_ld16x256_x2_pack16(dr + 0, klo[0]);
+      tmem_ld16x256_x2_pack16(dr + 32, klo[1]);
+      tmem_ld16x256_x2_pack16(dr + kHalf, khi[0]);
+      tmem_ld16x256_x2_pack16(dr + kHalf + 32, khi[1]);
       return true;
     };
 
-    // ---- stage 1: q_rot and RoPE of the reconstructed keys (in place)
-    auto rope_stage = [&](int jj) -> bool {
-      int u, jt, nt;
-      unit_of(p, wk, t_first + jj, &u, &jt, &nt);
-      if (u != rope_u) {
-        rope_u = u;
-        const __nv_bfloat16* qq =
-            p.q + ((size_t)(u / p.Hkv) * p.Hq + (u % p.Hkv) * kG + qh) * kD;
-        qlo = bf2f(qq[qi]);
-        qhi = bf2f(qq[qi + kHalf]);
+    bool ok = n_tiles > 0 && issue_k(0);
+    TileCursor cur(t_first, wk.tpu);
+    for (int jj = 0; jj < n_tiles && ok; ++jj, cur.next()) {
+      const int nt = cur.valid_rows(p.n_tokens);
+      if (jj == 0 || cur.jt == 0) {
+        if (jj > 0) write_partial();
+        reset();
+        cur_b = cur.u / p.Hkv;
+        cur_kvh = cur.u % p.Hkv;
+        cur_slot = cta - (int)(((long long)cur.u * wk.tpu) / wk.W);
       }
-      {
-        // q_rot = R_t0^T q (B operand of the score MMA); this buffer was last
-        // read by score(jj - 2), whose completion the softmax stage of jj - 2 saw
-        const double turns = (double)(jt * kTile) * p.rope_f[qi];
-        float sa, ca;
-        sincospif(2.f * (float)(turns - rint(turns)), &sa, &ca);
-        __half* qd = reinterpret_cast<__half*>(sm + kSmQ + (jj & 1) * 4096);
-        const float rl = ca * qlo + sa * qhi;
-        const float rh = ca * qhi - sa * qlo;
-        qd[((qh >> 3) * 2048 + (qi >> 3) * 128 + (qh & 7) * 16 + (qi & 7) * 2) / 2] =
-            __float2half_rn(rl);
-        const int qj = qi + kHalf;
-        qd[((qh >> 3) * 2048 + (qj >> 3) * 128 + (qh & 7) * 16 + (qj & 7) * 2) / 2] =
-            __float2half_rn(rh);
-      }
-      if (!mbar_wait(&bars.recon_done[jj & 1], (jj >> 1) & 1, abort, err)) return false;
-      tc_fence_after();
-      // K_hat (fp32, column = dim) -> K'' (f16x2, column c = dims 2c, 2c+1).
-      // This group rotates the low dims 32h..32h+31 against 64+32h..64+32h+31,
-      // in two halves of 16 pairs.
-      const uint32_t dr = tmem + lane_base + kColDr + (jj & 1) * 128;
-      const uint32_t ak = tmem + lane_base + kColAK + (jj & 1) * 64;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t lo[16], hi[16];
-        tmem_ld16(dr + 32 * h + 16 * half, lo);
-        tmem_ld16(dr + kHalf + 32 * h + 16 * half, hi);
-        tmem_wait_ld();
-        reg_fence(lo);
-        reg_fence(hi);
-        uint32_t xo[8], yo[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const __half2 x = __floats2half2_rn(__uint_as_float(lo[2 * k]), __uint_as_float(lo[2 * k + 1]));
-          const __half2 y = __floats2half2_rn(__uint_as_float(hi[2 * k]), __uint_as_float(hi[2 * k + 1]));
-          const __half2 C = *reinterpret_cast<const __half2*>(&cs[8 * half + k]);
-          const __half2 S = *reinterpret_cast<const __half2*>(&sn[8 * half + k]);
-          const __half2 xr = __hfma2(C, x, __hneg2(__hmul2(S, y)));   // k_i cos - k_{i+64} sin
-          const __half2 yr = __hfma2(C, y, __hmul2(S, x));            // k_{i+64} cos + k_i sin
-          xo[k] = *reinterpret_cast<const uint32_t*>(&xr);
-          yo[k] = *reinterpret_cast<const uint32_t*>(&yr);
-        }
-        tmem_st8(ak + 16 * h + 8 * half, xo);
-        tmem_st8(ak + 32 + 16 * h + 8 * half, yo);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      fence_proxy_async_smem();
-      mbar_arrive(&bars.kq_full[jj & 1]);
-      return true;
-    };
-
-    // ---- stage 2: scores, online softmax, P
-    auto softmax_stage = [&](int jj) -> bool {
-      int u, jt, nt;
-      unit_of(p, wk, t_first + jj, &u, &jt, &nt);
-      if (u != sm_u) {
-        if (sm_u >= 0 && !finish_unit(sm_last)) return false;
-        sm_u = u;
-        sm_b = u / p.Hkv;
-        sm_kvh = u % p.Hkv;
-        sm_slot = cta - (int)(((long long)u * wk.tpu) / wk.W);
-        m_ref[0] = m_ref[1] = -INFINITY;
-      }
-      const int sb = jj & 1;
-      if (!mbar_wait(&bars.score_done[sb], (jj >> 1) & 1, abort, err)) return false;
-      tc_fence_after();
-      uint32_t sr[2];
-      tmem_ld2(tmem + lane_base + kColS + sb * 16 + 2 * h, sr);
+      const int kb = dr_slot(jj), bd = slot_of<kNBLog2>(jj);
+      if (!(ok = mbar_wait(&bars.tile_in[bd], phase_of<kNBLog2>(jj), abort, err))) break;
       tmem_wait_ld();
-      reg_fence(sr);
-      const bool valid = row < nt;
-      float s2[2];
-      bool need = false;
+      reg_fence(klo[0]);
+      reg_fence(klo[1]);
+      reg_fence(khi[0]);
+      reg_fence(khi[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.dr_free[kb]);
+      // ---- q_rot fragments (heads 0..3 in lanes 0..15; lanes 16..31 read the
+      // buffer's zero blocks of the padding heads 4..7)
+      uint32_t qb[8][2];
+      {
+        const uint4* qf = reinterpret_cast<const uint4*>(sm + kSmQF + bd * kQfBytes + qblk * 64);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        s2[e] = valid ? __uint_as_float(sr[e]) * p.scale_log2 : -INFINITY;
-        need |= s2[e] > m_ref[e] + 8.f;
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x = qf[v ^ qsw];
+          qb[2 * v][0] = x.x;
+          qb[2 * v][1] = x.y;
+          qb[2 * v + 1][0] = x.z;
+          qb[2 * v + 1][1] = x.w;
+        }
       }
-      // P buffer sb was read by value(jj - 2)
-      if (jj >= 2 && !mbar_wait(&bars.v_done[(jj - 2) % kNB], ((jj - 2) / kNB) & 1, abort, err))
-        return false;
-      // a flag is reset two tiles after its last read (every thread of the
-      // group has passed the synchronisation in between)
-      const int fl = jj % 3;
-      if (gtid == 0) bars.flag[h][(jj + 1) % 3] = 0;
-      if (__any_sync(0xffffffffu, need) && lane == 0) atomicOr(&bars.flag[h][fl], 1);
-      if (!epi_sync()) return false;
-      if (bars.flag[h][fl]) {
-        // raise the reference maximum to the tile maximum, rescale acc
+      // ---- RoPE in registers, then the score MMA (k steps kk and kk + 4, two
+      // independent accumulator chains)
+      float sc[4] = {0.f, 0.f, 0.f, 0.f}, sh[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float tm = warp_max(s2[e]);
-          if (lane == 0) bars.wmax[h][ew][e] = tm;
-        }
-        if (!epi_sync()) return false;
-        float alpha[2];
-        bool any_scale = false;
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t xr[4], yr[4];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float mt = fmaxf(fmaxf(bars.wmax[h][0][e], bars.wmax[h][1][e]),
-                                 fmaxf(bars.wmax[h][2][e], bars.wmax[h][3][e]));
-          const float mn = fmaxf(m_ref[e], mt);
-          alpha[e] = (m_ref[e] == -INFINITY) ? 1.f : exp2f(m_ref[e] - mn);
-          any_scale |= (m_ref[e] != -INFINITY) && (mn > m_ref[e]);
-          m_ref[e] = mn;
+        for (int r = 0; r < 4; ++r) {            // r: (row r >> 1, dims pair-couple r & 1)
+          const __half2 x = *reinterpret_cast<const __half2*>(&klo[kk >> 1][4 * (kk & 1) + r]);
+          const __half2 y = *reinterpret_cast<const __half2*>(&khi[kk >> 1][4 * (kk & 1) + r]);
+          const __half2 C = *reinterpret_cast<const __half2*>(&cs[kk][r & 1][r >> 1]);
+          const __half2 S = *reinterpret_cast<const __half2*>(&sn[kk][r & 1][r >> 1]);
+          const __half2 xo = __hfma2(C, x, __hneg2(__hmul2(S, y)));   // k_i cos - k_{i+64} sin
+          const __half2 yo = __hfma2(C, y, __hmul2(S, x));            // k_{i+64} cos + k_i sin
+          xr[r] = *reinterpret_cast<const uint32_t*>(&xo);
+          yr[r] = *reinterpret_cast<const uint32_t*>(&yo);
         }
-        // while m_ref was -inf there is no earlier value MMA of this unit;
-        // any_scale is the same in every thread of the group
-        if (any_scale) {
-          if (!mbar_wait(&bars.v_done[(jj - 1) % kNB], ((jj - 1) / kNB) & 1, abort, err))
-            return false;
-          tc_fence_after();
-          uint32_t r[2];
-          tmem_ld2(tmem + lane_base + kColAcc + 2 * h, r);
-          tmem_wait_ld();
-          reg_fence(r);
-          r[0] = __float_as_uint(__uint_as_float(r[0]) * alpha[0]);
-          r[1] = __float_as_uint(__uint_as_float(r[1]) * alpha[1]);
-          tmem_st2(tmem + lane_base + kColAcc + 2 * h, r);
-          tmem_wait_st();
-          tc_fence_before();
-        }
-        if (!epi_sync()) return false;   // wmax is read by everyone before it is reused
+        const uint32_t alo[4] = {xr[0], xr[2], xr[1], xr[3]};
+        const uint32_t ahi[4] = {yr[0], yr[2], yr[1], yr[3]};
+        mma16816(sc, alo, qb[kk][0], qb[kk][1]);
+        mma16816(sh, ahi, qb[kk + 4][0], qb[kk + 4][1]);
       }
-      const float p0 = valid ? exp2f(s2[0] - m_ref[0]) : 0.f;
-      const float p1 = valid ? exp2f(s2[1] - m_ref[1]) : 0.f;
-      *reinterpret_cast<uint32_t*>(sm + kSmP + sb * 4096 + (row >> 3) * 128 + (row & 7) * 16 +
-                                   4 * h) = pack_h2(p0, p1);
-      fence_proxy_async_smem();
-      mbar_arrive(&bars.p_full[sb]);
-      sm_last = jj;
-      return true;
-    };
-
-    bool ok = true;
-    for (int jj = 0; jj <= n_tiles && ok; ++jj) {
-      if (jj < n_tiles) ok = rope_stage(jj);
-      if (ok && jj >= 1) ok = softmax_stage(jj - 1);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sc[i] += sh[i];
+      // next tile's K_hat loads fly while this tile finishes
+      if (jj + 1 < n_tiles && !(ok = issue_k(jj + 1))) break;
+      // ---- online softmax of this warp (rows r0, r1; heads 2c4, 2c4 + 1);
+      // scores are already in log2 units (the scale is folded into q_rot)
+      if (nt < kTile) {
+        if (r0 >= nt) sc[0] = sc[1] = -INFINITY;
+        if (r1 >= nt) sc[2] = sc[3] = -INFINITY;
+      }
+      const bool need = sc[0] > m_thr[0] || sc[2] > m_thr[0] || sc[1] > m_thr[1] ||
+                        sc[3] > m_thr[1];
+      if (__any_sync(0xffffffffu, need)) {
+        float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float n0 = fmaxf(m_ref[0], mx0), n1 = fmaxf(m_ref[1], mx1);
+        // a = 2^(m_old - m_new); 0 for a first maximum (m_old = -inf)
+        const float a0 = ex2_approx(m_ref[0] - n0), a1 = ex2_approx(m_ref[1] - n1);
+        l_sum[0] *= a0;
+        l_sum[1] *= a1;
+#pragma unroll
+        for (int mt = 0; mt < 3; ++mt) {
+          acc[mt][0] *= a0;
+          acc[mt][2] *= a0;
+          acc[mt][1] *= a1;
+          acc[mt][3] *= a1;
+        }
+        m_ref[0] = n0;
+        m_ref[1] = n1;
+        m_thr[0] = n0 + 8.f;
+        m_thr[1] = n1 + 8.f;
+      }
+      float pv[4];
+      pv[0] = ex2_approx(sc[0] - m_ref[0]);
+      pv[1] = ex2_approx(sc[1] - m_ref[1]);
+      pv[2] = ex2_approx(sc[2] - m_ref[0]);
+      pv[3] = ex2_approx(sc[3] - m_ref[1]);
+      if (nt < kTile) {
+        // rows past the end weigh nothing, also while no row of this warp has
+        // been seen (-inf - -inf would give NaN)
+        if (r0 >= nt) pv[0] = pv[1] = 0.f;
+        if (r1 >= nt) pv[2] = pv[3] = 0.f;
+      }
+      l_sum[0] += pv[0] + pv[2];
+      l_sum[1] += pv[1] + pv[3];
+      // P as the B operand (k = token, n = head): transpose the two 8x8 blocks
+      const uint32_t pb0 = movmatrix_trans(pack_h2(pv[0], pv[1]));
+      const uint32_t pb1 = movmatrix_trans(pack_h2(pv[2], pv[3]));
+      // ---- acc^T (rank x head) += L_v^T (rank x token) P (token x head)
+      {
+        const uint8_t* lvt = sm + kSmLV + bd * kLvBytes + lv_off;
+#pragma unroll
+        for (int mt = 0; mt < 3; ++mt) {
+          if (16 * mt < rv) {
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, lvt + 32 * mt);
+            mma16816(acc[mt], a, pb0, pb1);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.lv_free[bd]);
     }
-    if (ok && sm_u >= 0) finish_unit(sm_last);
+    if (ok && n_tiles > 0) write_partial();
+    if (!ok) tmem_wait_ld();   // no load of this thread may be in flight at exit
   }
 
   tc_fence_before();
@@ -621,12 +648,12 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
 bool rope_tc_supported(const Params& p) {
   return p.kind == KVC_LOWRANK && p.rope && p.bits == 4 && !p.resid && !p.page &&
          p.d == kD && p.G == kG && (p.rk == 16 || p.rk == 32) && p.g == 32 &&
-         p.rv % 8 == 0 && p.rv + 1 <= kVM && !p.seq_lens && p.n_tokens > 0 && p.L == 1 &&
+         p.rv % 8 == 0 && p.rv <= kRvMax && !p.seq_lens && p.n_tokens > 0 && p.L == 1 &&
          kTile * (p.lk_row + p.lksz_row + p.lv_row + p.lvsz_row) <= kStageMax;
 }
 
 // Persistent partition: grid CTAs of W tiles each; a unit of tpu tiles spans
-// at most ceil(tpu / W) + 1 CTAs, each with one partial per unit.
+// at most ceil(tpu / W) + 1 CTAs, each writing one partial per epilogue warp.
 void rope_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots) {
   const int t = (p.n_tokens + kTile - 1) / kTile;
   const int units = p.B * p.Hkv;
@@ -637,19 +664,21 @@ void rope_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots) {
   *grid = gr;
   *W = w;
   *tpu = t;
-  *slots = (t + w - 1) / w + 1;
+  *slots = ((t + w - 1) / w + 1) * kEpiWarps;
 }
 
 cudaError_t launch_rope_tc(const Params& p, uint32_t* err, cudaStream_t s) {
   int grid, W, tpu, slots;
   rope_tc_plan(p, &grid, &W, &tpu, &slots);
   Work wk{W, tpu, p.B * p.Hkv * tpu};
-  cudaError_t e = cudaFuncSetAttribute(rope_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmAlloc);
-  if (e != cudaSuccess) return e;
   static_assert(kSmTotal + 1024 <= kSmAlloc, "shared memory carve-up exceeds the allocation");
   static_assert(sizeof(Bars) <= 1024, "barrier block exceeds its slot");
-  rope_tc_kernel<<<grid, kThreads, kSmAlloc, s>>>(p, wk, err);
+  static_assert(kColALk + kNB * 16 <= kColDr && kColDr + kNDr * 128 <= kTmemCols,
+                "TMEM columns exceed the allocation");
+  auto kern = p.rk == 32 ? rope_tc_kernel<32> : rope_tc_kernel<16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmAlloc);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmAlloc, s>>>(p, wk, err);
   return cudaGetLastError();
 }
 

@@ -72,7 +72,7 @@ int fast_slots(const kvc_layout* L, int n_tokens) {
   const int total = L->d.batch * L->d.n_kv_heads * tpu;
   int g = total < kvc::kNumSMs ? total : kvc::kNumSMs;
   const int w = ceil_div(total, g);
-  return ceil_div(tpu, w) + 1;
+  return (ceil_div(tpu, w) + 1) * kvc::kRopeTcParts;
 }
 
 size_t ws_bytes(const kvc_layout* L, int n_tokens) {
@@ -446,6 +446,7 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
     p.S = slots;
     p.seg_W = W;
     p.seg_tpu = tpu;
+    p.seg_parts = kvc::kRopeTcParts;
   }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   char* ws = (char*)workspace;

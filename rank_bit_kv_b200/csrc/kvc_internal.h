@@ -61,6 +61,7 @@ struct Params {
   // persistent tensor-core path: contiguous ranges of seg_W tiles per CTA over
   // units of seg_tpu tiles (0 = split partials indexed by split)
   int seg_W, seg_tpu;
+  int seg_parts;         // partials written per CTA and unit on that path
   uint32_t* err;         // error word of the workspace (bounded waits that gave up)
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
   double rope_f[64];
@@ -97,7 +98,9 @@ struct AppendParams {
   int* off_v_w;
 };
 
-// tensor-core decode of pre-RoPE INT4 low-rank caches
+// tensor-core decode of pre-RoPE INT4 low-rank caches; every CTA writes one
+// partial per epilogue warp and unit it touches
+constexpr int kRopeTcParts = 8;
 bool rope_tc_supported(const Params& p);
 void rope_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
 cudaError_t launch_rope_tc(const Params& p, uint32_t* err, cudaStream_t s);

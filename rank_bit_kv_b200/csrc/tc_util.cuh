@@ -20,6 +20,8 @@ namespace tc {
 constexpr uint32_t kErrTimeout = 1u;
 // A wait gives up after this many nanoseconds (checked every 256 polls).
 constexpr uint64_t kWaitLimitNs = 500ull * 1000ull * 1000ull;
+// Longest single sleep inside a wait (ns); the phase completing wakes it earlier.
+constexpr uint32_t kSleepHintNs = 1000000u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -63,38 +65,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking probe of a phase (returns at once; try_wait may suspend the
-// thread for a while, which a scheduler polling several barriers cannot afford).
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes (or the hint in nanoseconds passes) instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSleepHintNs)
       : "memory");
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs: sets *abort (shared) and the error word and returns false.
+// Wait for the phase with the given parity to complete.  The waiting warp is
+// suspended in hardware, so it takes no issue slots or shared-memory bandwidth
+// from the working ones.  Gives up after kWaitLimitNs: sets *abort (shared)
+// and the error word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* err) {
-  // polls with the non-blocking probe: a thread suspended inside try_wait can
-  // resume well after the phase completes, which adds up along the per-tile
-  // chain of hand-offs between the warp roles
-  if (mbar_test(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_test(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        if (err) atomicOr(err, kErrTimeout);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      if (err) atomicOr(err, kErrTimeout);
+      return false;
     }
   }
 }
@@ -233,6 +232,27 @@ __device__ __forceinline__ void tmem_st2(uint32_t taddr, const uint32_t (&r)[2])
                : "memory");
 }
 
+// 16 lanes x 256 bit, repeated twice: the m16n8 accumulator-fragment layout of
+// two consecutive 8-column blocks (regs 0..3 block 0, 4..7 block 1; within a
+// block: (row lane/4, cols 2*(lane%4)+{0,1}), then row lane/4 + 8).
+__device__ __forceinline__ void tmem_ld16x256_x2(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+// Same shape over 16-bit data held one value per 32-bit column (an f16
+// accumulator): two adjacent columns are packed into each register, so a
+// repetition covers 16 columns -- regs 0,1: row lane/4, columns 4*(lane%4) +
+// {0,1} and {2,3}; regs 2,3: row lane/4 + 8; regs 4..7: the next 16 columns.
+__device__ __forceinline__ void tmem_ld16x256_x2_pack16(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.pack::16b.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -255,6 +275,32 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4])
                : "memory");
 }
 
+// ---------------------------------------------------------------- warp-level MMA
+
+// D(16x8 f32) += A(16x16 f16, row) * B(16x8 f16, col)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// transpose of an 8x8 b16 matrix held in the standard fragment layout
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// four transposed 8x8 b16 matrices; lanes 8i..8i+7 give the row addresses of matrix i
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row_addr)));
+}
+
 // ---------------------------------------------------------------- descriptors
 
 // Shared-memory matrix descriptor, no swizzle ("interleaved" 8 x 16-byte core
@@ -274,6 +320,13 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, i
                                                  int d_f16 = 0) {
   return ((d_f16 ? 0u : 1u) << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// 2^x (ex2.approx.ftz: relative error about 2^-22; 2^-inf = 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
