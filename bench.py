@@ -221,7 +221,7 @@ def cpu_oracle_rate(a, c, seconds):
             break
     gbs = done * _unit_bytes(c, c["T"]) / el / 1e9
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"{done} of {len(units)} (batch row, KV head) units at T={c['T']} "
+            "sample": f"{done} unit decodes cycling over the {len(units)} (batch row, KV head) units at T={c['T']} "
                       f"({done * _unit_bytes(c, c['T'])} compressed bytes) in {el:.1f} s, "
                       f"fp64 numpy"}
 
@@ -369,7 +369,7 @@ def run_kvc(args, rank, world, torch, dist):
     line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(ms_per_step, 5),
             "us_per_step": round(ms_per_step * 1e3, 2), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp16 MMA operands, fp32 accumulate",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic",
             "config": workload_config(c, f"{n} rotating cache copies of {step_bytes} B "
                                          f"({n * step_bytes} B > 126 MiB L2)"),
