@@ -14,13 +14,14 @@
 namespace kvc {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kMaxS = 1024;
 
 __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
   extern __shared__ float sm[];
   float* acc = sm;                       // [vdim]
   float* ws = sm + p.vdim;               // [S] weights
+  float* red = ws + p.S;                 // [kThreads] partial sums of the merge
   __shared__ float lsum;
   const int row = blockIdx.x;            // (l * B + b) * Hq + h
   const int h = row % p.Hq;
@@ -30,6 +31,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
   const size_t rows = (size_t)p.L * p.B * p.Hq;
   const int pst = p.vdim + 2;
   const float* part = p.part + (size_t)row * pst;
+  // launched as a programmatic dependent of the split kernel: wait for its
+  // partials here (the launch itself overlaps the split kernel's tail)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // partial slots of this row: all S splits, or -- on the persistent
   // tensor-core path -- one partial for every CTA whose tile range covers
@@ -55,13 +59,26 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
     if (tid == 0) lsum = lt;
   }
   __syncthreads();
-  for (int j = tid; j < p.vdim; j += kThreads) {
+  // merge: thread (j, k) sums the partials s = k, k + K, ... of value j, so
+  // that small value widths still keep every thread busy; then the K partial
+  // sums of each j are added
+  const int K = p.vdim < kThreads ? kThreads / p.vdim : 1;
+  for (int j0 = 0; j0 < p.vdim; j0 += kThreads / K) {
+    const int j = j0 + tid % (kThreads / K), k = tid / (kThreads / K);
     float a = 0.f;
-    for (int s = 0; s < nS; ++s)
-      if (ws[s] != 0.f) a = fmaf(ws[s], part[(size_t)s * rows * pst + j], a);
-    acc[j] = a;
+    if (j < p.vdim && k < K) {
+      for (int s = k; s < nS; s += K)
+        if (ws[s] != 0.f) a = fmaf(ws[s], part[(size_t)s * rows * pst + j], a);
+    }
+    red[tid] = a;
+    __syncthreads();
+    if (tid < kThreads / K && j0 + tid < p.vdim) {
+      float t = 0.f;
+      for (int kk = 0; kk < K; ++kk) t += red[kk * (kThreads / K) + tid];
+      acc[j0 + tid] = t;
+    }
+    __syncthreads();
   }
-  __syncthreads();
   const float L = lsum;
   const float inv_l = L > 0.f ? 1.f / L : 0.f;
   const int d = p.d;
@@ -72,23 +89,39 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
     // Q^T acc_res = diag(signs_v) H acc_res / sqrt(128)
     fwht_smem(acc + p.rv, kResidDim, tid, kThreads);
   }
-  for (int i = tid; i < d; i += kThreads) {
+  // up-projection: P threads per output dim i, each summing every P-th row of
+  // the factor (rows unrolled so that their loads are in flight together),
+  // then the P partial sums are added
+  const int P = d < kThreads ? kThreads / d : 1;
+  for (int i0 = 0; i0 < d; i0 += kThreads / P) {
+    const int i = i0 + tid % (kThreads / P), part_id = tid / (kThreads / P);
     float o = 0.f;
-    if (p.kind == KVC_LOWRANK || p.kind == KVC_VARRATE) {
-      const int r = p.kind == KVC_VARRATE ? 64 : p.rv;
-      const __half* bv = p.bv + (int64_t)kvh * r * d + i;
-      for (int j = 0; j < r; ++j) o = fmaf(acc[j], h2f(bv[(int64_t)j * d]), o);
-      if (p.kind == KVC_LOWRANK && p.resid)
-        o = fmaf((float)p.signs_v[i] * rsqrtf((float)kResidDim), acc[p.rv + i], o);
-    } else if (p.kind == KVC_BLOCK_SHARED) {
-      const __half* w = p.bv + (int64_t)l * p.D * p.Hkv * d + kvh * d + i;
-      for (int c = 0; c < p.D; ++c) o = fmaf(acc[c], h2f(w[(int64_t)c * p.Hkv * d]), o);
-    } else {
-      o = acc[i];
+    if (i < d && part_id < P) {
+      if (p.kind == KVC_LOWRANK || p.kind == KVC_VARRATE) {
+        const int r = p.kind == KVC_VARRATE ? 64 : p.rv;
+        const __half* bv = p.bv + (int64_t)kvh * r * d + i;
+#pragma unroll 8
+        for (int j = part_id; j < r; j += P) o = fmaf(acc[j], h2f(bv[(int64_t)j * d]), o);
+        if (p.kind == KVC_LOWRANK && p.resid && part_id == 0)
+          o = fmaf((float)p.signs_v[i] * rsqrtf((float)kResidDim), acc[p.rv + i], o);
+      } else if (p.kind == KVC_BLOCK_SHARED) {
+        const __half* w = p.bv + (int64_t)l * p.D * p.Hkv * d + kvh * d + i;
+#pragma unroll 8
+        for (int c = part_id; c < p.D; c += P) o = fmaf(acc[c], h2f(w[(int64_t)c * p.Hkv * d]), o);
+      } else if (part_id == 0) {
+        o = acc[i];
+      }
     }
-    o *= inv_l;
-    if (p.out_bf16) outb[(int64_t)row * d + i] = __float2bfloat16_rn(o);
-    else outf[(int64_t)row * d + i] = o;
+    red[tid] = o;
+    __syncthreads();
+    if (tid < kThreads / P && i0 + tid < d) {
+      float t = 0.f;
+      for (int k = 0; k < P; ++k) t += red[k * (kThreads / P) + tid];
+      t *= inv_l;
+      if (p.out_bf16) outb[(int64_t)row * d + i0 + tid] = __float2bfloat16_rn(t);
+      else outf[(int64_t)row * d + i0 + tid] = t;
+    }
+    __syncthreads();
   }
 }
 
@@ -97,12 +130,21 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
 cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   if (p.S > kMaxS) return cudaErrorInvalidValue;
   const int rows = p.L * p.B * p.Hq;
-  const size_t bytes = ((size_t)p.vdim + p.S) * sizeof(float);
+  const size_t bytes = ((size_t)p.vdim + p.S + kThreads) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(combine_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  combine_kernel<<<rows, kThreads, bytes, s>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 
 }  // namespace kvc

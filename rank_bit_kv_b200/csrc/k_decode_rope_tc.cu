@@ -60,7 +60,7 @@ constexpr int kHalf = 64;          // RoPE pairs
 constexpr int kG = 4;              // query heads per KV head
 constexpr int kRvMax = 48;         // value rank handled (3 m16 tiles)
 constexpr int kLvStride = 56;      // halves per L_v row in shared memory (48 + pad)
-constexpr int kNBLog2 = 2, kNB = 1 << kNBLog2;   // dequantized operand buffers (tile jj uses jj % kNB)
+constexpr int kNBLog2 = 3, kNB = 1 << kNBLog2;   // dequantized operand buffers (tile jj uses jj % kNB)
 
 // TMEM columns (512 allocated)
 constexpr uint32_t kColALk = 0;    // kNB x 16   recon A (128 x rk fp16, rk <= 32)
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       mbar_init(&bars.empty[s], 4);
     }
     for (int b = 0; b < kNB; ++b) {
-      mbar_init(&bars.tile_in[b], 4);
+      mbar_init(&bars.tile_in[b], 5);
       mbar_init(&bars.alk_free[b], 1);
       mbar_init(&bars.lv_free[b], kEpiWarps);
     }
@@ -207,7 +207,20 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
   const uint32_t tmem = bars.tmem_base;
 
   if (warp == kWarpProd) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer + q_rot
+    // q_rot: lane m rotates pairs 2m, 2m + 1.  The angle of pair i at
+    // t0 = 128 jt is jt * frac(128 f_i) turns; frac(128 f_i) is held in 32-bit
+    // fixed point so that jt * F mod 2^32 is exact.
+    uint32_t Fq[2];
+    float qv[kG][4];                         // q[h][2m], [2m+1], [2m+64], [2m+65] * scale
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      double x = 128.0 * p.rope_f[(2 * lane + e) & (kHalf - 1)];
+      x -= floor(x);
+      Fq[e] = (uint32_t)(unsigned long long)llrint(x * 4294967296.0);
+    }
+#pragma unroll
+    for (int h = 0; h < kG; ++h) qv[h][0] = qv[h][1] = qv[h][2] = qv[h][3] = 0.f;
     int issued_upto = 0;  // tiles issued
     TileCursor cur(t_first, wk.tpu);
     for (int jj = 0; jj < n_tiles && !*abort; ++jj, cur.next()) {
@@ -247,6 +260,39 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
         if (lane == 0) mbar_arrive(&bars.full[s]);
       }
       issued_upto = jj + 1;
+      // ---- q_rot = R_t0^T q (times the softmax scale) as score-MMA B fragments
+      const int bd = slot_of<kNBLog2>(jj);
+      if (jj == 0 || cur.jt == 0) {
+        const int kvh = cur.u % p.Hkv, b = cur.u / p.Hkv;
+        const __nv_bfloat16* qq = p.q + ((size_t)b * p.Hq + kvh * kG) * kD;
+#pragma unroll
+        for (int h = 0; h < kG; ++h) {
+          qv[h][0] = bf2f(qq[h * kD + 2 * lane]) * p.scale_log2;
+          qv[h][1] = bf2f(qq[h * kD + 2 * lane + 1]) * p.scale_log2;
+          qv[h][2] = bf2f(qq[h * kD + 2 * lane + kHalf]) * p.scale_log2;
+          qv[h][3] = bf2f(qq[h * kD + 2 * lane + kHalf + 1]) * p.scale_log2;
+        }
+      }
+      // the epilogue warps are done with this buffer's previous tile
+      if (jj >= kNB && !mbar_wait(&bars.lv_free[bd], phase_of<kNBLog2>(jj - kNB), abort, err)) break;
+      float ca[2], sa[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int turns = (int)((uint32_t)cur.jt * Fq[e]);      // in 2^-32 turns
+        __sincosf((float)turns * 1.4629180792671596e-09f, &sa[e], &ca[e]);   // 2 pi / 2^32
+      }
+      uint8_t* qf = sm + kSmQF + bd * kQfBytes;
+#pragma unroll
+      for (int h = 0; h < kG; ++h) {
+        const float lo0 = ca[0] * qv[h][0] + sa[0] * qv[h][2];
+        const float lo1 = ca[1] * qv[h][1] + sa[1] * qv[h][3];
+        const float hi0 = ca[0] * qv[h][2] - sa[0] * qv[h][0];
+        const float hi1 = ca[1] * qv[h][3] - sa[1] * qv[h][1];
+        *reinterpret_cast<uint32_t*>(qf + qf_offset(h, 2 * lane)) = pack_h2(lo0, lo1);
+        *reinterpret_cast<uint32_t*>(qf + qf_offset(h, 2 * lane + kHalf)) = pack_h2(hi0, hi1);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.tile_in[bd]);
     }
     // drain: every issued stage must have landed before the CTA may exit
     if (*abort && lane == 0) {
@@ -279,34 +325,61 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     }
     __syncwarp();
   } else if (warp < kWarpEpi) {
-    // ------------------------------------------------------------ dequantization + q_rot
+    // ------------------------------------------------------------ dequantization
+    // thread = token row.  Software-pipelined: the stage words of tile jj + 1
+    // are loaded into registers before tile jj is dequantized and stored.
     const int q4 = warp & 3;                 // TMEM lane quadrant
     const int row = 32 * q4 + lane;          // token row in the tile
     const int dt = threadIdx.x - 32 * kWarpDeq;   // 0..127
-    const bool qrot_warp = warp == kWarpDeq;
-    // q_rot: lane m of the first dequant warp rotates pairs 2m, 2m + 1.  The
-    // angle of pair i at t0 = 128 jt is jt * frac(128 f_i) turns; frac(128 f_i)
-    // is held in 32-bit fixed point so that jt * F mod 2^32 is exact.
-    uint32_t Fq[2];
-    float qv[kG][4];                         // q[h][2m], [2m+1], [2m+64], [2m+65] * scale
+    const int nwv = rv / 8;
+    // raw words of one tile's row: key codes, key (scale, zero), value codes,
+    // value (scale, zero) of both groups
+    struct RowWords {
+      uint32_t kc[RK / 8], ksz, vc[kRvMax / 8], vsz[2];
+    };
+    auto load_row = [&](int jj, RowWords& w) {
+      const uint8_t* st = sm + kSmStage + slot_of<kStagesLog2>(jj) * kStageMax;
+      if constexpr (RK == 32) {
+        const uint4 v = *reinterpret_cast<const uint4*>(st + row * (RK / 2));
+        w.kc[0] = v.x;
+        w.kc[1] = v.y;
+        w.kc[2] = v.z;
+        w.kc[3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(st + row * (RK / 2));
+        w.kc[0] = v.x;
+        w.kc[1] = v.y;
+      }
+      w.ksz = *reinterpret_cast<const uint32_t*>(st + kTile * (RK / 2) + row * lksz_row);
+      const uint8_t* vbase = st + kTile * (lk_row + lksz_row);
+      const uint32_t* codes = reinterpret_cast<const uint32_t*>(vbase + row * lv_row);
+      const uint32_t* sz = reinterpret_cast<const uint32_t*>(vbase + kTile * lv_row + row * lvsz_row);
+      // words past rv read neighbouring bytes of the stage and are dropped
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      double x = 128.0 * p.rope_f[(2 * lane + e) & (kHalf - 1)];
-      x -= floor(x);
-      Fq[e] = (uint32_t)(unsigned long long)llrint(x * 4294967296.0);
-    }
-#pragma unroll
-    for (int h = 0; h < kG; ++h) qv[h][0] = qv[h][1] = qv[h][2] = qv[h][3] = 0.f;
+      for (int j = 0; j < kRvMax / 8; ++j) w.vc[j] = codes[j];
+      w.vsz[0] = sz[0];
+      w.vsz[1] = sz[1];
+    };
+    RowWords cw, nw;
+    bool ok = n_tiles > 0 && mbar_wait(&bars.full[0], 0, abort, err);
+    if (ok) load_row(0, cw);
     TileCursor cur(t_first, wk.tpu);
-    for (int jj = 0; jj < n_tiles; ++jj, cur.next()) {
+    for (int jj = 0; jj < n_tiles && ok; ++jj, cur.next()) {
       const int nt = cur.valid_rows(p.n_tokens);
       const int bd = slot_of<kNBLog2>(jj), s = slot_of<kStagesLog2>(jj);
+      // prefetch the next tile's words (their latency hides behind this tile)
+      if (jj + 1 < n_tiles) {
+        if (!(ok = mbar_wait(&bars.full[slot_of<kStagesLog2>(jj + 1)], phase_of<kStagesLog2>(jj + 1),
+                             abort, err)))
+          break;
+        load_row(jj + 1, nw);
+      }
       if (jj == 0 || cur.jt == 0) {
         // new unit: Bk is rewritten once the previous tile's recon is done
-        if (jj > 0 && !mbar_wait(&bars.alk_free[slot_of<kNBLog2>(jj - 1)], phase_of<kNBLog2>(jj - 1),
-                                 abort, err))
+        if (jj > 0 && !(ok = mbar_wait(&bars.alk_free[slot_of<kNBLog2>(jj - 1)],
+                                       phase_of<kNBLog2>(jj - 1), abort, err)))
           break;
-        const int kvh = cur.u % p.Hkv, b = cur.u / p.Hkv;
+        const int kvh = cur.u % p.Hkv;
         // B operand of the reconstruction: N = 128 dims x K = rk (logical ranks),
         // K-major core matrices, logical k holds Bk row perm_rank(k)
         const __half* bk = p.bk + (size_t)kvh * RK * kD;
@@ -317,102 +390,51 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
               bk[(size_t)perm_rank(k) * kD + n];
         }
         fence_proxy_async_smem();
-        if (qrot_warp) {
-          const __nv_bfloat16* qq = p.q + ((size_t)b * p.Hq + kvh * kG) * kD;
-#pragma unroll
-          for (int h = 0; h < kG; ++h) {
-            qv[h][0] = bf2f(qq[h * kD + 2 * lane]) * p.scale_log2;
-            qv[h][1] = bf2f(qq[h * kD + 2 * lane + 1]) * p.scale_log2;
-            qv[h][2] = bf2f(qq[h * kD + 2 * lane + kHalf]) * p.scale_log2;
-            qv[h][3] = bf2f(qq[h * kD + 2 * lane + kHalf + 1]) * p.scale_log2;
-          }
-        }
       }
-      if (!mbar_wait(&bars.full[s], phase_of<kStagesLog2>(jj), abort, err)) break;
       if (jj >= kNB) {
         // recon(jj - kNB) read this A buffer; the epilogue warps are done with
-        // this L_v / q_rot buffer
-        if (!mbar_wait(&bars.alk_free[bd], phase_of<kNBLog2>(jj - kNB), abort, err)) break;
-        if (!mbar_wait(&bars.lv_free[bd], phase_of<kNBLog2>(jj - kNB), abort, err)) break;
+        // this L_v buffer
+        if (!(ok = mbar_wait(&bars.alk_free[bd], phase_of<kNBLog2>(jj - kNB), abort, err))) break;
+        if (!(ok = mbar_wait(&bars.lv_free[bd], phase_of<kNBLog2>(jj - kNB), abort, err))) break;
       }
       tc_fence_after();
       // rows past the end get scale = zero = 0 (bitwise: the stage bytes of
       // such rows are stale and may hold any fp16 pattern), hence zero latents
       const uint32_t vmask = row < nt ? 0xFFFFFFFFu : 0u;
-      const uint8_t* st = sm + kSmStage + s * kStageMax;
       // ---- keys: rk/8 words -> TMEM columns (A operand of the reconstruction)
       {
-        uint32_t cw[RK / 8];
-        if constexpr (RK == 32) {
-          const uint4 v = *reinterpret_cast<const uint4*>(st + row * (RK / 2));
-          cw[0] = v.x;
-          cw[1] = v.y;
-          cw[2] = v.z;
-          cw[3] = v.w;
-        } else {
-          const uint2 v = *reinterpret_cast<const uint2*>(st + row * (RK / 2));
-          cw[0] = v.x;
-          cw[1] = v.y;
-        }
-        const uint32_t szw =
-            *reinterpret_cast<const uint32_t*>(st + kTile * (RK / 2) + row * lksz_row) & vmask;
+        const uint32_t szw = cw.ksz & vmask;
         const __half2 sz0 = *reinterpret_cast<const __half2*>(&szw);
         const __half2 s2 = __low2half2(sz0), z2 = __high2half2(sz0);
         uint32_t ka[RK / 2];
 #pragma unroll
-        for (int j = 0; j < RK / 8; ++j) dequant_word(cw[j], s2, z2, ka + 4 * j);
+        for (int j = 0; j < RK / 8; ++j) dequant_word(cw.kc[j], s2, z2, ka + 4 * j);
         const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + kColALk + bd * 16;
         if constexpr (RK == 32) tmem_st16(ta, ka);
         else tmem_st8(ta, ka);
       }
       // ---- values: rv/8 words -> shared memory rows [token][logical rank]
       {
-        const uint8_t* vbase = st + kTile * (lk_row + lksz_row);
-        const uint32_t* codes = reinterpret_cast<const uint32_t*>(vbase + row * lv_row);
-        const uint32_t* sz = reinterpret_cast<const uint32_t*>(vbase + kTile * lv_row + row * lvsz_row);
         uint8_t* lv = sm + kSmLV + bd * kLvBytes + row * (kLvStride * 2);
-        // all loads first (words past rv read neighbouring bytes of the stage
-        // and are dropped), then branch-free dequantization
-        uint32_t vw[kRvMax / 8];
-#pragma unroll
-        for (int j = 0; j < kRvMax / 8; ++j) vw[j] = codes[j];
-        const uint32_t gw[2] = {sz[0] & vmask, sz[1] & vmask};   // groups of 32 ranks
+        const uint32_t gw[2] = {cw.vsz[0] & vmask, cw.vsz[1] & vmask};   // groups of 32 ranks
 #pragma unroll
         for (int j = 0; j < kRvMax / 8; ++j) {
-          if (j < rv / 8) {
+          if (j < nwv) {
             const __half2 szg = *reinterpret_cast<const __half2*>(&gw[j < 4 ? 0 : 1]);
             uint32_t r[4];
-            dequant_word(vw[j], __low2half2(szg), __high2half2(szg), r);
+            dequant_word(cw.vc[j], __low2half2(szg), __high2half2(szg), r);
             *reinterpret_cast<uint4*>(lv + j * 16) = make_uint4(r[0], r[1], r[2], r[3]);
           }
-        }
-      }
-      // ---- q_rot = R_t0^T q (times the softmax scale) as score-MMA B fragments
-      if (qrot_warp) {
-        float ca[2], sa[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int turns = (int)((uint32_t)cur.jt * Fq[e]);      // in 2^-32 turns
-          __sincosf((float)turns * 1.4629180792671596e-09f, &sa[e], &ca[e]);   // 2 pi / 2^32
-        }
-        uint8_t* qf = sm + kSmQF + bd * kQfBytes;
-#pragma unroll
-        for (int h = 0; h < kG; ++h) {
-          const float lo0 = ca[0] * qv[h][0] + sa[0] * qv[h][2];
-          const float lo1 = ca[1] * qv[h][1] + sa[1] * qv[h][3];
-          const float hi0 = ca[0] * qv[h][2] - sa[0] * qv[h][0];
-          const float hi1 = ca[1] * qv[h][3] - sa[1] * qv[h][1];
-          *reinterpret_cast<uint32_t*>(qf + qf_offset(h, 2 * lane)) = pack_h2(lo0, lo1);
-          *reinterpret_cast<uint32_t*>(qf + qf_offset(h, 2 * lane + kHalf)) = pack_h2(hi0, hi1);
         }
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bars.empty[s]);
+        mbar_arrive(&bars.empty[s]);       // tile jj's words were consumed above
         mbar_arrive(&bars.tile_in[bd]);
       }
+      cw = nw;
     }
   } else {
     // ------------------------------------------------------------ epilogue warps
@@ -493,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     };
 
     // K_hat of this warp's 16 rows of tile jj (f16, four 32-column loads),
-    // issued one tile ahead so that the TMEM latency hides behind softmax + V
+    // issued one iteration ahead so that the TMEM latency hides behind work
     uint32_t klo[2][8], khi[2][8];
     auto issue_k = [&](int jj) -> bool {
       const int kb = dr_slot(jj);
@@ -507,7 +529,63 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       return true;
     };
 
-    bool ok = n_tiles > 0 && issue_k(0);
+    // K_hat of tile jj is in registers: every epilogue warp releases its buffer
+    auto k_ready = [&](int jj) -> bool {
+      if (!mbar_wait(&bars.tile_in[slot_of<kNBLog2>(jj)], phase_of<kNBLog2>(jj), abort, err))
+        return false;
+      tmem_wait_ld();
+      reg_fence(klo[0]);
+      reg_fence(klo[1]);
+      reg_fence(khi[0]);
+      reg_fence(khi[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.dr_free[dr_slot(jj)]);
+      return true;
+    };
+    // RoPE in registers, then the score MMA (k steps kk and kk + 4 in two
+    // independent accumulator chains); the query fragments of k steps
+    // {2h, 2h+1} and {2h+4, 2h+5} sit in 16-byte chunks h and h + 2.  Scores
+    // come out in log2 units (the softmax scale is folded into q_rot).
+    auto score_tile = [&](int bd, float (&out)[4]) {
+      const uint4* qf = reinterpret_cast<const uint4*>(sm + kSmQF + bd * kQfBytes + qblk * 64);
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint4 qlo = qf[hh ^ qsw], qhi = qf[(hh + 2) ^ qsw];
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int kk = 2 * hh + k2;
+          uint32_t xr[4], yr[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {          // r: (row r >> 1, dims pair-couple r & 1)
+            const __half2 x = *reinterpret_cast<const __half2*>(&klo[hh][4 * k2 + r]);
+            const __half2 y = *reinterpret_cast<const __half2*>(&khi[hh][4 * k2 + r]);
+            const __half2 C = *reinterpret_cast<const __half2*>(&cs[kk][r & 1][r >> 1]);
+            const __half2 S = *reinterpret_cast<const __half2*>(&sn[kk][r & 1][r >> 1]);
+            const __half2 xo = __hfma2(C, x, __hneg2(__hmul2(S, y)));   // k_i cos - k_{i+64} sin
+            const __half2 yo = __hfma2(C, y, __hmul2(S, x));            // k_{i+64} cos + k_i sin
+            xr[r] = *reinterpret_cast<const uint32_t*>(&xo);
+            yr[r] = *reinterpret_cast<const uint32_t*>(&yo);
+          }
+          const uint32_t alo[4] = {xr[0], xr[2], xr[1], xr[3]};
+          const uint32_t ahi[4] = {yr[0], yr[2], yr[1], yr[3]};
+          mma16816(sa, alo, k2 ? qlo.z : qlo.x, k2 ? qlo.w : qlo.y);
+          mma16816(sb, ahi, k2 ? qhi.z : qhi.x, k2 ? qhi.w : qhi.y);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) out[i] = sa[i] + sb[i];
+    };
+
+    // Software pipeline: iteration jj scores tile jj + 1 and runs the softmax
+    // and value product of tile jj, so the two dependency chains interleave.
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    bool ok = n_tiles > 0 && issue_k(0) && k_ready(0);
+    if (ok) {
+      score_tile(0, sc);
+      if (n_tiles > 1) ok = issue_k(1);
+    }
     TileCursor cur(t_first, wk.tpu);
     for (int jj = 0; jj < n_tiles && ok; ++jj, cur.next()) {
       const int nt = cur.valid_rows(p.n_tokens);
@@ -518,66 +596,23 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
         cur_kvh = cur.u % p.Hkv;
         cur_slot = cta - (int)(((long long)cur.u * wk.tpu) / wk.W);
       }
-      const int kb = dr_slot(jj), bd = slot_of<kNBLog2>(jj);
-      if (!(ok = mbar_wait(&bars.tile_in[bd], phase_of<kNBLog2>(jj), abort, err))) break;
-      tmem_wait_ld();
-      reg_fence(klo[0]);
-      reg_fence(klo[1]);
-      reg_fence(khi[0]);
-      reg_fence(khi[1]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.dr_free[kb]);
-      // ---- q_rot fragments (heads 0..3 in lanes 0..15; lanes 16..31 read the
-      // buffer's zero blocks of the padding heads 4..7)
-      uint32_t qb[8][2];
-      {
-        const uint4* qf = reinterpret_cast<const uint4*>(sm + kSmQF + bd * kQfBytes + qblk * 64);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 x = qf[v ^ qsw];
-          qb[2 * v][0] = x.x;
-          qb[2 * v][1] = x.y;
-          qb[2 * v + 1][0] = x.z;
-          qb[2 * v + 1][1] = x.w;
-        }
-      }
-      // ---- RoPE in registers, then the score MMA (k steps kk and kk + 4, two
-      // independent accumulator chains)
-      float sc[4] = {0.f, 0.f, 0.f, 0.f}, sh[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t xr[4], yr[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {            // r: (row r >> 1, dims pair-couple r & 1)
-          const __half2 x = *reinterpret_cast<const __half2*>(&klo[kk >> 1][4 * (kk & 1) + r]);
-          const __half2 y = *reinterpret_cast<const __half2*>(&khi[kk >> 1][4 * (kk & 1) + r]);
-          const __half2 C = *reinterpret_cast<const __half2*>(&cs[kk][r & 1][r >> 1]);
-          const __half2 S = *reinterpret_cast<const __half2*>(&sn[kk][r & 1][r >> 1]);
-          const __half2 xo = __hfma2(C, x, __hneg2(__hmul2(S, y)));   // k_i cos - k_{i+64} sin
-          const __half2 yo = __hfma2(C, y, __hmul2(S, x));            // k_{i+64} cos + k_i sin
-          xr[r] = *reinterpret_cast<const uint32_t*>(&xo);
-          yr[r] = *reinterpret_cast<const uint32_t*>(&yo);
-        }
-        const uint32_t alo[4] = {xr[0], xr[2], xr[1], xr[3]};
-        const uint32_t ahi[4] = {yr[0], yr[2], yr[1], yr[3]};
-        mma16816(sc, alo, qb[kk][0], qb[kk][1]);
-        mma16816(sh, ahi, qb[kk + 4][0], qb[kk + 4][1]);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sc[i] += sh[i];
-      // next tile's K_hat loads fly while this tile finishes
-      if (jj + 1 < n_tiles && !(ok = issue_k(jj + 1))) break;
-      // ---- online softmax of this warp (rows r0, r1; heads 2c4, 2c4 + 1);
-      // scores are already in log2 units (the scale is folded into q_rot)
-      if (nt < kTile) {
-        if (r0 >= nt) sc[0] = sc[1] = -INFINITY;
-        if (r1 >= nt) sc[2] = sc[3] = -INFINITY;
-      }
-      const bool need = sc[0] > m_thr[0] || sc[2] > m_thr[0] || sc[1] > m_thr[1] ||
-                        sc[3] > m_thr[1];
+      const int bd = slot_of<kNBLog2>(jj);
+      if (jj + 1 < n_tiles && !(ok = k_ready(jj + 1))) break;
+      // ---- score of tile jj + 1 (after the last tile: stale registers, dropped)
+      float sn1[4];
+      score_tile(slot_of<kNBLog2>(jj + 1), sn1);
+      // ---- online softmax of tile jj (rows r0, r1; heads 2c4, 2c4 + 1)
+      const bool v0 = r0 < nt, v1 = r1 < nt;     // rows past the end weigh nothing
+      const float s0 = v0 ? sc[0] : -INFINITY, s1 = v0 ? sc[1] : -INFINITY;
+      const float s2 = v1 ? sc[2] : -INFINITY, s3 = v1 ? sc[3] : -INFINITY;
+      const bool need = s0 > m_thr[0] || s2 > m_thr[0] || s1 > m_thr[1] || s3 > m_thr[1];
+      float pv[4];
+      pv[0] = ex2_approx(s0 - m_ref[0]);
+      pv[1] = ex2_approx(s1 - m_ref[1]);
+      pv[2] = ex2_approx(s2 - m_ref[0]);
+      pv[3] = ex2_approx(s3 - m_ref[1]);
       if (__any_sync(0xffffffffu, need)) {
-        float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
           mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
@@ -599,18 +634,15 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
         m_ref[1] = n1;
         m_thr[0] = n0 + 8.f;
         m_thr[1] = n1 + 8.f;
+        pv[0] = ex2_approx(s0 - n0);
+        pv[1] = ex2_approx(s1 - n1);
+        pv[2] = ex2_approx(s2 - n0);
+        pv[3] = ex2_approx(s3 - n1);
       }
-      float pv[4];
-      pv[0] = ex2_approx(sc[0] - m_ref[0]);
-      pv[1] = ex2_approx(sc[1] - m_ref[1]);
-      pv[2] = ex2_approx(sc[2] - m_ref[0]);
-      pv[3] = ex2_approx(sc[3] - m_ref[1]);
-      if (nt < kTile) {
-        // rows past the end weigh nothing, also while no row of this warp has
-        // been seen (-inf - -inf would give NaN)
-        if (r0 >= nt) pv[0] = pv[1] = 0.f;
-        if (r1 >= nt) pv[2] = pv[3] = 0.f;
-      }
+      // masked rows: select, not multiply (-inf - -inf is NaN while no row of
+      // this warp has been seen)
+      if (!v0) pv[0] = pv[1] = 0.f;
+      if (!v1) pv[2] = pv[3] = 0.f;
       l_sum[0] += pv[0] + pv[2];
       l_sum[1] += pv[1] + pv[3];
       // P as the B operand (k = token, n = head): transpose the two 8x8 blocks
@@ -630,6 +662,10 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.lv_free[bd]);
+      // the K_hat loads of tile jj + 2 fly during the next iteration's waits
+      if (jj + 2 < n_tiles && !(ok = issue_k(jj + 2))) break;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sc[i] = sn1[i];
     }
     if (ok && n_tiles > 0) write_partial();
     if (!ok) tmem_wait_ld();   // no load of this thread may be in flight at exit
