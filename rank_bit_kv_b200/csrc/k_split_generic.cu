@@ -357,7 +357,8 @@ __global__ void __launch_bounds__(kThreads) split_generic_kernel(Params p) {
 }  // namespace
 
 cudaError_t launch_split(const Params& p, cudaStream_t s) {
-  if (p.seg_W > 0) return launch_rope_tc(p, p.err, s);
+  if (p.seg_W > 0)
+    return p.kind == KVC_DENSE_BF16 ? launch_dense_tc(p, s) : launch_rope_tc(p, p.err, s);
   const Geo g = geometry(p);
   const Smem S = carve(p, g);
   const size_t bytes = (size_t)S.total * sizeof(float);

@@ -78,7 +78,9 @@ int fast_slots(const kvc_layout* L, int n_tokens) {
 size_t ws_bytes(const kvc_layout* L, int n_tokens) {
   int S, len;
   plan(L, n_tokens, &S, &len);
-  const int Sf = fast_slots(L, n_tokens);
+  const int Sf = L->d.kind == KVC_DENSE_BF16
+                     ? kvc::dense_tc_slots(L->d.batch, L->d.n_kv_heads, n_tokens > 0 ? n_tokens : 1)
+                     : fast_slots(L, n_tokens);
   if (Sf > S) S = Sf;
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   size_t b = kWsHeader + round_up(rows * L->qdim * sizeof(float), 256);
@@ -447,6 +449,13 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
     p.seg_W = W;
     p.seg_tpu = tpu;
     p.seg_parts = kvc::kRopeTcParts;
+  } else if (kvc::dense_tc_supported(p)) {
+    int grid, W, tpu, slots;
+    kvc::dense_tc_plan(p, &grid, &W, &tpu, &slots);
+    p.S = slots;
+    p.seg_W = W;
+    p.seg_tpu = tpu;
+    p.seg_parts = 1;
   }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   char* ws = (char*)workspace;

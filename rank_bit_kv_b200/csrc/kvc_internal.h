@@ -105,6 +105,12 @@ bool rope_tc_supported(const Params& p);
 void rope_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
 cudaError_t launch_rope_tc(const Params& p, uint32_t* err, cudaStream_t s);
 
+// warp-level tensor-core decode of dense bf16 caches (the baseline layout)
+bool dense_tc_supported(const Params& p);
+void dense_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
+int dense_tc_slots(int batch, int n_kv_heads, int n_tokens);
+cudaError_t launch_dense_tc(const Params& p, cudaStream_t s);
+
 // Record a status and message for kvc_last_error(); returns st.
 kvc_status report_error(kvc_status st, const char* fmt, ...);
 

@@ -121,6 +121,25 @@ def test_dense_bf16_small():
     assert_close(run_decode(cfg, a, 700), oracle(cfg, a, 700), what="dense")
 
 
+@pytest.mark.parametrize("G,T", [(4, 1), (4, 16), (4, 17), (1, 300), (8, 1000)])
+def test_dense_tensor_core_shapes(G, T):
+    """Dense bf16 decode on the warp-level MMA path: GQA groups 1..8, tiles of
+    16 tokens with ragged tails, a single token."""
+    Hkv = 4
+    cfg = dict(kind="dense", B=2, Hq=G * Hkv, Hkv=Hkv, d=128, T=T)
+    a = synth.dense_cache(2, G * Hkv, Hkv, 128, T, seed=11 + G)
+    assert_close(run_decode(cfg, a, T), oracle(cfg, a, T), what=f"dense G={G} T={T}")
+
+
+def test_dense_peaked():
+    """q x 8: a near one-hot softmax, so the probabilities' own rounding shows."""
+    cfg = dict(kind="dense", B=1, Hq=32, Hkv=8, d=128, T=2000)
+    a = synth.dense_cache(1, 32, 8, 128, 2000, seed=21)
+    q = synth.to_bf16_bits(synth.bf16_bits_to_f32(a["q"]) * 8.0)
+    a["q"] = q
+    assert_close(run_decode(cfg, a, 2000), oracle(cfg, a, 2000), what="dense peaked")
+
+
 def test_dense_layered():
     cfg = dict(kind="dense", B=1, Hq=8, Hkv=2, d=128, T=129, L=2)
     a = synth.dense_cache(1, 8, 2, 128, 129, seed=6, n_layers=2)
