@@ -5,7 +5,7 @@
 // t ("JoLT: Near-Lossless KV Cache Compression", Key findings: the method works
 // pre-RoPE; the FlashJoLT decode "attends directly on the stored core,
 // factors and residual").  For a tile of 128 tokens starting at t0 the kernel
-//   1. stages the compressed rows with 1-D bulk copies (no multicast),
+//   1. stages the compressed rows with 16-byte cp.async copies,
 //   2. dequantizes L_k into TMEM and L_v into shared memory,
 //   3. reconstructs K_hat = L_k Bk with one tcgen05 MMA per 16 ranks
 //      (M = 128 tokens, N = 128 dims, f16 accumulator in TMEM),
@@ -32,15 +32,18 @@
 // into equal contiguous ranges, one per CTA, so every SM streams the same
 // number of bytes; a range may cross a unit boundary (a partial per part).
 //
-// Warp roles (448 threads, one CTA per SM):
-//   warp 0      bulk-copy producer (6-stage ring of compressed tiles)
+// Warp roles (480 threads, one CTA per SM):
+//   warp 0      producer: 8-stage ring of compressed tiles, 16-byte cp.async
+//               from all lanes, completion counted on the stage barrier
 //   warp 1      TMEM allocation + tcgen05 reconstruction MMAs (one lane)
-//   warps 2-5   dequantization (thread = token row); warp 2 also rotates the
-//               queries of each tile
+//   warps 2-5   dequantization (thread = token row), software-pipelined: the
+//               stage words of tile jj + 1 are loaded before tile jj is stored
 //   warps 6-13  epilogue: each owns 16 rows of every tile, in its TMEM lane
-//               quadrant
+//               quadrant; iteration jj scores tile jj + 1 and runs the softmax
+//               and value product of tile jj
+//   warp 14     q_rot of every tile
 // Every wait is bounded; on a timeout the CTA sets an error bit in the
-// workspace, drains its own bulk copies and MMAs, frees TMEM and exits.
+// workspace, drains its own copies and MMAs, frees TMEM and exits.
 #include <math.h>
 
 #include "kvc_device.cuh"
@@ -53,8 +56,9 @@ using namespace tc;
 
 constexpr int kTile = 128;
 constexpr int kStagesLog2 = 3, kStages = 1 << kStagesLog2;
-constexpr int kThreads = 448;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpDeq = 2, kWarpEpi = 6, kEpiWarps = kRopeTcParts;
+constexpr int kThreads = 480;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpDeq = 2, kWarpEpi = 6, kEpiWarps = kRopeTcParts,
+              kWarpQrot = 14;
 constexpr int kD = 128;            // head dim
 constexpr int kHalf = 64;          // RoPE pairs
 constexpr int kG = 4;              // query heads per KV head
@@ -171,12 +175,11 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
   const int t_first = cta * wk.W;
   const int n_tiles = min(wk.W, wk.total - t_first);
   const int lk_row = p.lk_row, lv_row = p.lv_row, lksz_row = p.lksz_row, lvsz_row = p.lvsz_row;
-  const int stage_bytes = kTile * (lk_row + lksz_row + lv_row + lvsz_row);
   const int rv = p.rv;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.full[s], 32);
       mbar_init(&bars.empty[s], 4);
     }
     for (int b = 0; b < kNB; ++b) {
@@ -207,21 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
   const uint32_t tmem = bars.tmem_base;
 
   if (warp == kWarpProd) {
-    // ------------------------------------------------------------ producer + q_rot
-    // q_rot: lane m rotates pairs 2m, 2m + 1.  The angle of pair i at
-    // t0 = 128 jt is jt * frac(128 f_i) turns; frac(128 f_i) is held in 32-bit
-    // fixed point so that jt * F mod 2^32 is exact.
-    uint32_t Fq[2];
-    float qv[kG][4];                         // q[h][2m], [2m+1], [2m+64], [2m+65] * scale
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      double x = 128.0 * p.rope_f[(2 * lane + e) & (kHalf - 1)];
-      x -= floor(x);
-      Fq[e] = (uint32_t)(unsigned long long)llrint(x * 4294967296.0);
-    }
-#pragma unroll
-    for (int h = 0; h < kG; ++h) qv[h][0] = qv[h][1] = qv[h][2] = qv[h][3] = 0.f;
-    int issued_upto = 0;  // tiles issued
+    // ------------------------------------------------------------ producer
+    // 16-byte cp.async copies spread over the 32 lanes (a tile's four
+    // components are 416 chunks); each lane's completion arrives on the
+    // stage's full barrier (32 arrivals per phase).
     TileCursor cur(t_first, wk.tpu);
     for (int jj = 0; jj < n_tiles && !*abort; ++jj, cur.next()) {
       const int s = slot_of<kStagesLog2>(jj);
@@ -234,33 +226,54 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
                                p.lv + row0 * lv_row,
                                reinterpret_cast<const uint8_t*>(p.lvsz) + row0 * lvsz_row};
       const int rowb[4] = {lk_row, lksz_row, lv_row, lvsz_row};
-      // bulk copies need 16-byte aligned sources: a unit base u * max_tokens * row
-      // is aligned only when max_tokens * row is a multiple of 16
+      // 16-byte copies need 16-byte aligned sources: a unit base
+      // u * max_tokens * row is aligned only when max_tokens * row is a
+      // multiple of 16
       bool aligned = true;
+#pragma unroll
       for (int c = 0; c < 4; ++c) aligned &= (reinterpret_cast<uintptr_t>(src[c]) & 15u) == 0;
-      if (nt == kTile && aligned) {
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&bars.full[s], stage_bytes);
-          int off = 0;
-          for (int c = 0; c < 4; ++c) {
-            bulk_g2s(st + off, src[c], kTile * rowb[c], &bars.full[s]);
-            off += kTile * rowb[c];
+      int off = 0;
+      if (aligned) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int bytes = nt * rowb[c];
+          for (int i = lane; 16 * i < bytes; i += 32) {
+            const int rem = bytes - 16 * i;
+            cp_async16(st + off + 16 * i, src[c] + 16 * i, rem < 16 ? rem : 16);
           }
+          off += kTile * rowb[c];
         }
+        cp_async_mbar_arrive(&bars.full[s]);
       } else {
-        // ragged last tile of a unit, or unaligned rows: plain copies of the nt
-        // valid rows
-        int off = 0;
+        // unaligned rows: plain copies of the nt valid rows
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int n = nt * rowb[c];
           for (int i = lane; i < n; i += 32) st[off + i] = src[c][i];
           off += kTile * rowb[c];
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.full[s]);
+        mbar_arrive(&bars.full[s]);
       }
-      issued_upto = jj + 1;
-      // ---- q_rot = R_t0^T q (times the softmax scale) as score-MMA B fragments
+    }
+    // no copy of this lane may still be in flight when the CTA exits
+    cp_async_wait_all();
+  } else if (warp == kWarpQrot) {
+    // ------------------------------------------------------------ q_rot of every tile
+    // lane m rotates pairs 2m, 2m + 1.  The angle of pair i at t0 = 128 jt is
+    // jt * frac(128 f_i) turns; frac(128 f_i) is held in 32-bit fixed point so
+    // that jt * F mod 2^32 is exact.
+    uint32_t Fq[2];
+    float qv[kG][4];                         // q[h][2m], [2m+1], [2m+64], [2m+65] * scale
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      double x = 128.0 * p.rope_f[(2 * lane + e) & (kHalf - 1)];
+      x -= floor(x);
+      Fq[e] = (uint32_t)(unsigned long long)llrint(x * 4294967296.0);
+    }
+#pragma unroll
+    for (int h = 0; h < kG; ++h) qv[h][0] = qv[h][1] = qv[h][2] = qv[h][3] = 0.f;
+    TileCursor cur(t_first, wk.tpu);
+    for (int jj = 0; jj < n_tiles; ++jj, cur.next()) {
       const int bd = slot_of<kNBLog2>(jj);
       if (jj == 0 || cur.jt == 0) {
         const int kvh = cur.u % p.Hkv, b = cur.u / p.Hkv;
@@ -293,13 +306,6 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.tile_in[bd]);
-    }
-    // drain: every issued stage must have landed before the CTA may exit
-    if (*abort && lane == 0) {
-      for (int jj = max(0, issued_upto - kStages); jj < issued_upto; ++jj) {
-        volatile int no_abort = 0;
-        mbar_wait(&bars.full[slot_of<kStagesLog2>(jj)], phase_of<kStagesLog2>(jj), &no_abort, nullptr);
-      }
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ reconstruction MMAs
