@@ -5,7 +5,7 @@
 // t ("JoLT: Near-Lossless KV Cache Compression", Key findings: the method works
 // pre-RoPE; the FlashJoLT decode "attends directly on the stored core,
 // factors and residual").  For a tile of 128 tokens starting at t0 the kernel
-//   1. stages the compressed rows with 16-byte cp.async copies,
+//   1. stages the compressed rows with 1-D bulk copies (no multicast),
 //   2. dequantizes L_k into TMEM and L_v into shared memory,
 //   3. reconstructs K_hat = L_k Bk with one tcgen05 MMA per 16 ranks
 //      (M = 128 tokens, N = 128 dims, f16 accumulator in TMEM),
@@ -33,8 +33,8 @@
 // number of bytes; a range may cross a unit boundary (a partial per part).
 //
 // Warp roles (480 threads, one CTA per SM):
-//   warp 0      producer: 8-stage ring of compressed tiles, 16-byte cp.async
-//               from all lanes, completion counted on the stage barrier
+//   warp 0      producer: 8-stage ring of compressed tiles, four 1-D bulk
+//               copies per tile (no multicast)
 //   warp 1      TMEM allocation + tcgen05 reconstruction MMAs (one lane)
 //   warps 2-5   dequantization (thread = token row), software-pipelined: the
 //               stage words of tile jj + 1 are loaded before tile jj is stored
@@ -43,7 +43,7 @@
 //               and value product of tile jj
 //   warp 14     q_rot of every tile
 // Every wait is bounded; on a timeout the CTA sets an error bit in the
-// workspace, drains its own copies and MMAs, frees TMEM and exits.
+// workspace, drains its own bulk copies and MMAs, frees TMEM and exits.
 #include <math.h>
 
 #include "kvc_device.cuh"
@@ -175,11 +175,12 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
   const int t_first = cta * wk.W;
   const int n_tiles = min(wk.W, wk.total - t_first);
   const int lk_row = p.lk_row, lv_row = p.lv_row, lksz_row = p.lksz_row, lvsz_row = p.lvsz_row;
+  const int stage_bytes = kTile * (lk_row + lksz_row + lv_row + lvsz_row);
   const int rv = p.rv;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars.full[s], 32);
+      mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 4);
     }
     for (int b = 0; b < kNB; ++b) {
@@ -211,9 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
 
   if (warp == kWarpProd) {
     // ------------------------------------------------------------ producer
-    // 16-byte cp.async copies spread over the 32 lanes (a tile's four
-    // components are 416 chunks); each lane's completion arrives on the
-    // stage's full barrier (32 arrivals per phase).
+    // one lane issues the tile's four components as 1-D bulk copies (no
+    // multicast) completing on the stage's full barrier
+    int issued_upto = 0;  // tiles issued
     TileCursor cur(t_first, wk.tpu);
     for (int jj = 0; jj < n_tiles && !*abort; ++jj, cur.next()) {
       const int s = slot_of<kStagesLog2>(jj);
@@ -226,37 +227,43 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
                                p.lv + row0 * lv_row,
                                reinterpret_cast<const uint8_t*>(p.lvsz) + row0 * lvsz_row};
       const int rowb[4] = {lk_row, lksz_row, lv_row, lvsz_row};
-      // 16-byte copies need 16-byte aligned sources: a unit base
-      // u * max_tokens * row is aligned only when max_tokens * row is a
-      // multiple of 16
+      // bulk copies need 16-byte aligned sources: a unit base u * max_tokens * row
+      // is aligned only when max_tokens * row is a multiple of 16
       bool aligned = true;
 #pragma unroll
       for (int c = 0; c < 4; ++c) aligned &= (reinterpret_cast<uintptr_t>(src[c]) & 15u) == 0;
-      int off = 0;
-      if (aligned) {
+      if (nt == kTile && aligned) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars.full[s], stage_bytes);
+          int off = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int bytes = nt * rowb[c];
-          for (int i = lane; 16 * i < bytes; i += 32) {
-            const int rem = bytes - 16 * i;
-            cp_async16(st + off + 16 * i, src[c] + 16 * i, rem < 16 ? rem : 16);
+          for (int c = 0; c < 4; ++c) {
+            bulk_g2s(st + off, src[c], kTile * rowb[c], &bars.full[s]);
+            off += kTile * rowb[c];
           }
-          off += kTile * rowb[c];
         }
-        cp_async_mbar_arrive(&bars.full[s]);
       } else {
-        // unaligned rows: plain copies of the nt valid rows
+        // ragged last tile of a unit, or unaligned rows: plain copies of the nt
+        // valid rows
+        int off = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int n = nt * rowb[c];
           for (int i = lane; i < n; i += 32) st[off + i] = src[c][i];
           off += kTile * rowb[c];
         }
-        mbar_arrive(&bars.full[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.full[s]);
+      }
+      issued_upto = jj + 1;
+    }
+    // drain: every issued stage must have landed before the CTA may exit
+    if (*abort && lane == 0) {
+      for (int jj = max(0, issued_upto - kStages); jj < issued_upto; ++jj) {
+        volatile int no_abort = 0;
+        mbar_wait(&bars.full[slot_of<kStagesLog2>(jj)], phase_of<kStagesLog2>(jj), &no_abort, nullptr);
       }
     }
-    // no copy of this lane may still be in flight when the CTA exits
-    cp_async_wait_all();
   } else if (warp == kWarpQrot) {
     // ------------------------------------------------------------ q_rot of every tile
     // lane m rotates pairs 2m, 2m + 1.  The angle of pair i at t0 = 128 jt is
