@@ -269,6 +269,21 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(torch, dist, value, device):
+    """The slowest rank's time: every rank passes its own device-timed value."""
+    if not dist:
+        return value
+    tt = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_rate(world, step_bytes, steps, ms):
+    """Whole-job compressed GB/s: the bytes of all ranks' replicas over the
+    max-over-ranks time."""
+    return world * step_bytes * steps / (ms / 1e3) / 1e9
+
+
 def workload_config(c, l2):
     return {"workload": WORKLOAD_NAME, "batch": c["B"], "q_heads": c["Hq"], "kv_heads": c["Hkv"],
             "head_dim": c["d"], "context": c["T"], "rank_k": c["rk"], "rank_v": c["rv"],
@@ -314,12 +329,9 @@ def run_kvc(args, rank, world, torch, dist):
     clocks = sampler.stop()
     ms = t0.elapsed_time(t1)
     hot_us = statistics.mean(e[0].elapsed_ms(e[1]) for e in ev) * 1e3
-    if dist:
-        tt = torch.tensor([ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(torch, dist, ms, device)
     ms_per_step = ms / K
-    value = world * step_bytes * K / (ms / 1e3) / 1e9
+    value = job_rate(world, step_bytes, K, ms)
 
     # end to end through the C ABI with host buffers: q in, output out, each step
     q_host = q.cpu().pin_memory()
@@ -340,11 +352,8 @@ def run_kvc(args, rank, world, torch, dist):
     t1.record(stream)
     torch.cuda.synchronize()
     ems = t0.elapsed_time(t1)
-    if dist:
-        tt = torch.tensor([ems], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ems = float(tt.item())
-    e2e = {"value": round(world * step_bytes * K / (ems / 1e3) / 1e9, 1), "unit": "GB/s",
+    ems = max_over_ranks(torch, dist, ems, device)
+    e2e = {"value": round(job_rate(world, step_bytes, K, ems), 1), "unit": "GB/s",
            "us_per_step": round(ems * 1e3 / K, 2),
            "h2d_bytes_per_step": int(q.numel() * q.element_size()),
            "d2h_bytes_per_step": int(out.numel() * out.element_size())}
