@@ -125,11 +125,115 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
   }
 }
 
+
+// Low-rank layouts without residual, head dim 128, value rank <= 64 and at
+// most 64 partials per row: every global load of the row (the partials'
+// maxima and sums, their accumulators, the Bv column slice) is issued before
+// any arithmetic, so the row costs one round trip to memory instead of one per
+// step.
+constexpr int kFastS = 64, kFastVals = 16;
+
+__global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
+  __shared__ float ws[kFastS];
+  __shared__ float red[kThreads];
+  __shared__ float acc[64];
+  __shared__ float lsum;
+  const int row = blockIdx.x;            // b * Hq + h
+  const int h = row % p.Hq;
+  const int kvh = h / p.G;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const size_t rows = (size_t)p.B * p.Hq;
+  const int pst = p.vdim + 2, rv = p.rv;
+  const float* part = p.part + (size_t)row * pst;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  int nS = p.S;
+  if (p.seg_W > 0) {
+    const int u = (row / p.Hq) * p.Hkv + kvh;
+    const long long a = (long long)u * p.seg_tpu, e = (long long)(u + 1) * p.seg_tpu - 1;
+    nS = (int)(e / p.seg_W - a / p.seg_W + 1) * p.seg_parts;
+  }
+  // ---- issue every load
+  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+  if (tid < 32) {
+    if (lane < nS) {
+      m_a = part[(size_t)lane * rows * pst + rv];
+      l_a = part[(size_t)lane * rows * pst + rv + 1];
+    }
+    if (lane + 32 < nS) {
+      m_b = part[(size_t)(lane + 32) * rows * pst + rv];
+      l_b = part[(size_t)(lane + 32) * rows * pst + rv + 1];
+    }
+  }
+  const int K = kThreads / rv;           // partial groups per value index
+  const int j = tid % rv, k = tid / rv;
+  float pv[kFastVals];
+#pragma unroll
+  for (int i = 0; i < kFastVals; ++i) {
+    const int sidx = k + i * K;
+    pv[i] = (k < K && sidx < nS) ? part[(size_t)sidx * rows * pst + j] : 0.f;
+  }
+  const int oi = tid & 127, half = tid >> 7;          // output dim, half of the ranks
+  const __half* bv = p.bv + (size_t)kvh * rv * 128 + oi;
+  float bw[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int r = half + 2 * i;
+    bw[i] = r < rv ? h2f(bv[(size_t)r * 128]) : 0.f;
+  }
+  // ---- weights
+  if (tid < 32) {
+    const float mx = warp_max(fmaxf(m_a, m_b));
+    const float wa = (mx == -INFINITY || m_a == -INFINITY) ? 0.f : exp2f(m_a - mx);
+    const float wb = (mx == -INFINITY || m_b == -INFINITY) ? 0.f : exp2f(m_b - mx);
+    if (lane < nS) ws[lane] = wa;
+    if (lane + 32 < nS) ws[lane + 32] = wb;
+    const float lt = warp_sum((wa != 0.f ? wa * l_a : 0.f) + (wb != 0.f ? wb * l_b : 0.f));
+    if (lane == 0) lsum = lt;
+  }
+  __syncthreads();
+  // ---- merge
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < kFastVals; ++i) {
+    const int sidx = k + i * K;
+    if (k < K && sidx < nS) {
+      const float w = ws[sidx];
+      if (w != 0.f) a = fmaf(w, pv[i], a);
+    }
+  }
+  red[tid] = a;
+  __syncthreads();
+  if (tid < rv) {
+    float t = 0.f;
+    for (int kk = 0; kk < K; ++kk) t += red[kk * rv + tid];
+    acc[tid] = t;
+  }
+  __syncthreads();
+  // ---- up-projection o = acc Bv / l (two halves of the ranks per output)
+  float o = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int r = half + 2 * i;
+    if (r < rv) o = fmaf(acc[r], bw[i], o);
+  }
+  red[tid] = o;
+  __syncthreads();
+  if (tid < 128) {
+    const float L = lsum;
+    const float t = (red[tid] + red[tid + 128]) * (L > 0.f ? 1.f / L : 0.f);
+    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * 128 + tid] = __float2bfloat16_rn(t);
+    else reinterpret_cast<float*>(p.out)[(size_t)row * 128 + tid] = t;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   if (p.S > kMaxS) return cudaErrorInvalidValue;
   const int rows = p.L * p.B * p.Hq;
+  const bool fast = p.kind == KVC_LOWRANK && !p.resid && p.d == 128 && p.L == 1 &&
+                    p.vdim == p.rv && p.rv >= 16 && p.rv <= 64 && p.S <= kFastS &&
+                    (p.S + kThreads / p.rv - 1) / (kThreads / p.rv) <= kFastVals;
   const size_t bytes = ((size_t)p.vdim + p.S + kThreads) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(combine_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -137,13 +241,14 @@ cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = bytes;
+  cfg.dynamicSmemBytes = fast ? 0 : bytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (fast) return cudaLaunchKernelEx(&cfg, combine_lowrank_kernel, p);
   return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 
