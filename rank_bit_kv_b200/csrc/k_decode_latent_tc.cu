@@ -1,0 +1,564 @@
+// Split-T decode on INT4 low-rank caches whose keys carry no RoPE, with or
+// without the 2-bit residual in the rotated (signed Walsh-Hadamard) basis,
+// contiguous or paged (16-token pages).  Attention runs in the latent space:
+//   s_t = q~ . l^k_t (+ q^ . y^k_t),   acc += sum_t p_t l^v_t (+ p_t y^v_t),
+// with q~ = Bk q and q^ = Q q from the query projection, and the combine
+// kernel maps acc back through Bv (and Q^T).
+//
+// Every warp streams its own contiguous range of 16-token tiles (one page of a
+// (batch row, KV head) unit) through a private ring of shared-memory stages
+// filled with 16-byte cp.async copies, and runs both contractions on mma.sync
+// m16n8k16 (f16 operands, fp32 accumulate) with the GQA group as N:
+//   - No code is dequantized element by element.  An INT4 or 2-bit code c,
+//     masked into the low mantissa bits of an f16 (exponent field zero), is
+//     the subnormal c * 2^-24 (times a power of two eps <= 256 for the fields
+//     that sit higher up in the mantissa, undone on the other operand or at the
+//     end).  The per-token scale and zero are applied after the score MMA
+//     (s = scale * (c . q~) + zero * sum(q~)) and, on the value side, folded
+//     into the probabilities (P' = p * scale as the B operand; the zero term
+//     sum_t p_t zero_t is kept on the CUDA cores).
+//   - The ordering of rank indices inside an MMA's K dimension is free (the
+//     query operand uses the same order), and so is the ordering of value rows
+//     (undone when the partials are written); both are chosen so that one
+//     32-bit shared-memory word feeds whole operand registers.
+//   - Online softmax with a lazily raised reference maximum (raised only when
+//     a score exceeds it by more than 8 in log2 units).
+// Shared-memory rows of 32 bytes are stored with tokens 4..7 (mod 8) swapped
+// pairwise, which makes the value-operand loads free of bank conflicts.
+#include <math.h>
+
+#include "kvc_device.cuh"
+#include "tc_util.cuh"
+
+namespace kvc {
+namespace {
+
+using namespace tc;
+
+constexpr int kLT = 16;                  // tokens per tile (one page)
+constexpr int kLWarps = 12;
+constexpr int kLThreads = 32 * kLWarps;
+constexpr int kLStages = 8;
+constexpr int kLRank = 32;               // key rank handled (one scale group)
+constexpr float kTwo24 = 16777216.f;     // code c held as the f16 bit pattern c is c * 2^-24
+
+// Stage layout of one tile: the components of the cache in their own order,
+// each the tile's 16 consecutive rows.
+template <int RV, bool RES>
+struct Stage {
+  static constexpr int NVG = (RV + 31) / 32;          // value scale groups
+  static constexpr int VT = RV / 16;                  // latent value M-tiles
+  static constexpr int LK = 0;
+  static constexpr int LKS = LK + kLT * kLRank / 2;
+  static constexpr int LV = LKS + kLT * 4;
+  static constexpr int LVS = LV + kLT * RV / 2;
+  static constexpr int RKC = LVS + kLT * NVG * 4;
+  static constexpr int RKS = RKC + (RES ? kLT * 32 : 0);
+  static constexpr int RVC = RKS + (RES ? kLT * 2 : 0);
+  static constexpr int RVS = RVC + (RES ? kLT * 32 : 0);
+  static constexpr int BYTES = RVS + (RES ? kLT * 2 : 0);
+  static constexpr int CHUNKS = BYTES / 16;
+  static constexpr int CPL = (CHUNKS + 31) / 32;     // chunks per lane
+  static constexpr int SMEM = kLWarps * kLStages * BYTES;
+};
+
+struct LWork {
+  int W, tpu, total;                     // tiles per warp, tiles per unit, all tiles
+};
+
+// smem row of token t in a component with 32-byte rows
+__device__ __forceinline__ int swz(int t) { return t ^ ((t >> 2) & 1); }
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 unpack_h2(uint32_t x) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&x));
+}
+
+__device__ __forceinline__ uint32_t lds32(const uint8_t* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
+
+// 2-bit field mu (0..7) of both 16-bit halves, scaled by eps2(mu)
+__host__ __device__ constexpr uint32_t mask2(int mu) {
+  return mu < 5 ? 0x00030003u << (2 * mu) : 0x00030003u << (2 * (mu - 3));
+}
+__host__ __device__ constexpr float eps2(int mu) {
+  return mu == 0 ? 1.f : mu == 1 ? 4.f : mu == 2 ? 16.f : mu == 3 ? 64.f
+       : mu == 4 ? 256.f : mu == 5 ? 16.f : mu == 6 ? 64.f : 256.f;
+}
+__device__ __forceinline__ uint32_t field2(uint32_t x, uint32_t x6, int mu) {
+  return (mu < 5 ? x : x6) & mask2(mu);
+}
+constexpr uint32_t kN0 = 0x000F000Fu;    // nibble 0 of both halves (eps 1)
+constexpr uint32_t kN1 = 0x00F000F0u;    // nibble 1 of both halves (eps 16)
+
+template <int RV, bool RES>
+__global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork wk) {
+  using L = Stage<RV, RES>;
+  constexpr int NVG = L::NVG, VT = L::VT;
+  constexpr bool kHalfGroup = (RV % 32) != 0;   // last value group holds 16 ranks
+  extern __shared__ __align__(128) uint8_t lsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * kLWarps + warp;
+  const int t_first = gw * wk.W;
+  const int n_tiles = min(wk.W, wk.total - t_first);
+  if (n_tiles <= 0) return;
+  uint8_t* ring = lsm + warp * (kLStages * L::BYTES);
+  const int G = p.G, Hkv = p.Hkv;
+  const int g = lane >> 2, c4 = lane & 3;
+  const size_t rows_q = (size_t)p.B * p.Hq;
+  const int pst = p.vdim + 2;
+  const int npp = p.tmax / kLT;          // tiles (pages) per batch row
+
+  // ---- this lane's copy chunks: source component, its row bytes, smem offset
+  const uint8_t* c_src[L::CPL];
+  int c_rowb[L::CPL], c_dst[L::CPL], c_tok[L::CPL];
+#pragma unroll
+  for (int i = 0; i < L::CPL; ++i) {
+    const int c = lane + 32 * i, o = 16 * c;
+    const uint8_t* base;
+    int off, rowb;
+    if (o < L::LKS) base = p.lk, off = L::LK, rowb = kLRank / 2;
+    else if (o < L::LV) base = reinterpret_cast<const uint8_t*>(p.lksz), off = L::LKS, rowb = 4;
+    else if (o < L::LVS) base = p.lv, off = L::LV, rowb = RV / 2;
+    else if (o < L::RKC) base = reinterpret_cast<const uint8_t*>(p.lvsz), off = L::LVS, rowb = NVG * 4;
+    else if (o < L::RKS) base = p.rkc, off = L::RKC, rowb = 32;
+    else if (o < L::RVC) base = reinterpret_cast<const uint8_t*>(p.rks), off = L::RKS, rowb = 2;
+    else if (o < L::RVS) base = p.rvc, off = L::RVC, rowb = 32;
+    else base = reinterpret_cast<const uint8_t*>(p.rvs), off = L::RVS, rowb = 2;
+    const int j = (o - off) / 16;                        // chunk within the component
+    c_src[i] = base + (size_t)16 * j;
+    c_rowb[i] = rowb;
+    c_tok[i] = c < L::CHUNKS ? (16 * j) / rowb : kLT;    // first token of the chunk
+    c_dst[i] = off + (rowb == 32 ? 32 * swz(j >> 1) + 16 * (j & 1) : 16 * j);
+  }
+
+  // ---- first cache row of tile t of the range (page table or contiguous),
+  // produced 32 tiles at a time, one per lane, a block ahead of its use
+  auto tile_row = [&](int jj) -> int {
+    const int t = t_first + jj;
+    if (jj >= n_tiles) return 0;
+    const int u = t / wk.tpu, jt = t % wk.tpu;
+    const int b = u / Hkv, kvh = u % Hkv;
+    if (p.page) return (__ldg(p.page_table + (size_t)b * npp + jt) * Hkv + kvh) * kLT;
+    return u * p.tmax + jt * kLT;
+  };
+  int rows_cur = tile_row(lane), rows_next = tile_row(32 + lane);
+
+  auto issue = [&](int jj, int row0) {
+    const int t = t_first + jj;
+    const int jt = t % wk.tpu;
+    const int nt = min(kLT, p.n_tokens - jt * kLT);
+    uint8_t* st = ring + (jj % kLStages) * L::BYTES;
+#pragma unroll
+    for (int i = 0; i < L::CPL; ++i) {
+      if (lane + 32 * i < L::CHUNKS)
+        cp_async16(st + c_dst[i], c_src[i] + (size_t)row0 * c_rowb[i], c_tok[i] < nt ? 16 : 0);
+    }
+  };
+
+  // prologue: kLStages - 1 tiles in flight
+#pragma unroll
+  for (int i = 0; i < kLStages - 1; ++i) {
+    const int r = __shfl_sync(0xffffffffu, rows_cur, i);
+    if (i < n_tiles) issue(i, r);
+    cp_async_commit();
+  }
+
+  // ---- per-unit state
+  uint32_t bq[2][2];                     // q~ (latent key) B fragments
+  uint32_t br[RES ? 8 : 1][2];           // q^ (residual key) B fragments
+  float sumL[2], sumR[2];                // sum of the effective q~ / q^ of columns 2c4 + e
+  float m_ref[2], m_thr[2], l_sum[2];
+  float accV[VT][4];
+  float accR[RES ? 8 : 1][4];
+  float zs[NVG][2];                      // sum_t p_t zero_t per value group
+  float sR[2];                           // sum_t p_t scale_t of the residual
+  int cur_u = -1, cur_slot = 0;
+
+  auto reset = [&](int u) {
+    const int b = u / Hkv, kvh = u % Hkv;
+    const float sl = p.scale_log2;
+    const bool vq = g < G;
+    const float* qr = p.qt + ((size_t)b * p.Hq + kvh * G + min(g, G - 1)) * p.qdim;
+    float own_l = 0.f, own_r = 0.f;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int r0 = 8 * c4 + 2 * s;
+      const float x0 = vq ? qr[r0] * sl : 0.f, x4 = vq ? qr[r0 + 4] * sl : 0.f;
+      const float x1 = vq ? qr[r0 + 1] * sl * (1.f / 16.f) : 0.f;
+      const float x5 = vq ? qr[r0 + 5] * sl * (1.f / 16.f) : 0.f;
+      bq[s][0] = pack_h2(x0, x4);
+      bq[s][1] = pack_h2(x1, x5);
+      const float2 e0 = unpack_h2(bq[s][0]), e1 = unpack_h2(bq[s][1]);
+      own_l += e0.x + e0.y + 16.f * (e1.x + e1.y);
+    }
+    if constexpr (RES) {
+      const float* qh = qr + kLRank;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int w = 2 * c4 + (s >> 2), k = s & 3;
+        const int d0 = 16 * w + 2 * k;
+        const float e_a = eps2(2 * k), e_b = eps2(2 * k + 1);
+        const float y0 = vq ? qh[d0] * sl / e_a : 0.f, y8 = vq ? qh[d0 + 8] * sl / e_a : 0.f;
+        const float y1 = vq ? qh[d0 + 1] * sl / e_b : 0.f, y9 = vq ? qh[d0 + 9] * sl / e_b : 0.f;
+        br[s][0] = pack_h2(y0, y8);
+        br[s][1] = pack_h2(y1, y9);
+        const float2 f0 = unpack_h2(br[s][0]), f1 = unpack_h2(br[s][1]);
+        own_r += e_a * (f0.x + f0.y) + e_b * (f1.x + f1.y);
+      }
+    }
+    own_l += __shfl_xor_sync(0xffffffffu, own_l, 1);
+    own_l += __shfl_xor_sync(0xffffffffu, own_l, 2);
+    own_r += __shfl_xor_sync(0xffffffffu, own_r, 1);
+    own_r += __shfl_xor_sync(0xffffffffu, own_r, 2);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      sumL[e] = __shfl_sync(0xffffffffu, own_l, 4 * (2 * c4 + e));
+      sumR[e] = __shfl_sync(0xffffffffu, own_r, 4 * (2 * c4 + e));
+      m_ref[e] = m_thr[e] = -INFINITY;
+      l_sum[e] = 0.f;
+      sR[e] = 0.f;
+#pragma unroll
+      for (int v = 0; v < NVG; ++v) zs[v][e] = 0.f;
+    }
+#pragma unroll
+    for (int mt = 0; mt < VT; ++mt) accV[mt][0] = accV[mt][1] = accV[mt][2] = accV[mt][3] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < (RES ? 8 : 1); ++mt)
+      accR[mt][0] = accR[mt][1] = accR[mt][2] = accR[mt][3] = 0.f;
+  };
+
+  auto write_partial = [&]() {
+    float l2[2] = {l_sum[0], l_sum[1]}, s2[2] = {sR[0], sR[1]};
+    float z2[NVG][2];
+#pragma unroll
+    for (int v = 0; v < NVG; ++v) z2[v][0] = zs[v][0], z2[v][1] = zs[v][1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        l2[e] += __shfl_xor_sync(0xffffffffu, l2[e], o);
+        s2[e] += __shfl_xor_sync(0xffffffffu, s2[e], o);
+#pragma unroll
+        for (int v = 0; v < NVG; ++v) z2[v][e] += __shfl_xor_sync(0xffffffffu, z2[v][e], o);
+      }
+    }
+    const int b = cur_u / Hkv, kvh = cur_u % Hkv;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * c4 + e;
+      if (h >= G) continue;
+      float* dst = p.part + ((size_t)cur_slot * rows_q + (size_t)b * p.Hq + kvh * G + h) * pst;
+#pragma unroll
+      for (int mt = 0; mt < VT; ++mt) {
+        const int v = mt >> 1;
+        int r0;
+        if (kHalfGroup && mt == VT - 1) r0 = 32 * v + 2 * g;
+        else r0 = 32 * v + 4 * g + 2 * (mt & 1);
+        dst[r0] = accV[mt][e] * kTwo24 + z2[v][e];
+        dst[r0 + 1] = accV[mt][2 + e] * (kTwo24 / 16.f) + z2[v][e];
+      }
+      if constexpr (RES) {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int k0 = 2 * mt;
+          dst[RV + 16 * g + k0] = accR[mt][e] * (kTwo24 / eps2(k0 & 7)) - 1.5f * s2[e];
+          dst[RV + 16 * g + k0 + 1] = accR[mt][2 + e] * (kTwo24 / eps2((k0 + 1) & 7)) - 1.5f * s2[e];
+        }
+      }
+      if (g == 0) {
+        dst[p.vdim] = m_ref[e];
+        dst[p.vdim + 1] = l2[e];
+      }
+    }
+  };
+
+  // value-operand selectors: bytes (2h, 2h + 1) of two words side by side
+  const uint32_t sel_v = (g & 1) ? 0x7632u : 0x5410u;
+  const uint32_t bh = g & 3;
+  const uint32_t sel_h = bh | (bh << 4) | ((4 + bh) << 8) | ((4 + bh) << 12);
+  const int tA0 = 2 * c4, tA1 = 2 * c4 + 1, tB0 = 2 * c4 + 8, tB1 = 2 * c4 + 9;
+
+  for (int jj = 0; jj < n_tiles; ++jj) {
+    const int t = t_first + jj;
+    const int u = t / wk.tpu, jt = t % wk.tpu;
+    const int nt = min(kLT, p.n_tokens - jt * kLT);
+    if (u != cur_u) {
+      if (cur_u >= 0) write_partial();
+      cur_u = u;
+      cur_slot = gw - (int)(((long long)u * wk.tpu) / wk.W);
+      reset(u);
+    }
+    // keep kLStages - 1 tiles in flight; the cache rows come 32 tiles at a time
+    {
+      const int ji = jj + kLStages - 1;
+      if ((ji & 31) == 0 && ji > 0) {
+        rows_cur = rows_next;
+        rows_next = tile_row(ji + 32 + lane);
+      }
+      const int r = __shfl_sync(0xffffffffu, rows_cur, ji & 31);
+      if (ji < n_tiles) issue(ji, r);
+    }
+    cp_async_commit();
+    cp_async_wait<kLStages - 1>();
+    __syncwarp();
+    const uint8_t* st = ring + (jj % kLStages) * L::BYTES;
+
+    // ---------------- scores: rows g, g + 8 = tokens; columns 2c4, 2c4 + 1 = heads
+    float s[4];
+    {
+      const uint32_t k0 = lds32(st + L::LK + 16 * g + 4 * c4);
+      const uint32_t k1 = lds32(st + L::LK + 16 * (g + 8) + 4 * c4);
+      float aL[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const uint32_t a[4] = {k0 & kN0, k1 & kN0, k0 & kN1, k1 & kN1};
+        mma16816(aL, a, bq[0][0], bq[0][1]);
+        const uint32_t y0 = k0 >> 8, y1 = k1 >> 8;
+        const uint32_t a2[4] = {y0 & kN0, y1 & kN0, y0 & kN1, y1 & kN1};
+        mma16816(aL, a2, bq[1][0], bq[1][1]);
+      }
+      const float2 sz0 = unpack_h2(lds32(st + L::LKS + 4 * g));
+      const float2 sz1 = unpack_h2(lds32(st + L::LKS + 4 * (g + 8)));
+      float c0[2], c1[2];                // per-token constant of each column
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        c0[e] = sz0.y * sumL[e];
+        c1[e] = sz1.y * sumL[e];
+      }
+      float aR0[4] = {0.f, 0.f, 0.f, 0.f}, aR1[4] = {0.f, 0.f, 0.f, 0.f};
+      float sr0 = 0.f, sr1 = 0.f;
+      if constexpr (RES) {
+        const uint2 r0 = *reinterpret_cast<const uint2*>(st + L::RKC + 32 * swz(g) + 8 * c4);
+        const uint2 r1 = *reinterpret_cast<const uint2*>(st + L::RKC + 32 * swz(g + 8) + 8 * c4);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t w0 = h ? r0.y : r0.x, w1 = h ? r1.y : r1.x;
+          const uint32_t w06 = w0 >> 6, w16 = w1 >> 6;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t a[4] = {field2(w0, w06, 2 * k), field2(w1, w16, 2 * k),
+                                   field2(w0, w06, 2 * k + 1), field2(w1, w16, 2 * k + 1)};
+            if (k & 1) mma16816(aR1, a, br[4 * h + k][0], br[4 * h + k][1]);
+            else mma16816(aR0, a, br[4 * h + k][0], br[4 * h + k][1]);
+          }
+        }
+        sr0 = __half2float(*reinterpret_cast<const __half*>(st + L::RKS + 2 * g));
+        sr1 = __half2float(*reinterpret_cast<const __half*>(st + L::RKS + 2 * (g + 8)));
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          c0[e] = fmaf(-1.5f * sr0, sumR[e], c0[e]);
+          c1[e] = fmaf(-1.5f * sr1, sumR[e], c1[e]);
+        }
+      }
+      const float k0s = sz0.x * kTwo24, k1s = sz1.x * kTwo24;
+      const float r0s = sr0 * kTwo24, r1s = sr1 * kTwo24;
+      s[0] = fmaf(k0s, aL[0], fmaf(r0s, aR0[0] + aR1[0], c0[0]));
+      s[1] = fmaf(k0s, aL[1], fmaf(r0s, aR0[1] + aR1[1], c0[1]));
+      s[2] = fmaf(k1s, aL[2], fmaf(r1s, aR0[2] + aR1[2], c1[0]));
+      s[3] = fmaf(k1s, aL[3], fmaf(r1s, aR0[3] + aR1[3], c1[1]));
+      if (nt < kLT) {
+        if (g >= nt) s[0] = s[1] = -INFINITY;
+        if (g + 8 >= nt) s[2] = s[3] = -INFINITY;
+      }
+    }
+
+    // ---------------- online softmax (lazy maximum, raised by more than 2^8)
+    const bool need = s[0] > m_thr[0] || s[2] > m_thr[0] || s[1] > m_thr[1] || s[3] > m_thr[1];
+    if (__any_sync(0xffffffffu, need)) {
+      float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float n0 = fmaxf(m_ref[0], mx0), n1 = fmaxf(m_ref[1], mx1);
+      const float al[2] = {ex2_approx(m_ref[0] - n0), ex2_approx(m_ref[1] - n1)};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        l_sum[e] *= al[e];
+        sR[e] *= al[e];
+#pragma unroll
+        for (int v = 0; v < NVG; ++v) zs[v][e] *= al[e];
+#pragma unroll
+        for (int mt = 0; mt < VT; ++mt) accV[mt][e] *= al[e], accV[mt][2 + e] *= al[e];
+        if constexpr (RES) {
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) accR[mt][e] *= al[e], accR[mt][2 + e] *= al[e];
+        }
+      }
+      m_ref[0] = n0;
+      m_ref[1] = n1;
+      m_thr[0] = n0 + 8.f;
+      m_thr[1] = n1 + 8.f;
+    }
+    float pv[4];
+    pv[0] = ex2_approx(s[0] - m_ref[0]);
+    pv[1] = ex2_approx(s[1] - m_ref[1]);
+    pv[2] = ex2_approx(s[2] - m_ref[0]);
+    pv[3] = ex2_approx(s[3] - m_ref[1]);
+    if (nt < kLT) {
+      if (g >= nt) pv[0] = pv[1] = 0.f;
+      if (g + 8 >= nt) pv[2] = pv[3] = 0.f;
+    }
+    l_sum[0] += pv[0] + pv[2];
+    l_sum[1] += pv[1] + pv[3];
+
+    // ---------------- values: acc^T (value row x head) += V^T (row x token) P'
+    {
+      // scales and zeros of tokens g, g + 8 (zeroed past the end of the unit)
+      float vs[NVG][2], vz[NVG][2];
+#pragma unroll
+      for (int v = 0; v < NVG; ++v) {
+        const float2 a0 = unpack_h2(lds32(st + L::LVS + NVG * 4 * g + 4 * v));
+        const float2 a1 = unpack_h2(lds32(st + L::LVS + NVG * 4 * (g + 8) + 4 * v));
+        vs[v][0] = a0.x;
+        vz[v][0] = a0.y;
+        vs[v][1] = a1.x;
+        vz[v][1] = a1.y;
+      }
+      if (nt < kLT) {
+#pragma unroll
+        for (int v = 0; v < NVG; ++v) {
+          if (g >= nt) vs[v][0] = vz[v][0] = 0.f;
+          if (g + 8 >= nt) vs[v][1] = vz[v][1] = 0.f;
+        }
+      }
+      auto rowv = [&](int tok) -> int { return RV == 64 ? 32 * swz(tok) : (RV / 2) * tok; };
+#pragma unroll
+      for (int v = 0; v < NVG; ++v) {
+        zs[v][0] = fmaf(pv[0], vz[v][0], fmaf(pv[2], vz[v][1], zs[v][0]));
+        zs[v][1] = fmaf(pv[1], vz[v][0], fmaf(pv[3], vz[v][1], zs[v][1]));
+        const uint32_t h01 = pack_h2(pv[0] * vs[v][0], pv[1] * vs[v][0]);
+        const uint32_t h23 = pack_h2(pv[2] * vs[v][1], pv[3] * vs[v][1]);
+        const uint32_t b0 = movmatrix_trans(h01), b1 = movmatrix_trans(h23);
+        const bool half = kHalfGroup && v == NVG - 1;
+        const int word = half ? 4 * v + (g >> 2) : 4 * v + (g >> 1);
+        const uint32_t sel = half ? sel_h : sel_v;
+        const uint32_t xA = prmt(lds32(st + L::LV + rowv(tA0) + 4 * word),
+                                 lds32(st + L::LV + rowv(tA1) + 4 * word), sel);
+        const uint32_t xB = prmt(lds32(st + L::LV + rowv(tB0) + 4 * word),
+                                 lds32(st + L::LV + rowv(tB1) + 4 * word), sel);
+        {
+          const uint32_t a[4] = {xA & kN0, xA & kN1, xB & kN0, xB & kN1};
+          mma16816(accV[2 * v], a, b0, b1);
+        }
+        if (!half) {
+          const uint32_t yA = xA >> 8, yB = xB >> 8;
+          const uint32_t a[4] = {yA & kN0, yA & kN1, yB & kN0, yB & kN1};
+          mma16816(accV[2 * v + 1], a, b0, b1);
+        }
+      }
+      if constexpr (RES) {
+        float rs0 = __half2float(*reinterpret_cast<const __half*>(st + L::RVS + 2 * g));
+        float rs1 = __half2float(*reinterpret_cast<const __half*>(st + L::RVS + 2 * (g + 8)));
+        if (nt < kLT) {
+          if (g >= nt) rs0 = 0.f;
+          if (g + 8 >= nt) rs1 = 0.f;
+        }
+        const float q0 = pv[0] * rs0, q1 = pv[1] * rs0, q2 = pv[2] * rs1, q3 = pv[3] * rs1;
+        sR[0] += q0 + q2;
+        sR[1] += q1 + q3;
+        const uint32_t b0 = movmatrix_trans(pack_h2(q0, q1));
+        const uint32_t b1 = movmatrix_trans(pack_h2(q2, q3));
+        const uint32_t wA0 = lds32(st + L::RVC + 32 * swz(tA0) + 4 * g);
+        const uint32_t wA1 = lds32(st + L::RVC + 32 * swz(tA1) + 4 * g);
+        const uint32_t wB0 = lds32(st + L::RVC + 32 * swz(tB0) + 4 * g);
+        const uint32_t wB1 = lds32(st + L::RVC + 32 * swz(tB1) + 4 * g);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t sl = hh ? 0x7632u : 0x5410u;
+          const uint32_t xA = prmt(wA0, wA1, sl), xB = prmt(wB0, wB1, sl);
+          const uint32_t xA6 = xA >> 6, xB6 = xB >> 6;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t a[4] = {field2(xA, xA6, 2 * k), field2(xA, xA6, 2 * k + 1),
+                                   field2(xB, xB6, 2 * k), field2(xB, xB6, 2 * k + 1)};
+            mma16816(accR[4 * hh + k], a, b0, b1);
+          }
+        }
+      }
+    }
+    __syncwarp();                        // this stage is refilled next iteration
+  }
+  cp_async_wait<0>();
+  write_partial();
+}
+
+template <int RV, bool RES>
+cudaError_t launch_t(const Params& p, const LWork& wk, int grid, cudaStream_t s) {
+  using L = Stage<RV, RES>;
+  cudaError_t e = cudaFuncSetAttribute(latent_tc_kernel<RV, RES>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  if (e != cudaSuccess) return e;
+  latent_tc_kernel<RV, RES><<<grid, kLThreads, L::SMEM, s>>>(p, wk);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool latent_tc_supported(const Params& p) {
+  if (p.kind != KVC_LOWRANK || p.rope || p.bits != 4 || p.g != 32 || p.d != 128) return false;
+  if (p.rk != kLRank || (p.rv != 32 && p.rv != 48 && p.rv != 64)) return false;
+  if (p.resid != 0 && p.resid != 2) return false;
+  if (p.page != 0 && p.page != kLT) return false;
+  if (p.L != 1 || p.seq_lens || p.n_tokens <= 0 || p.G < 1 || p.G > 8) return false;
+  if (p.tmax % kLT) return false;
+  const long long rows = p.page ? (long long)p.n_pages * p.Hkv * kLT : (long long)p.B * p.Hkv * p.tmax;
+  return rows < (1LL << 31) && p.vdim == p.rv + (p.resid ? kResidDim : 0) &&
+         p.qdim == p.rk + (p.resid ? kResidDim : 0);
+}
+
+// Equal contiguous tile ranges per warp; a unit of tpu tiles spans at most
+// ceil(tpu / W) + 1 warps, each writing one partial.
+void latent_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots) {
+  const int t = (p.n_tokens + kLT - 1) / kLT;
+  const long long total = (long long)p.B * p.Hkv * t;
+  const long long warps_max = (long long)kNumSMs * kLWarps;
+  const long long w = (total + warps_max - 1) / warps_max;
+  const long long n_warps = (total + w - 1) / w;
+  *grid = (int)((n_warps + kLWarps - 1) / kLWarps);
+  *W = (int)w;
+  *tpu = t;
+  *slots = (int)((t + w - 1) / w + 1);
+}
+
+int latent_tc_slots(int batch, int n_kv_heads, int n_tokens) {
+  const int t = (n_tokens + kLT - 1) / kLT;
+  const long long total = (long long)batch * n_kv_heads * t;
+  const long long warps_max = (long long)kNumSMs * kLWarps;
+  const long long w = (total + warps_max - 1) / warps_max;
+  return (int)((t + w - 1) / w + 1);
+}
+
+cudaError_t launch_latent_tc(const Params& p, cudaStream_t s) {
+  int grid, W, tpu, slots;
+  latent_tc_plan(p, &grid, &W, &tpu, &slots);
+  const LWork wk{W, tpu, p.B * p.Hkv * tpu};
+  const bool res = p.resid != 0;
+  switch (p.rv) {
+    case 32: return res ? launch_t<32, true>(p, wk, grid, s) : launch_t<32, false>(p, wk, grid, s);
+    case 48: return res ? launch_t<48, true>(p, wk, grid, s) : launch_t<48, false>(p, wk, grid, s);
+    default: return res ? launch_t<64, true>(p, wk, grid, s) : launch_t<64, false>(p, wk, grid, s);
+  }
+}
+
+}  // namespace kvc

@@ -358,7 +358,9 @@ __global__ void __launch_bounds__(kThreads) split_generic_kernel(Params p) {
 
 cudaError_t launch_split(const Params& p, cudaStream_t s) {
   if (p.seg_W > 0)
-    return p.kind == KVC_DENSE_BF16 ? launch_dense_tc(p, s) : launch_rope_tc(p, p.err, s);
+    return p.kind == KVC_DENSE_BF16 ? launch_dense_tc(p, s)
+           : p.rope                 ? launch_rope_tc(p, p.err, s)
+                                    : launch_latent_tc(p, s);
   const Geo g = geometry(p);
   const Smem S = carve(p, g);
   const size_t bytes = (size_t)S.total * sizeof(float);

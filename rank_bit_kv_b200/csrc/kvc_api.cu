@@ -78,10 +78,15 @@ int fast_slots(const kvc_layout* L, int n_tokens) {
 size_t ws_bytes(const kvc_layout* L, int n_tokens) {
   int S, len;
   plan(L, n_tokens, &S, &len);
+  const int nt1 = n_tokens > 0 ? n_tokens : 1;
   const int Sf = L->d.kind == KVC_DENSE_BF16
-                     ? kvc::dense_tc_slots(L->d.batch, L->d.n_kv_heads, n_tokens > 0 ? n_tokens : 1)
+                     ? kvc::dense_tc_slots(L->d.batch, L->d.n_kv_heads, nt1)
                      : fast_slots(L, n_tokens);
   if (Sf > S) S = Sf;
+  if (L->d.kind == KVC_LOWRANK) {
+    const int Sl = kvc::latent_tc_slots(L->d.batch, L->d.n_kv_heads, nt1);
+    if (Sl > S) S = Sl;
+  }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   size_t b = kWsHeader + round_up(rows * L->qdim * sizeof(float), 256);
   b += round_up((size_t)S * rows * (L->vdim + 2) * sizeof(float), 256);
@@ -449,6 +454,13 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
     p.seg_W = W;
     p.seg_tpu = tpu;
     p.seg_parts = kvc::kRopeTcParts;
+  } else if (kvc::latent_tc_supported(p)) {
+    int grid, W, tpu, slots;
+    kvc::latent_tc_plan(p, &grid, &W, &tpu, &slots);
+    p.S = slots;
+    p.seg_W = W;
+    p.seg_tpu = tpu;
+    p.seg_parts = 1;
   } else if (kvc::dense_tc_supported(p)) {
     int grid, W, tpu, slots;
     kvc::dense_tc_plan(p, &grid, &W, &tpu, &slots);

@@ -111,6 +111,13 @@ void dense_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
 int dense_tc_slots(int batch, int n_kv_heads, int n_tokens);
 cudaError_t launch_dense_tc(const Params& p, cudaStream_t s);
 
+// warp-level tensor-core decode of INT4 low-rank caches without RoPE (latent-
+// space scores), with or without the rotated 2-bit residual, contiguous or paged
+bool latent_tc_supported(const Params& p);
+void latent_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
+int latent_tc_slots(int batch, int n_kv_heads, int n_tokens);
+cudaError_t launch_latent_tc(const Params& p, cudaStream_t s);
+
 // Record a status and message for kvc_last_error(); returns st.
 kvc_status report_error(kvc_status st, const char* fmt, ...);
 

@@ -253,3 +253,36 @@ def test_rope_tensor_core_path_against_oracle_and_generic(B, T):
     kvc.decode(lay, cache, q, out, ws)
     torch.cuda.synchronize()
     assert_close(out.cpu().numpy(), ref, what=f"generic B={B} T={T}")
+
+
+# ------------------------------------------------------------------ latent-space tensor-core path
+
+
+@pytest.mark.parametrize("rv,resid,page,Hq,B,n,cap", [
+    (64, 2, 16, 32, 2, 400, 400),     # C5 shape, paged, whole pages
+    (64, 2, 16, 32, 2, 333, 400),     # ragged last page
+    (64, 2, 0, 8, 1, 1, 32),          # one token, contiguous, one query head per KV head
+    (48, 0, 0, 32, 2, 1000, 1008),    # C2 ranks without RoPE, contiguous
+    (48, 2, 16, 16, 3, 4111, 4112),   # two query heads per KV head
+    (32, 0, 16, 64, 2, 2049, 2064),   # eight query heads per KV head
+    (32, 2, 0, 32, 1, 17, 32),        # one full tile and one token
+])
+def test_latent_tensor_core_path(rv, resid, page, Hq, B, n, cap):
+    """INT4 low-rank layouts without RoPE run on the warp-level mma.sync kernel
+    (latent-space scores; codes used as MMA operands without dequantization).
+    Per-row lengths force the generic CUDA-core kernel; both must match the oracle."""
+    c = synth.config("c5", B=B, Hq=Hq, T=cap, rv=rv, resid=resid, page=page, seed=11 + rv)
+    a = synth.lowrank_cache(c)
+    ref = oracle(c, a, n)
+    assert_close(run_decode(c, a, n, capacity=cap), ref, what=f"latent mma rv={rv} n={n}")
+    got = run_decode(c, a, n, capacity=cap, seq_lens=[n] * B)
+    assert_close(got, ref, what=f"generic rv={rv} n={n}")
+
+
+def test_latent_tensor_core_peaked():
+    """q scaled by 8: scores spread over tens of log2 units, so the lazily raised
+    softmax maximum is raised many times inside a warp's range."""
+    c = synth.config("c5", B=2, T=4096)
+    a = synth.lowrank_cache(c)
+    a["q"] = synth.to_bf16_bits(synth.bf16_bits_to_f32(a["q"]) * 8)
+    assert_close(run_decode(c, a, 4096), oracle(c, a, 4096), what="latent peaked")
