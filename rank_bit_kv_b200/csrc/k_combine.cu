@@ -126,24 +126,25 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
 }
 
 
-// Low-rank layouts without residual, head dim 128, value rank <= 64 and at
-// most 64 partials per row: every global load of the row (the partials'
-// maxima and sums, their accumulators, the Bv column slice) is issued before
-// any arithmetic, so the row costs one round trip to memory instead of one per
-// step.
+// Low-rank layouts, head dim 128, value rank <= 64 (plus the 128 rotated
+// residual values, if any) and few partials per row: every global load of the
+// row (the partials' maxima and sums, their accumulators, the Bv column slice,
+// the signs) is issued before any arithmetic, so the row costs one round trip
+// to memory instead of one per step.  The residual accumulator is mapped back
+// with the in-register Hadamard transform of one warp.
 constexpr int kFastS = 64, kFastVals = 16;
 
 __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
   __shared__ float ws[kFastS];
   __shared__ float red[kThreads];
-  __shared__ float acc[64];
+  __shared__ float acc[256];
   __shared__ float lsum;
   const int row = blockIdx.x;            // b * Hq + h
   const int h = row % p.Hq;
   const int kvh = h / p.G;
   const int tid = threadIdx.x, lane = tid & 31;
   const size_t rows = (size_t)p.B * p.Hq;
-  const int pst = p.vdim + 2, rv = p.rv;
+  const int pst = p.vdim + 2, rv = p.rv, vdim = p.vdim;
   const float* part = p.part + (size_t)row * pst;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int nS = p.S;
@@ -156,16 +157,16 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
   float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
   if (tid < 32) {
     if (lane < nS) {
-      m_a = part[(size_t)lane * rows * pst + rv];
-      l_a = part[(size_t)lane * rows * pst + rv + 1];
+      m_a = part[(size_t)lane * rows * pst + vdim];
+      l_a = part[(size_t)lane * rows * pst + vdim + 1];
     }
     if (lane + 32 < nS) {
-      m_b = part[(size_t)(lane + 32) * rows * pst + rv];
-      l_b = part[(size_t)(lane + 32) * rows * pst + rv + 1];
+      m_b = part[(size_t)(lane + 32) * rows * pst + vdim];
+      l_b = part[(size_t)(lane + 32) * rows * pst + vdim + 1];
     }
   }
-  const int K = kThreads / rv;           // partial groups per value index
-  const int j = tid % rv, k = tid / rv;
+  const int K = kThreads / vdim;         // partial groups per value index
+  const int j = tid % vdim, k = tid / vdim;
   float pv[kFastVals];
 #pragma unroll
   for (int i = 0; i < kFastVals; ++i) {
@@ -180,6 +181,7 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
     const int r = half + 2 * i;
     bw[i] = r < rv ? h2f(bv[(size_t)r * 128]) : 0.f;
   }
+  const float sgn = p.resid ? (float)p.signs_v[oi] * rsqrtf((float)kResidDim) : 0.f;
   // ---- weights
   if (tid < 32) {
     const float mx = warp_max(fmaxf(m_a, m_b));
@@ -203,12 +205,24 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
   }
   red[tid] = a;
   __syncthreads();
-  if (tid < rv) {
+  if (tid < vdim) {
     float t = 0.f;
-    for (int kk = 0; kk < K; ++kk) t += red[kk * rv + tid];
+    for (int kk = 0; kk < K; ++kk) t += red[kk * vdim + tid];
     acc[tid] = t;
   }
   __syncthreads();
+  if (p.resid) {
+    // Q^T acc_res = diag(signs_v) H acc_res / sqrt(128); H here, the rest below
+    if (tid < 32) {
+      float x[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) x[kk] = acc[rv + 4 * lane + kk];
+      fwht128_warp(x, lane);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) acc[rv + 4 * lane + kk] = x[kk];
+    }
+    __syncthreads();
+  }
   // ---- up-projection o = acc Bv / l (two halves of the ranks per output)
   float o = 0.f;
 #pragma unroll
@@ -216,6 +230,7 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
     const int r = half + 2 * i;
     if (r < rv) o = fmaf(acc[r], bw[i], o);
   }
+  if (p.resid && half) o = fmaf(sgn, acc[rv + oi], o);
   red[tid] = o;
   __syncthreads();
   if (tid < 128) {
@@ -231,9 +246,10 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
 cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   if (p.S > kMaxS) return cudaErrorInvalidValue;
   const int rows = p.L * p.B * p.Hq;
-  const bool fast = p.kind == KVC_LOWRANK && !p.resid && p.d == 128 && p.L == 1 &&
-                    p.vdim == p.rv && p.rv >= 16 && p.rv <= 64 && p.S <= kFastS &&
-                    (p.S + kThreads / p.rv - 1) / (kThreads / p.rv) <= kFastVals;
+  const bool fast = p.kind == KVC_LOWRANK && p.d == 128 && p.L == 1 &&
+                    p.vdim == p.rv + (p.resid ? kResidDim : 0) && p.rv >= 16 && p.rv <= 64 &&
+                    p.S <= kFastS &&
+                    (p.S + kThreads / p.vdim - 1) / (kThreads / p.vdim) <= kFastVals;
   const size_t bytes = ((size_t)p.vdim + p.S + kThreads) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(combine_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);

@@ -42,8 +42,8 @@ constexpr int kLStages = 8;
 constexpr int kLRank = 32;               // key rank handled (one scale group)
 constexpr float kTwo24 = 16777216.f;     // code c held as the f16 bit pattern c is c * 2^-24
 
-// Stage layout of one tile: the components of the cache in their own order,
-// each the tile's 16 consecutive rows.
+// Stage layout of one tile: each component of the cache as the tile's 16
+// consecutive rows.
 template <int RV, bool RES>
 struct Stage {
   static constexpr int NVG = (RV + 31) / 32;          // value scale groups
@@ -53,12 +53,12 @@ struct Stage {
   static constexpr int LV = LKS + kLT * 4;
   static constexpr int LVS = LV + kLT * RV / 2;
   static constexpr int RKC = LVS + kLT * NVG * 4;
-  static constexpr int RKS = RKC + (RES ? kLT * 32 : 0);
-  static constexpr int RVC = RKS + (RES ? kLT * 2 : 0);
-  static constexpr int RVS = RVC + (RES ? kLT * 32 : 0);
+  static constexpr int RVC = RKC + (RES ? kLT * 32 : 0);
+  static constexpr int RKS = RVC + (RES ? kLT * 32 : 0);
+  static constexpr int RVS = RKS + (RES ? kLT * 2 : 0);
   static constexpr int BYTES = RVS + (RES ? kLT * 2 : 0);
-  static constexpr int CHUNKS = BYTES / 16;
-  static constexpr int CPL = (CHUNKS + 31) / 32;     // chunks per lane
+  static constexpr int CHUNKS = BYTES / 16;          // 16-byte copy chunks
+  static constexpr int CPL = (CHUNKS + 31) / 32;      // chunks per lane
   static constexpr int SMEM = kLWarps * kLStages * BYTES;
 };
 
@@ -66,9 +66,13 @@ struct LWork {
   int W, tpu, total;                     // tiles per warp, tiles per unit, all tiles
 };
 
-// smem row of token t in a component with 32-byte rows
-__device__ __forceinline__ int swz(int t) { return t ^ ((t >> 2) & 1); }
 
+// 16-byte cp.async to shared byte address dst + OFF
+template <int OFF>
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0+%2], [%1], 16;" ::"r"(dst), "l"(src), "n"(OFF)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -114,6 +118,7 @@ template <int RV, bool RES>
 __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork wk) {
   using L = Stage<RV, RES>;
   constexpr int NVG = L::NVG, VT = L::VT;
+  constexpr int RVB = RV / 2;                   // latent value row bytes
   constexpr bool kHalfGroup = (RV % 32) != 0;   // last value group holds 16 ranks
   extern __shared__ __align__(128) uint8_t lsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -121,34 +126,34 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
   const int t_first = gw * wk.W;
   const int n_tiles = min(wk.W, wk.total - t_first);
   if (n_tiles <= 0) return;
-  uint8_t* ring = lsm + warp * (kLStages * L::BYTES);
+  const uint32_t ring_s = smem_u32(lsm) + warp * (kLStages * L::BYTES);
+  const uint8_t* const ring = lsm + warp * (kLStages * L::BYTES);
   const int G = p.G, Hkv = p.Hkv;
   const int g = lane >> 2, c4 = lane & 3;
   const size_t rows_q = (size_t)p.B * p.Hq;
   const int pst = p.vdim + 2;
-  const int npp = p.tmax / kLT;          // tiles (pages) per batch row
+  const int npp = p.tmax / kLT;                 // tiles (pages) per batch row
 
-  // ---- this lane's copy chunks: source component, its row bytes, smem offset
+  // ---- chunk c = lane + 32 i (16 bytes) of every stage: source component,
+  // the chunk's offset inside the component's 16 rows, and its row bytes;
+  // each copy instruction of the warp moves 512 contiguous stage bytes
   const uint8_t* c_src[L::CPL];
-  int c_rowb[L::CPL], c_dst[L::CPL], c_tok[L::CPL];
+  int c_rowb[L::CPL];
 #pragma unroll
   for (int i = 0; i < L::CPL; ++i) {
-    const int c = lane + 32 * i, o = 16 * c;
-    const uint8_t* base;
-    int off, rowb;
+    const int o = 16 * (lane + 32 * i);
+    const uint8_t* base = nullptr;
+    int off = 0, rowb = 0;
     if (o < L::LKS) base = p.lk, off = L::LK, rowb = kLRank / 2;
     else if (o < L::LV) base = reinterpret_cast<const uint8_t*>(p.lksz), off = L::LKS, rowb = 4;
-    else if (o < L::LVS) base = p.lv, off = L::LV, rowb = RV / 2;
+    else if (o < L::LVS) base = p.lv, off = L::LV, rowb = RVB;
     else if (o < L::RKC) base = reinterpret_cast<const uint8_t*>(p.lvsz), off = L::LVS, rowb = NVG * 4;
-    else if (o < L::RKS) base = p.rkc, off = L::RKC, rowb = 32;
-    else if (o < L::RVC) base = reinterpret_cast<const uint8_t*>(p.rks), off = L::RKS, rowb = 2;
-    else if (o < L::RVS) base = p.rvc, off = L::RVC, rowb = 32;
-    else base = reinterpret_cast<const uint8_t*>(p.rvs), off = L::RVS, rowb = 2;
-    const int j = (o - off) / 16;                        // chunk within the component
-    c_src[i] = base + (size_t)16 * j;
+    else if (o < L::RVC) base = p.rkc, off = L::RKC, rowb = 32;
+    else if (o < L::RKS) base = p.rvc, off = L::RVC, rowb = 32;
+    else if (o < L::RVS) base = reinterpret_cast<const uint8_t*>(p.rks), off = L::RKS, rowb = 2;
+    else if (o < L::BYTES) base = reinterpret_cast<const uint8_t*>(p.rvs), off = L::RVS, rowb = 2;
+    c_src[i] = base ? base + (o - off) : nullptr;
     c_rowb[i] = rowb;
-    c_tok[i] = c < L::CHUNKS ? (16 * j) / rowb : kLT;    // first token of the chunk
-    c_dst[i] = off + (rowb == 32 ? 32 * swz(j >> 1) + 16 * (j & 1) : 16 * j);
   }
 
   // ---- first cache row of tile t of the range (page table or contiguous),
@@ -163,15 +168,22 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
   };
   int rows_cur = tile_row(lane), rows_next = tile_row(32 + lane);
 
-  auto issue = [&](int jj, int row0) {
-    const int t = t_first + jj;
-    const int jt = t % wk.tpu;
-    const int nt = min(kLT, p.n_tokens - jt * kLT);
-    uint8_t* st = ring + (jj % kLStages) * L::BYTES;
+  // whole 16-row blocks are copied, also on a unit's last, partial tile: the
+  // rows past its end exist (the capacity is a multiple of 16 and pages are
+  // whole), and their values are never used unmasked
+  auto issue = [&](int stage, int row0) {
+    const uint32_t dst = ring_s + stage * L::BYTES + 16 * lane;
 #pragma unroll
     for (int i = 0; i < L::CPL; ++i) {
-      if (lane + 32 * i < L::CHUNKS)
-        cp_async16(st + c_dst[i], c_src[i] + (size_t)row0 * c_rowb[i], c_tok[i] < nt ? 16 : 0);
+      if (lane + 32 * i < L::CHUNKS) {
+        const uint8_t* src = c_src[i] + (size_t)row0 * c_rowb[i];
+        switch (i) {
+          case 0: cp16<0>(dst, src); break;
+          case 1: cp16<512>(dst, src); break;
+          case 2: cp16<1024>(dst, src); break;
+          default: cp16<1536>(dst, src); break;
+        }
+      }
     }
   };
 
@@ -183,10 +195,13 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
     cp_async_commit();
   }
 
-  // ---- per-unit state
+  // the projected queries come from the kernel launched just before this one
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // ---- per-unit state (scores are kept in units of 2^-24 log2)
   uint32_t bq[2][2];                     // q~ (latent key) B fragments
   uint32_t br[RES ? 8 : 1][2];           // q^ (residual key) B fragments
-  float sumL[2], sumR[2];                // sum of the effective q~ / q^ of columns 2c4 + e
+  float sumL[2], kR[2];                  // 2^-24 sum q~ ; -1.5 * 2^-24 sum q^ (columns 2c4 + e)
   float m_ref[2], m_thr[2], l_sum[2];
   float accV[VT][4];
   float accR[RES ? 8 : 1][4];
@@ -232,8 +247,8 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
     own_r += __shfl_xor_sync(0xffffffffu, own_r, 2);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      sumL[e] = __shfl_sync(0xffffffffu, own_l, 4 * (2 * c4 + e));
-      sumR[e] = __shfl_sync(0xffffffffu, own_r, 4 * (2 * c4 + e));
+      sumL[e] = __shfl_sync(0xffffffffu, own_l, 4 * (2 * c4 + e)) * (1.f / kTwo24);
+      kR[e] = __shfl_sync(0xffffffffu, own_r, 4 * (2 * c4 + e)) * (-1.5f / kTwo24);
       m_ref[e] = m_thr[e] = -INFINITY;
       l_sum[e] = 0.f;
       sR[e] = 0.f;
@@ -286,21 +301,37 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         }
       }
       if (g == 0) {
-        dst[p.vdim] = m_ref[e];
+        dst[p.vdim] = m_ref[e] * kTwo24;
         dst[p.vdim + 1] = l2[e];
       }
     }
   };
 
-  // value-operand selectors: bytes (2h, 2h + 1) of two words side by side
+  // MMA row slot i holds token (i & 8) | ((i & 7) >> 1) | ((i & 1) << 2):
+  // score rows g, g + 8 read tokens tg, tg + 8, and the value operand's token
+  // slots 2c4, 2c4 + 1, 2c4 + 8, 2c4 + 9 read tokens c4, c4 + 4, c4 + 8,
+  // c4 + 12, so every shared-memory load is a per-thread base plus a constant
+  // and the value loads of a warp hit 32 distinct banks
+  const int tg = (g >> 1) | ((g & 1) << 2);
+  const int o_lk = L::LK + 16 * tg + 4 * c4;
+  const int o_lks = L::LKS + 4 * tg;
+  const int o_rk = L::RKC + 32 * tg + 8 * c4;
+  const int o_rks = L::RKS + 2 * tg;
+  const int o_lvs = L::LVS + NVG * 4 * tg;
+  const int o_rv = L::RVC + 32 * c4 + 4 * g;
+  const int o_rvs = L::RVS + 2 * tg;
+  // latent value words: full group v -> word 4v + g/2 (half g & 1), half group
+  // -> word 4v + g/4 (byte g & 3)
+  const int o_lv = L::LV + RVB * c4 + 4 * (g >> 1);
+  const int o_lvh = L::LV + RVB * c4 + 4 * (g >> 2);
   const uint32_t sel_v = (g & 1) ? 0x7632u : 0x5410u;
   const uint32_t bh = g & 3;
   const uint32_t sel_h = bh | (bh << 4) | ((4 + bh) << 8) | ((4 + bh) << 12);
-  const int tA0 = 2 * c4, tA1 = 2 * c4 + 1, tB0 = 2 * c4 + 8, tB1 = 2 * c4 + 9;
 
-  for (int jj = 0; jj < n_tiles; ++jj) {
-    const int t = t_first + jj;
-    const int u = t / wk.tpu, jt = t % wk.tpu;
+  int jt = t_first % wk.tpu, u = t_first / wk.tpu;
+  int s_iss = (kLStages - 1) % kLStages, s_use = 0;
+  for (int jj = 0; jj < n_tiles; ++jj, ++jt) {
+    if (jt == wk.tpu) jt = 0, ++u;
     const int nt = min(kLT, p.n_tokens - jt * kLT);
     if (u != cur_u) {
       if (cur_u >= 0) write_partial();
@@ -311,23 +342,23 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
     // keep kLStages - 1 tiles in flight; the cache rows come 32 tiles at a time
     {
       const int ji = jj + kLStages - 1;
-      if ((ji & 31) == 0 && ji > 0) {
+      if ((ji & 31) == 0) {
         rows_cur = rows_next;
         rows_next = tile_row(ji + 32 + lane);
       }
       const int r = __shfl_sync(0xffffffffu, rows_cur, ji & 31);
-      if (ji < n_tiles) issue(ji, r);
+      if (ji < n_tiles) issue(s_iss, r);
+      cp_async_commit();
+      s_iss = s_iss + 1 == kLStages ? 0 : s_iss + 1;
     }
-    cp_async_commit();
     cp_async_wait<kLStages - 1>();
     __syncwarp();
-    const uint8_t* st = ring + (jj % kLStages) * L::BYTES;
+    const uint8_t* st = ring + s_use * L::BYTES;
 
-    // ---------------- scores: rows g, g + 8 = tokens; columns 2c4, 2c4 + 1 = heads
+    // ---------------- scores: rows g, g + 8 = token slots; columns 2c4, 2c4 + 1 = heads
     float s[4];
     {
-      const uint32_t k0 = lds32(st + L::LK + 16 * g + 4 * c4);
-      const uint32_t k1 = lds32(st + L::LK + 16 * (g + 8) + 4 * c4);
+      const uint32_t k0 = lds32(st + o_lk), k1 = lds32(st + o_lk + 128);
       float aL[4] = {0.f, 0.f, 0.f, 0.f};
       {
         const uint32_t a[4] = {k0 & kN0, k1 & kN0, k0 & kN1, k1 & kN1};
@@ -336,19 +367,13 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         const uint32_t a2[4] = {y0 & kN0, y1 & kN0, y0 & kN1, y1 & kN1};
         mma16816(aL, a2, bq[1][0], bq[1][1]);
       }
-      const float2 sz0 = unpack_h2(lds32(st + L::LKS + 4 * g));
-      const float2 sz1 = unpack_h2(lds32(st + L::LKS + 4 * (g + 8)));
-      float c0[2], c1[2];                // per-token constant of each column
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        c0[e] = sz0.y * sumL[e];
-        c1[e] = sz1.y * sumL[e];
-      }
-      float aR0[4] = {0.f, 0.f, 0.f, 0.f}, aR1[4] = {0.f, 0.f, 0.f, 0.f};
-      float sr0 = 0.f, sr1 = 0.f;
+      const float2 sz0 = unpack_h2(lds32(st + o_lks));
+      const float2 sz1 = unpack_h2(lds32(st + o_lks + 32));
       if constexpr (RES) {
-        const uint2 r0 = *reinterpret_cast<const uint2*>(st + L::RKC + 32 * swz(g) + 8 * c4);
-        const uint2 r1 = *reinterpret_cast<const uint2*>(st + L::RKC + 32 * swz(g + 8) + 8 * c4);
+        // the -1.5 offset of the residual levels enters as the chain's start value
+        float aR0[4] = {kR[0], kR[1], kR[0], kR[1]}, aR1[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint2 r0 = *reinterpret_cast<const uint2*>(st + o_rk);
+        const uint2 r1 = *reinterpret_cast<const uint2*>(st + o_rk + 256);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint32_t w0 = h ? r0.y : r0.x, w1 = h ? r1.y : r1.x;
@@ -361,23 +386,21 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
             else mma16816(aR0, a, br[4 * h + k][0], br[4 * h + k][1]);
           }
         }
-        sr0 = __half2float(*reinterpret_cast<const __half*>(st + L::RKS + 2 * g));
-        sr1 = __half2float(*reinterpret_cast<const __half*>(st + L::RKS + 2 * (g + 8)));
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          c0[e] = fmaf(-1.5f * sr0, sumR[e], c0[e]);
-          c1[e] = fmaf(-1.5f * sr1, sumR[e], c1[e]);
-        }
+        const float sr0 = __half2float(*reinterpret_cast<const __half*>(st + o_rks));
+        const float sr1 = __half2float(*reinterpret_cast<const __half*>(st + o_rks + 16));
+        s[0] = fmaf(sz0.x, aL[0], fmaf(sr0, aR0[0] + aR1[0], sz0.y * sumL[0]));
+        s[1] = fmaf(sz0.x, aL[1], fmaf(sr0, aR0[1] + aR1[1], sz0.y * sumL[1]));
+        s[2] = fmaf(sz1.x, aL[2], fmaf(sr1, aR0[2] + aR1[2], sz1.y * sumL[0]));
+        s[3] = fmaf(sz1.x, aL[3], fmaf(sr1, aR0[3] + aR1[3], sz1.y * sumL[1]));
+      } else {
+        s[0] = fmaf(sz0.x, aL[0], sz0.y * sumL[0]);
+        s[1] = fmaf(sz0.x, aL[1], sz0.y * sumL[1]);
+        s[2] = fmaf(sz1.x, aL[2], sz1.y * sumL[0]);
+        s[3] = fmaf(sz1.x, aL[3], sz1.y * sumL[1]);
       }
-      const float k0s = sz0.x * kTwo24, k1s = sz1.x * kTwo24;
-      const float r0s = sr0 * kTwo24, r1s = sr1 * kTwo24;
-      s[0] = fmaf(k0s, aL[0], fmaf(r0s, aR0[0] + aR1[0], c0[0]));
-      s[1] = fmaf(k0s, aL[1], fmaf(r0s, aR0[1] + aR1[1], c0[1]));
-      s[2] = fmaf(k1s, aL[2], fmaf(r1s, aR0[2] + aR1[2], c1[0]));
-      s[3] = fmaf(k1s, aL[3], fmaf(r1s, aR0[3] + aR1[3], c1[1]));
       if (nt < kLT) {
-        if (g >= nt) s[0] = s[1] = -INFINITY;
-        if (g + 8 >= nt) s[2] = s[3] = -INFINITY;
+        if (tg >= nt) s[0] = s[1] = -INFINITY;
+        if (tg + 8 >= nt) s[2] = s[3] = -INFINITY;
       }
     }
 
@@ -391,7 +414,8 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
       const float n0 = fmaxf(m_ref[0], mx0), n1 = fmaxf(m_ref[1], mx1);
-      const float al[2] = {ex2_approx(m_ref[0] - n0), ex2_approx(m_ref[1] - n1)};
+      const float al[2] = {ex2_approx((m_ref[0] - n0) * kTwo24),
+                           ex2_approx((m_ref[1] - n1) * kTwo24)};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         l_sum[e] *= al[e];
@@ -407,29 +431,30 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
       }
       m_ref[0] = n0;
       m_ref[1] = n1;
-      m_thr[0] = n0 + 8.f;
-      m_thr[1] = n1 + 8.f;
+      m_thr[0] = n0 + 8.f / kTwo24;
+      m_thr[1] = n1 + 8.f / kTwo24;
     }
+    const float nm0 = -m_ref[0] * kTwo24, nm1 = -m_ref[1] * kTwo24;
     float pv[4];
-    pv[0] = ex2_approx(s[0] - m_ref[0]);
-    pv[1] = ex2_approx(s[1] - m_ref[1]);
-    pv[2] = ex2_approx(s[2] - m_ref[0]);
-    pv[3] = ex2_approx(s[3] - m_ref[1]);
+    pv[0] = ex2_approx(fmaf(s[0], kTwo24, nm0));
+    pv[1] = ex2_approx(fmaf(s[1], kTwo24, nm1));
+    pv[2] = ex2_approx(fmaf(s[2], kTwo24, nm0));
+    pv[3] = ex2_approx(fmaf(s[3], kTwo24, nm1));
     if (nt < kLT) {
-      if (g >= nt) pv[0] = pv[1] = 0.f;
-      if (g + 8 >= nt) pv[2] = pv[3] = 0.f;
+      if (tg >= nt) pv[0] = pv[1] = 0.f;
+      if (tg + 8 >= nt) pv[2] = pv[3] = 0.f;
     }
     l_sum[0] += pv[0] + pv[2];
     l_sum[1] += pv[1] + pv[3];
 
     // ---------------- values: acc^T (value row x head) += V^T (row x token) P'
     {
-      // scales and zeros of tokens g, g + 8 (zeroed past the end of the unit)
+      // scales and zeros of the tokens of rows g, g + 8 (zeroed past the end)
       float vs[NVG][2], vz[NVG][2];
 #pragma unroll
       for (int v = 0; v < NVG; ++v) {
-        const float2 a0 = unpack_h2(lds32(st + L::LVS + NVG * 4 * g + 4 * v));
-        const float2 a1 = unpack_h2(lds32(st + L::LVS + NVG * 4 * (g + 8) + 4 * v));
+        const float2 a0 = unpack_h2(lds32(st + o_lvs + 4 * v));
+        const float2 a1 = unpack_h2(lds32(st + o_lvs + NVG * 32 + 4 * v));
         vs[v][0] = a0.x;
         vz[v][0] = a0.y;
         vs[v][1] = a1.x;
@@ -438,11 +463,10 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
       if (nt < kLT) {
 #pragma unroll
         for (int v = 0; v < NVG; ++v) {
-          if (g >= nt) vs[v][0] = vz[v][0] = 0.f;
-          if (g + 8 >= nt) vs[v][1] = vz[v][1] = 0.f;
+          if (tg >= nt) vs[v][0] = vz[v][0] = 0.f;
+          if (tg + 8 >= nt) vs[v][1] = vz[v][1] = 0.f;
         }
       }
-      auto rowv = [&](int tok) -> int { return RV == 64 ? 32 * swz(tok) : (RV / 2) * tok; };
 #pragma unroll
       for (int v = 0; v < NVG; ++v) {
         zs[v][0] = fmaf(pv[0], vz[v][0], fmaf(pv[2], vz[v][1], zs[v][0]));
@@ -451,12 +475,10 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         const uint32_t h23 = pack_h2(pv[2] * vs[v][1], pv[3] * vs[v][1]);
         const uint32_t b0 = movmatrix_trans(h01), b1 = movmatrix_trans(h23);
         const bool half = kHalfGroup && v == NVG - 1;
-        const int word = half ? 4 * v + (g >> 2) : 4 * v + (g >> 1);
+        const uint8_t* lv = st + (half ? o_lvh : o_lv) + 16 * v;
         const uint32_t sel = half ? sel_h : sel_v;
-        const uint32_t xA = prmt(lds32(st + L::LV + rowv(tA0) + 4 * word),
-                                 lds32(st + L::LV + rowv(tA1) + 4 * word), sel);
-        const uint32_t xB = prmt(lds32(st + L::LV + rowv(tB0) + 4 * word),
-                                 lds32(st + L::LV + rowv(tB1) + 4 * word), sel);
+        const uint32_t xA = prmt(lds32(lv), lds32(lv + 4 * RVB), sel);
+        const uint32_t xB = prmt(lds32(lv + 8 * RVB), lds32(lv + 12 * RVB), sel);
         {
           const uint32_t a[4] = {xA & kN0, xA & kN1, xB & kN0, xB & kN1};
           mma16816(accV[2 * v], a, b0, b1);
@@ -468,21 +490,19 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         }
       }
       if constexpr (RES) {
-        float rs0 = __half2float(*reinterpret_cast<const __half*>(st + L::RVS + 2 * g));
-        float rs1 = __half2float(*reinterpret_cast<const __half*>(st + L::RVS + 2 * (g + 8)));
+        float rs0 = __half2float(*reinterpret_cast<const __half*>(st + o_rvs));
+        float rs1 = __half2float(*reinterpret_cast<const __half*>(st + o_rvs + 16));
         if (nt < kLT) {
-          if (g >= nt) rs0 = 0.f;
-          if (g + 8 >= nt) rs1 = 0.f;
+          if (tg >= nt) rs0 = 0.f;
+          if (tg + 8 >= nt) rs1 = 0.f;
         }
         const float q0 = pv[0] * rs0, q1 = pv[1] * rs0, q2 = pv[2] * rs1, q3 = pv[3] * rs1;
         sR[0] += q0 + q2;
         sR[1] += q1 + q3;
         const uint32_t b0 = movmatrix_trans(pack_h2(q0, q1));
         const uint32_t b1 = movmatrix_trans(pack_h2(q2, q3));
-        const uint32_t wA0 = lds32(st + L::RVC + 32 * swz(tA0) + 4 * g);
-        const uint32_t wA1 = lds32(st + L::RVC + 32 * swz(tA1) + 4 * g);
-        const uint32_t wB0 = lds32(st + L::RVC + 32 * swz(tB0) + 4 * g);
-        const uint32_t wB1 = lds32(st + L::RVC + 32 * swz(tB1) + 4 * g);
+        const uint32_t wA0 = lds32(st + o_rv), wA1 = lds32(st + o_rv + 128);
+        const uint32_t wB0 = lds32(st + o_rv + 256), wB1 = lds32(st + o_rv + 384);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const uint32_t sl = hh ? 0x7632u : 0x5410u;
@@ -498,6 +518,7 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
       }
     }
     __syncwarp();                        // this stage is refilled next iteration
+    if (++s_use == kLStages) s_use = 0;
   }
   cp_async_wait<0>();
   write_partial();
@@ -509,8 +530,19 @@ cudaError_t launch_t(const Params& p, const LWork& wk, int grid, cudaStream_t s)
   cudaError_t e = cudaFuncSetAttribute(latent_tc_kernel<RV, RES>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  latent_tc_kernel<RV, RES><<<grid, kLThreads, L::SMEM, s>>>(p, wk);
-  return cudaGetLastError();
+  // a programmatic dependent of the query projection: its prologue copies
+  // overlap the projection's tail
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kLThreads);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, latent_tc_kernel<RV, RES>, p, wk);
 }
 
 }  // namespace

@@ -58,6 +58,27 @@ __device__ __forceinline__ void fwht_smem(float* x, int n, int tid, int nthreads
   __syncthreads();
 }
 
+// Unnormalised Walsh-Hadamard transform (Sylvester order) of 128 values held
+// by one warp, lane l holding x[k] = v[4 l + k]: butterflies (a, b) ->
+// (a + b, a - b) over blocks of doubling size, the first two inside a lane and
+// the rest between lanes l and l ^ m (the lower index keeps a + b).
+__device__ __forceinline__ void fwht128_warp(float (&x)[4], int lane) {
+  float a = x[0] + x[1], b = x[0] - x[1], c = x[2] + x[3], e = x[2] - x[3];
+  x[0] = a + c;
+  x[1] = b + e;
+  x[2] = a - c;
+  x[3] = b - e;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool hi = lane & m;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[k], m);
+      x[k] = hi ? o - x[k] : x[k] + o;
+    }
+  }
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
