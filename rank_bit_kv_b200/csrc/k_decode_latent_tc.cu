@@ -27,6 +27,8 @@
 // pairwise, which makes the value-operand loads free of bank conflicts.
 #include <math.h>
 
+#include <type_traits>
+
 #include "kvc_device.cuh"
 #include "tc_util.cuh"
 
@@ -95,6 +97,9 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_h2(uint32_t x) {
   return __half22float2(*reinterpret_cast<const __half2*>(&x));
 }
+
+__device__ __forceinline__ __half2 u2h2(uint32_t x) { return *reinterpret_cast<__half2*>(&x); }
+__device__ __forceinline__ uint32_t h2u(__half2 x) { return *reinterpret_cast<uint32_t*>(&x); }
 
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) {
   return *reinterpret_cast<const uint32_t*>(p);
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
   uint32_t bq[2][2];                     // q~ (latent key) B fragments
   uint32_t br[RES ? 8 : 1][2];           // q^ (residual key) B fragments
   float sumL[2], kR[2];                  // 2^-24 sum q~ ; -1.5 * 2^-24 sum q^ (columns 2c4 + e)
-  float m_ref[2], m_thr[2], l_sum[2];
+  float m_ref[2], m_thr[2], l_sum[2], nm[2];   // nm = -m_ref * 2^24
   float accV[VT][4];
   float accR[RES ? 8 : 1][4];
   float zs[NVG][2];                      // sum_t p_t zero_t per value group
@@ -250,6 +255,7 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
       sumL[e] = __shfl_sync(0xffffffffu, own_l, 4 * (2 * c4 + e)) * (1.f / kTwo24);
       kR[e] = __shfl_sync(0xffffffffu, own_r, 4 * (2 * c4 + e)) * (-1.5f / kTwo24);
       m_ref[e] = m_thr[e] = -INFINITY;
+      nm[e] = INFINITY;
       l_sum[e] = 0.f;
       sR[e] = 0.f;
 #pragma unroll
@@ -328,32 +334,13 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
   const uint32_t bh = g & 3;
   const uint32_t sel_h = bh | (bh << 4) | ((4 + bh) << 8) | ((4 + bh) << 12);
 
-  int jt = t_first % wk.tpu, u = t_first / wk.tpu;
-  int s_iss = (kLStages - 1) % kLStages, s_use = 0;
-  for (int jj = 0; jj < n_tiles; ++jj, ++jt) {
-    if (jt == wk.tpu) jt = 0, ++u;
-    const int nt = min(kLT, p.n_tokens - jt * kLT);
-    if (u != cur_u) {
-      if (cur_u >= 0) write_partial();
-      cur_u = u;
-      cur_slot = gw - (int)(((long long)u * wk.tpu) / wk.W);
-      reset(u);
-    }
-    // keep kLStages - 1 tiles in flight; the cache rows come 32 tiles at a time
-    {
-      const int ji = jj + kLStages - 1;
-      if ((ji & 31) == 0) {
-        rows_cur = rows_next;
-        rows_next = tile_row(ji + 32 + lane);
-      }
-      const int r = __shfl_sync(0xffffffffu, rows_cur, ji & 31);
-      if (ji < n_tiles) issue(s_iss, r);
-      cp_async_commit();
-      s_iss = s_iss + 1 == kLStages ? 0 : s_iss + 1;
-    }
-    cp_async_wait<kLStages - 1>();
-    __syncwarp();
+  // ---- one tile of the current unit from stage s_use; TAIL: the unit's last
+  // tile holds nt < 16 tokens (rows past nt are masked out)
+  int s_use = 0;
+  auto tile = [&](auto tail_tag, int nt) {
+    constexpr bool TAIL = decltype(tail_tag)::value;
     const uint8_t* st = ring + s_use * L::BYTES;
+    const bool ok0 = !TAIL || tg < nt, ok1 = !TAIL || tg + 8 < nt;
 
     // ---------------- scores: rows g, g + 8 = token slots; columns 2c4, 2c4 + 1 = heads
     float s[4];
@@ -398,9 +385,9 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         s[2] = fmaf(sz1.x, aL[2], sz1.y * sumL[0]);
         s[3] = fmaf(sz1.x, aL[3], sz1.y * sumL[1]);
       }
-      if (nt < kLT) {
-        if (tg >= nt) s[0] = s[1] = -INFINITY;
-        if (tg + 8 >= nt) s[2] = s[3] = -INFINITY;
+      if constexpr (TAIL) {
+        if (!ok0) s[0] = s[1] = -INFINITY;
+        if (!ok1) s[2] = s[3] = -INFINITY;
       }
     }
 
@@ -433,95 +420,128 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
       m_ref[1] = n1;
       m_thr[0] = n0 + 8.f / kTwo24;
       m_thr[1] = n1 + 8.f / kTwo24;
+      nm[0] = -n0 * kTwo24;
+      nm[1] = -n1 * kTwo24;
     }
-    const float nm0 = -m_ref[0] * kTwo24, nm1 = -m_ref[1] * kTwo24;
     float pv[4];
-    pv[0] = ex2_approx(fmaf(s[0], kTwo24, nm0));
-    pv[1] = ex2_approx(fmaf(s[1], kTwo24, nm1));
-    pv[2] = ex2_approx(fmaf(s[2], kTwo24, nm0));
-    pv[3] = ex2_approx(fmaf(s[3], kTwo24, nm1));
-    if (nt < kLT) {
-      if (tg >= nt) pv[0] = pv[1] = 0.f;
-      if (tg + 8 >= nt) pv[2] = pv[3] = 0.f;
+    pv[0] = ex2_approx(fmaf(s[0], kTwo24, nm[0]));
+    pv[1] = ex2_approx(fmaf(s[1], kTwo24, nm[1]));
+    pv[2] = ex2_approx(fmaf(s[2], kTwo24, nm[0]));
+    pv[3] = ex2_approx(fmaf(s[3], kTwo24, nm[1]));
+    if constexpr (TAIL) {
+      if (!ok0) pv[0] = pv[1] = 0.f;
+      if (!ok1) pv[2] = pv[3] = 0.f;
     }
     l_sum[0] += pv[0] + pv[2];
     l_sum[1] += pv[1] + pv[3];
+    // probabilities of the rows' tokens, packed per row: (head 2c4, head 2c4 + 1)
+    const __half2 hp01 = __floats2half2_rn(pv[0], pv[1]);
+    const __half2 hp23 = __floats2half2_rn(pv[2], pv[3]);
 
     // ---------------- values: acc^T (value row x head) += V^T (row x token) P'
-    {
-      // scales and zeros of the tokens of rows g, g + 8 (zeroed past the end)
-      float vs[NVG][2], vz[NVG][2];
+    // P' = p * scale and the zero term p * zero are formed in f16x2 per tile
+    // (scale and zero are fp16 already); the zero terms are summed in fp32
 #pragma unroll
-      for (int v = 0; v < NVG; ++v) {
-        const float2 a0 = unpack_h2(lds32(st + o_lvs + 4 * v));
-        const float2 a1 = unpack_h2(lds32(st + o_lvs + NVG * 32 + 4 * v));
-        vs[v][0] = a0.x;
-        vz[v][0] = a0.y;
-        vs[v][1] = a1.x;
-        vz[v][1] = a1.y;
+    for (int v = 0; v < NVG; ++v) {
+      __half2 sz_0 = u2h2(lds32(st + o_lvs + 4 * v));
+      __half2 sz_1 = u2h2(lds32(st + o_lvs + NVG * 32 + 4 * v));
+      if constexpr (TAIL) {          // rows past the end may hold any bits
+        if (!ok0) sz_0 = __float2half2_rn(0.f);
+        if (!ok1) sz_1 = __float2half2_rn(0.f);
       }
-      if (nt < kLT) {
-#pragma unroll
-        for (int v = 0; v < NVG; ++v) {
-          if (tg >= nt) vs[v][0] = vz[v][0] = 0.f;
-          if (tg + 8 >= nt) vs[v][1] = vz[v][1] = 0.f;
-        }
+      const __half2 zt = __hfma2(hp23, __high2half2(sz_1), __hmul2(hp01, __high2half2(sz_0)));
+      const float2 ztf = __half22float2(zt);
+      zs[v][0] += ztf.x;
+      zs[v][1] += ztf.y;
+      const uint32_t b0 = movmatrix_trans(h2u(__hmul2(hp01, __low2half2(sz_0))));
+      const uint32_t b1 = movmatrix_trans(h2u(__hmul2(hp23, __low2half2(sz_1))));
+      const bool half = kHalfGroup && v == NVG - 1;
+      const uint8_t* lv = st + (half ? o_lvh : o_lv) + 16 * v;
+      const uint32_t sel = half ? sel_h : sel_v;
+      const uint32_t xA = prmt(lds32(lv), lds32(lv + 4 * RVB), sel);
+      const uint32_t xB = prmt(lds32(lv + 8 * RVB), lds32(lv + 12 * RVB), sel);
+      {
+        const uint32_t a[4] = {xA & kN0, xA & kN1, xB & kN0, xB & kN1};
+        mma16816(accV[2 * v], a, b0, b1);
       }
-#pragma unroll
-      for (int v = 0; v < NVG; ++v) {
-        zs[v][0] = fmaf(pv[0], vz[v][0], fmaf(pv[2], vz[v][1], zs[v][0]));
-        zs[v][1] = fmaf(pv[1], vz[v][0], fmaf(pv[3], vz[v][1], zs[v][1]));
-        const uint32_t h01 = pack_h2(pv[0] * vs[v][0], pv[1] * vs[v][0]);
-        const uint32_t h23 = pack_h2(pv[2] * vs[v][1], pv[3] * vs[v][1]);
-        const uint32_t b0 = movmatrix_trans(h01), b1 = movmatrix_trans(h23);
-        const bool half = kHalfGroup && v == NVG - 1;
-        const uint8_t* lv = st + (half ? o_lvh : o_lv) + 16 * v;
-        const uint32_t sel = half ? sel_h : sel_v;
-        const uint32_t xA = prmt(lds32(lv), lds32(lv + 4 * RVB), sel);
-        const uint32_t xB = prmt(lds32(lv + 8 * RVB), lds32(lv + 12 * RVB), sel);
-        {
-          const uint32_t a[4] = {xA & kN0, xA & kN1, xB & kN0, xB & kN1};
-          mma16816(accV[2 * v], a, b0, b1);
-        }
-        if (!half) {
-          const uint32_t yA = xA >> 8, yB = xB >> 8;
-          const uint32_t a[4] = {yA & kN0, yA & kN1, yB & kN0, yB & kN1};
-          mma16816(accV[2 * v + 1], a, b0, b1);
-        }
+      if (!half) {
+        const uint32_t yA = xA >> 8, yB = xB >> 8;
+        const uint32_t a[4] = {yA & kN0, yA & kN1, yB & kN0, yB & kN1};
+        mma16816(accV[2 * v + 1], a, b0, b1);
       }
-      if constexpr (RES) {
-        float rs0 = __half2float(*reinterpret_cast<const __half*>(st + o_rvs));
-        float rs1 = __half2float(*reinterpret_cast<const __half*>(st + o_rvs + 16));
-        if (nt < kLT) {
-          if (tg >= nt) rs0 = 0.f;
-          if (tg + 8 >= nt) rs1 = 0.f;
-        }
-        const float q0 = pv[0] * rs0, q1 = pv[1] * rs0, q2 = pv[2] * rs1, q3 = pv[3] * rs1;
-        sR[0] += q0 + q2;
-        sR[1] += q1 + q3;
-        const uint32_t b0 = movmatrix_trans(pack_h2(q0, q1));
-        const uint32_t b1 = movmatrix_trans(pack_h2(q2, q3));
-        const uint32_t wA0 = lds32(st + o_rv), wA1 = lds32(st + o_rv + 128);
-        const uint32_t wB0 = lds32(st + o_rv + 256), wB1 = lds32(st + o_rv + 384);
+    }
+    if constexpr (RES) {
+      __half2 rs_0 = __half2half2(*reinterpret_cast<const __half*>(st + o_rvs));
+      __half2 rs_1 = __half2half2(*reinterpret_cast<const __half*>(st + o_rvs + 16));
+      if constexpr (TAIL) {
+        if (!ok0) rs_0 = __float2half2_rn(0.f);
+        if (!ok1) rs_1 = __float2half2_rn(0.f);
+      }
+      const __half2 q01 = __hmul2(hp01, rs_0), q23 = __hmul2(hp23, rs_1);
+      const float2 qs = __half22float2(__hadd2(q01, q23));
+      sR[0] += qs.x;
+      sR[1] += qs.y;
+      const uint32_t b0 = movmatrix_trans(h2u(q01));
+      const uint32_t b1 = movmatrix_trans(h2u(q23));
+      const uint32_t wA0 = lds32(st + o_rv), wA1 = lds32(st + o_rv + 128);
+      const uint32_t wB0 = lds32(st + o_rv + 256), wB1 = lds32(st + o_rv + 384);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t sl = hh ? 0x7632u : 0x5410u;
-          const uint32_t xA = prmt(wA0, wA1, sl), xB = prmt(wB0, wB1, sl);
-          const uint32_t xA6 = xA >> 6, xB6 = xB >> 6;
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t sl = hh ? 0x7632u : 0x5410u;
+        const uint32_t xA = prmt(wA0, wA1, sl), xB = prmt(wB0, wB1, sl);
+        const uint32_t xA6 = xA >> 6, xB6 = xB >> 6;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t a[4] = {field2(xA, xA6, 2 * k), field2(xA, xA6, 2 * k + 1),
-                                   field2(xB, xB6, 2 * k), field2(xB, xB6, 2 * k + 1)};
-            mma16816(accR[4 * hh + k], a, b0, b1);
-          }
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t a[4] = {field2(xA, xA6, 2 * k), field2(xA, xA6, 2 * k + 1),
+                                 field2(xB, xB6, 2 * k), field2(xB, xB6, 2 * k + 1)};
+          mma16816(accR[4 * hh + k], a, b0, b1);
         }
       }
     }
-    __syncwarp();                        // this stage is refilled next iteration
+    __syncwarp();                        // this stage is refilled by the next step
     if (++s_use == kLStages) s_use = 0;
+  };
+
+  // ---- next copy: keep kLStages - 1 tiles in flight, then wait for the oldest;
+  // the cache rows come 32 tiles at a time
+  int ji = kLStages - 1, s_iss = (kLStages - 1) % kLStages;
+  auto step = [&]() {
+    if ((ji & 31) == 0) {
+      rows_cur = rows_next;
+      rows_next = tile_row(ji + 32 + lane);
+    }
+    const int r = __shfl_sync(0xffffffffu, rows_cur, ji & 31);
+    if (ji < n_tiles) issue(s_iss, r);
+    cp_async_commit();
+    ++ji;
+    s_iss = s_iss + 1 == kLStages ? 0 : s_iss + 1;
+    cp_async_wait<kLStages - 1>();
+    __syncwarp();
+  };
+
+  // ---- the units of this warp's range, one partial each
+  const int tail_nt = p.n_tokens % kLT;          // tokens of a unit's last tile, 0 = whole
+  int u = t_first / wk.tpu, jt0 = t_first % wk.tpu;
+  for (int jj = 0; jj < n_tiles;) {
+    const int cnt = min(wk.tpu - jt0, n_tiles - jj);
+    const bool tail = tail_nt != 0 && jt0 + cnt == wk.tpu;
+    cur_u = u;
+    cur_slot = gw - (int)(((long long)u * wk.tpu) / wk.W);
+    reset(u);
+    for (int k = tail ? 1 : 0; k < cnt; ++k) {
+      step();
+      tile(std::false_type(), kLT);
+    }
+    if (tail) {
+      step();
+      tile(std::true_type(), tail_nt);
+    }
+    write_partial();
+    jj += cnt;
+    ++u;
+    jt0 = 0;
   }
   cp_async_wait<0>();
-  write_partial();
 }
 
 template <int RV, bool RES>
