@@ -41,27 +41,31 @@ constexpr int kLT = 16;                  // tokens per tile (one page)
 constexpr int kLWarps = 12;
 constexpr int kLThreads = 32 * kLWarps;
 constexpr int kLStages = 8;
+constexpr int kDist = kLStages - 2;      // tiles in flight ahead of the one computed
 constexpr int kLRank = 32;               // key rank handled (one scale group)
 constexpr float kTwo24 = 16777216.f;     // code c held as the f16 bit pattern c is c * 2^-24
 
 // Stage layout of one tile: each component of the cache as the tile's 16
-// consecutive rows.
+// consecutive rows; the small ones first, then (residual layouts) the residual
+// key codes at byte 512, so that one copy instruction of the warp moves them
+// and places their rows in MMA-slot order, then the value codes.
 template <int RV, bool RES>
 struct Stage {
   static constexpr int NVG = (RV + 31) / 32;          // value scale groups
   static constexpr int VT = RV / 16;                  // latent value M-tiles
   static constexpr int LK = 0;
   static constexpr int LKS = LK + kLT * kLRank / 2;
-  static constexpr int LV = LKS + kLT * 4;
-  static constexpr int LVS = LV + kLT * RV / 2;
-  static constexpr int RKC = LVS + kLT * NVG * 4;
-  static constexpr int RVC = RKC + (RES ? kLT * 32 : 0);
-  static constexpr int RKS = RVC + (RES ? kLT * 32 : 0);
+  static constexpr int LVS = LKS + kLT * 4;
+  static constexpr int RKS = LVS + kLT * NVG * 4;
   static constexpr int RVS = RKS + (RES ? kLT * 2 : 0);
-  static constexpr int BYTES = RVS + (RES ? kLT * 2 : 0);
+  static constexpr int RKC = RES ? 512 : RVS;
+  static constexpr int LV = RKC + (RES ? kLT * 32 : 0);
+  static constexpr int RVC = LV + kLT * RV / 2;
+  static constexpr int BYTES = RVC + (RES ? kLT * 32 : 0);
   static constexpr int CHUNKS = BYTES / 16;          // 16-byte copy chunks
   static constexpr int CPL = (CHUNKS + 31) / 32;      // chunks per lane
   static constexpr int SMEM = kLWarps * kLStages * BYTES;
+  static_assert(!RES || RVS + kLT * 2 <= 512, "residual keys must start at byte 512");
 };
 
 struct LWork {
@@ -150,13 +154,14 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
     const uint8_t* base = nullptr;
     int off = 0, rowb = 0;
     if (o < L::LKS) base = p.lk, off = L::LK, rowb = kLRank / 2;
-    else if (o < L::LV) base = reinterpret_cast<const uint8_t*>(p.lksz), off = L::LKS, rowb = 4;
-    else if (o < L::LVS) base = p.lv, off = L::LV, rowb = RVB;
-    else if (o < L::RKC) base = reinterpret_cast<const uint8_t*>(p.lvsz), off = L::LVS, rowb = NVG * 4;
-    else if (o < L::RVC) base = p.rkc, off = L::RKC, rowb = 32;
-    else if (o < L::RKS) base = p.rvc, off = L::RVC, rowb = 32;
-    else if (o < L::RVS) base = reinterpret_cast<const uint8_t*>(p.rks), off = L::RKS, rowb = 2;
-    else if (o < L::BYTES) base = reinterpret_cast<const uint8_t*>(p.rvs), off = L::RVS, rowb = 2;
+    else if (o < L::LVS) base = reinterpret_cast<const uint8_t*>(p.lksz), off = L::LKS, rowb = 4;
+    else if (o < L::RKS) base = reinterpret_cast<const uint8_t*>(p.lvsz), off = L::LVS, rowb = NVG * 4;
+    else if (RES && o < L::RVS) base = reinterpret_cast<const uint8_t*>(p.rks), off = L::RKS, rowb = 2;
+    else if (RES && o < L::RVS + kLT * 2) base = reinterpret_cast<const uint8_t*>(p.rvs), off = L::RVS, rowb = 2;
+    else if (o < L::RKC) base = nullptr;               // padding before the residual keys
+    else if (o < L::LV) base = p.rkc, off = L::RKC, rowb = 32;
+    else if (o < L::RVC) base = p.lv, off = L::LV, rowb = RVB;
+    else if (o < L::BYTES) base = p.rvc, off = L::RVC, rowb = 32;
     c_src[i] = base ? base + (o - off) : nullptr;
     c_rowb[i] = rowb;
   }
@@ -176,15 +181,23 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
   // whole 16-row blocks are copied, also on a unit's last, partial tile: the
   // rows past its end exist (the capacity is a multiple of 16 and pages are
   // whole), and their values are never used unmasked
+  // residual key rows are stored in MMA-slot order: chunk j (token j / 2,
+  // half j % 2) of that component goes to slot (token) ^-1 -- see tg below
+  const int rk_tok = lane >> 1;
+  const int rk_dst = L::RKC + 32 * ((rk_tok & 8) | ((rk_tok & 3) << 1) | ((rk_tok >> 2) & 1)) +
+                     16 * (lane & 1);
   auto issue = [&](int stage, int row0) {
     const uint32_t dst = ring_s + stage * L::BYTES + 16 * lane;
 #pragma unroll
     for (int i = 0; i < L::CPL; ++i) {
-      if (lane + 32 * i < L::CHUNKS) {
+      if (lane + 32 * i < L::CHUNKS && (16 * (lane + 32 * i) >= L::RKC || 16 * (lane + 32 * i) < L::RVS + (RES ? kLT * 2 : 0))) {
         const uint8_t* src = c_src[i] + (size_t)row0 * c_rowb[i];
         switch (i) {
           case 0: cp16<0>(dst, src); break;
-          case 1: cp16<512>(dst, src); break;
+          case 1:
+            if (RES) cp16<0>(ring_s + stage * L::BYTES + rk_dst, src);
+            else cp16<512>(dst, src);
+            break;
           case 2: cp16<1024>(dst, src); break;
           default: cp16<1536>(dst, src); break;
         }
@@ -192,9 +205,9 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
     }
   };
 
-  // prologue: kLStages - 1 tiles in flight
+  // prologue: kDist tiles in flight
 #pragma unroll
-  for (int i = 0; i < kLStages - 1; ++i) {
+  for (int i = 0; i < kDist; ++i) {
     const int r = __shfl_sync(0xffffffffu, rows_cur, i);
     if (i < n_tiles) issue(i, r);
     cp_async_commit();
@@ -321,7 +334,7 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
   const int tg = (g >> 1) | ((g & 1) << 2);
   const int o_lk = L::LK + 16 * tg + 4 * c4;
   const int o_lks = L::LKS + 4 * tg;
-  const int o_rk = L::RKC + 32 * tg + 8 * c4;
+  const int o_rk = L::RKC + 32 * g + 8 * c4;     // rows stored in slot order
   const int o_rks = L::RKS + 2 * tg;
   const int o_lvs = L::LVS + NVG * 4 * tg;
   const int o_rv = L::RVC + 32 * c4 + 4 * g;
@@ -336,14 +349,10 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
 
   // ---- one tile of the current unit from stage s_use; TAIL: the unit's last
   // tile holds nt < 16 tokens (rows past nt are masked out)
-  int s_use = 0;
-  auto tile = [&](auto tail_tag, int nt) {
+  auto scores = [&](auto tail_tag, const uint8_t* st, int nt, float (&s)[4]) {
     constexpr bool TAIL = decltype(tail_tag)::value;
-    const uint8_t* st = ring + s_use * L::BYTES;
     const bool ok0 = !TAIL || tg < nt, ok1 = !TAIL || tg + 8 < nt;
-
-    // ---------------- scores: rows g, g + 8 = token slots; columns 2c4, 2c4 + 1 = heads
-    float s[4];
+    // rows g, g + 8 = token slots; columns 2c4, 2c4 + 1 = heads
     {
       const uint32_t k0 = lds32(st + o_lk), k1 = lds32(st + o_lk + 128);
       float aL[4] = {0.f, 0.f, 0.f, 0.f};
@@ -391,6 +400,11 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
       }
     }
 
+  };
+
+  auto values = [&](auto tail_tag, const uint8_t* st, int nt, const float (&s)[4]) {
+    constexpr bool TAIL = decltype(tail_tag)::value;
+    const bool ok0 = !TAIL || tg < nt, ok1 = !TAIL || tg + 8 < nt;
     // ---------------- online softmax (lazy maximum, raised by more than 2^8)
     const bool need = s[0] > m_thr[0] || s[2] > m_thr[0] || s[1] > m_thr[1] || s[3] > m_thr[1];
     if (__any_sync(0xffffffffu, need)) {
@@ -498,14 +512,14 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         }
       }
     }
-    __syncwarp();                        // this stage is refilled by the next step
-    if (++s_use == kLStages) s_use = 0;
   };
 
-  // ---- next copy: keep kLStages - 1 tiles in flight, then wait for the oldest;
-  // the cache rows come 32 tiles at a time
-  int ji = kLStages - 1, s_iss = (kLStages - 1) % kLStages;
-  auto step = [&]() {
+  // ---- next copy: keep kDist tiles in flight, then wait for the oldest; the
+  // stage of the tile before the oldest is refilled (the oldest's values are
+  // still to be computed); the cache rows come 32 tiles at a time
+  int ji = kDist, s_iss = kDist, s_use = 0;
+  auto step = [&]() -> const uint8_t* {
+    __syncwarp();                        // every lane is done with the stage refilled now
     if ((ji & 31) == 0) {
       rows_cur = rows_next;
       rows_next = tile_row(ji + 32 + lane);
@@ -515,8 +529,11 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
     cp_async_commit();
     ++ji;
     s_iss = s_iss + 1 == kLStages ? 0 : s_iss + 1;
-    cp_async_wait<kLStages - 1>();
+    cp_async_wait<kDist>();
     __syncwarp();
+    const uint8_t* st = ring + s_use * L::BYTES;
+    s_use = s_use + 1 == kLStages ? 0 : s_use + 1;
+    return st;
   };
 
   // ---- the units of this warp's range, one partial each
@@ -528,14 +545,31 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
     cur_u = u;
     cur_slot = gw - (int)(((long long)u * wk.tpu) / wk.W);
     reset(u);
-    for (int k = tail ? 1 : 0; k < cnt; ++k) {
-      step();
-      tile(std::false_type(), kLT);
+    // software pipeline: the scores of tile k + 1 are formed before the
+    // softmax and value update of tile k
+    float s_cur[4], s_nxt[4];
+    const uint8_t* st_cur = step();
+    if (tail && cnt == 1) scores(std::true_type(), st_cur, tail_nt, s_cur);
+    else scores(std::false_type(), st_cur, kLT, s_cur);
+    for (int k = 0; k + 2 < cnt; ++k) {
+      const uint8_t* st_nxt = step();
+      scores(std::false_type(), st_nxt, kLT, s_nxt);
+      values(std::false_type(), st_cur, kLT, s_cur);
+      st_cur = st_nxt;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s_cur[i] = s_nxt[i];
     }
-    if (tail) {
-      step();
-      tile(std::true_type(), tail_nt);
+    if (cnt >= 2) {
+      const uint8_t* st_nxt = step();
+      if (tail) scores(std::true_type(), st_nxt, tail_nt, s_nxt);
+      else scores(std::false_type(), st_nxt, kLT, s_nxt);
+      values(std::false_type(), st_cur, kLT, s_cur);
+      st_cur = st_nxt;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s_cur[i] = s_nxt[i];
     }
+    if (tail) values(std::true_type(), st_cur, tail_nt, s_cur);
+    else values(std::false_type(), st_cur, kLT, s_cur);
     write_partial();
     jj += cnt;
     ++u;
