@@ -1,0 +1,87 @@
+"""Run (and time) the decode step of a named synthetic workload.
+
+    python -m rank_bit_kv_b200.step c5 [--batch B] [--steps N] [--time]
+
+Builds the seeded synthetic cache of the workload (optionally with a smaller
+batch), then calls kvc_decode_attn N times on the current CUDA device.  With
+--time it flushes L2 (a 512 MiB write) before every call and prints, per call
+median, the whole step (query projection, split-T kernel, combine) and the
+split-T kernel alone, both from CUDA events, with the compressed bytes the step
+reads.  Without --time it only runs the calls (the form used under a profiler).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import statistics
+
+
+def _cache(kvc, synth, c):
+    lay = kvc.Layout(kvc.desc_from_config(c))
+    if c["kind"] == "varrate":
+        fill = synth.varrate_cache(c)
+    elif c["kind"] == "block_shared":
+        fill = synth.block_shared_cache(c)
+    else:
+        fill = synth.lowrank_cache(c)
+    cache = kvc.Cache(lay, fill=fill)
+    cache.n_tokens = c["T"]
+    return lay, cache, fill
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("config", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--time", action="store_true")
+    args = ap.parse_args(argv)
+
+    import numpy as np
+    import torch
+
+    from rank_bit_kv_b200 import kvc, synth
+
+    over = {} if args.batch is None else {"B": args.batch}
+    c = synth.config(args.config, **over)
+    lay, cache, fill = _cache(kvc, synth, c)
+    q = torch.from_numpy(np.ascontiguousarray(fill["q"]).view(np.int16)).cuda().view(torch.bfloat16)
+    out = torch.empty(q.shape, device="cuda")
+    ws = torch.zeros(lay.workspace_bytes(c["T"]), dtype=torch.uint8, device="cuda")
+    if not args.time:
+        for _ in range(args.steps):
+            kvc.decode(lay, cache, q, out, ws)
+        torch.cuda.synchronize()
+        print(json.dumps({"config": args.config, "batch": c["B"], "steps": args.steps,
+                          "finite": bool(torch.isfinite(out).all().item()),
+                          "err_word": int(ws[:4].view(torch.int32).item())}))
+        return
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        kvc.decode(lay, cache, q, out, ws)
+    torch.cuda.synchronize()
+    step_us, kern_us = [], []
+    for _ in range(args.steps):
+        flush.zero_()
+        ev = (kvc.RawEvent(), kvc.RawEvent())
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kvc.decode(lay, cache, q, out, ws, events=ev)
+        e1.record()
+        torch.cuda.synchronize()
+        step_us.append(e0.elapsed_time(e1) * 1e3)
+        kern_us.append(ev[0].elapsed_ms(ev[1]) * 1e3)
+    nbytes = lay.step_bytes(c["T"])
+    st, kt = statistics.median(step_us), statistics.median(kern_us)
+    print(json.dumps({"config": args.config, "batch": c["B"], "context": c["T"],
+                      "bytes_per_step": nbytes, "step_us": round(st, 2),
+                      "split_kernel_us": round(kt, 2), "step_gbs": round(nbytes / st / 1e3, 1),
+                      "split_kernel_gbs": round(nbytes / kt / 1e3, 1),
+                      "finite": bool(torch.isfinite(out).all().item()),
+                      "err_word": int(ws[:4].view(torch.int32).item()),
+                      "kernel_version": kvc.lib().kvc_version().decode()}))
+
+
+if __name__ == "__main__":
+    main()
