@@ -357,10 +357,13 @@ __global__ void __launch_bounds__(kThreads) split_generic_kernel(Params p) {
 }  // namespace
 
 cudaError_t launch_split(const Params& p, cudaStream_t s) {
-  if (p.seg_W > 0)
-    return p.kind == KVC_DENSE_BF16 ? launch_dense_tc(p, s)
-           : p.rope                 ? launch_rope_tc(p, p.err, s)
-                                    : launch_latent_tc(p, s);
+  switch (p.path) {
+    case 1: return launch_rope_tc(p, p.err, s);
+    case 2: return launch_dense_tc(p, s);
+    case 3: return launch_latent_tc(p, s);
+    case 4: return launch_rope_mma(p, s);
+    default: break;
+  }
   const Geo g = geometry(p);
   const Smem S = carve(p, g);
   const size_t bytes = (size_t)S.total * sizeof(float);

@@ -86,6 +86,8 @@ size_t ws_bytes(const kvc_layout* L, int n_tokens) {
   if (L->d.kind == KVC_LOWRANK) {
     const int Sl = kvc::latent_tc_slots(L->d.batch, L->d.n_kv_heads, nt1);
     if (Sl > S) S = Sl;
+    const int Sr = kvc::rope_mma_slots(L->d.batch, L->d.n_kv_heads, nt1);
+    if (Sr > S) S = Sr;
   }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   size_t b = kWsHeader + round_up(rows * L->qdim * sizeof(float), 256);
@@ -447,27 +449,30 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
   p.out = out;
   p.out_bf16 = L->d.out_bf16;
   plan(L, c->n_tokens, &p.S, &p.split_len);
-  if (kvc::rope_tc_supported(p)) {
-    int grid, W, tpu, slots;
-    kvc::rope_tc_plan(p, &grid, &W, &tpu, &slots);
-    p.S = slots;
-    p.seg_W = W;
-    p.seg_tpu = tpu;
-    p.seg_parts = kvc::kRopeTcParts;
-  } else if (kvc::latent_tc_supported(p)) {
-    int grid, W, tpu, slots;
-    kvc::latent_tc_plan(p, &grid, &W, &tpu, &slots);
-    p.S = slots;
-    p.seg_W = W;
-    p.seg_tpu = tpu;
-    p.seg_parts = 1;
-  } else if (kvc::dense_tc_supported(p)) {
-    int grid, W, tpu, slots;
-    kvc::dense_tc_plan(p, &grid, &W, &tpu, &slots);
-    p.S = slots;
-    p.seg_W = W;
-    p.seg_tpu = tpu;
-    p.seg_parts = 1;
+  {
+    // the warp- / CTA-level tensor-core kernels run equal contiguous tile
+    // ranges (seg_W tiles of the flattened (unit, tile) space per warp or CTA)
+    int grid = 0, W = 0, tpu = 0, slots = 0, parts = 1;
+    if (kvc::rope_mma_supported(p)) {
+      kvc::rope_mma_plan(p, &grid, &W, &tpu, &slots);
+      p.path = 4;
+    } else if (kvc::rope_tc_supported(p)) {
+      kvc::rope_tc_plan(p, &grid, &W, &tpu, &slots);
+      p.path = 1;
+      parts = kvc::kRopeTcParts;
+    } else if (kvc::latent_tc_supported(p)) {
+      kvc::latent_tc_plan(p, &grid, &W, &tpu, &slots);
+      p.path = 3;
+    } else if (kvc::dense_tc_supported(p)) {
+      kvc::dense_tc_plan(p, &grid, &W, &tpu, &slots);
+      p.path = 2;
+    }
+    if (p.path) {
+      p.S = slots;
+      p.seg_W = W;
+      p.seg_tpu = tpu;
+      p.seg_parts = parts;
+    }
   }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   char* ws = (char*)workspace;

@@ -62,6 +62,7 @@ struct Params {
   // units of seg_tpu tiles (0 = split partials indexed by split)
   int seg_W, seg_tpu;
   int seg_parts;         // partials written per CTA and unit on that path
+  int path;              // split kernel: 0 generic, 1 rope_tc, 2 dense_tc, 3 latent_tc, 4 rope_mma
   uint32_t* err;         // error word of the workspace (bounded waits that gave up)
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
   double rope_f[64];
@@ -117,6 +118,13 @@ bool latent_tc_supported(const Params& p);
 void latent_tc_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
 int latent_tc_slots(int batch, int n_kv_heads, int n_tokens);
 cudaError_t launch_latent_tc(const Params& p, cudaStream_t s);
+
+// warp-level tensor-core decode of pre-RoPE INT4 low-rank caches (reconstruction,
+// rotation and scores on mma.sync)
+bool rope_mma_supported(const Params& p);
+void rope_mma_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
+int rope_mma_slots(int batch, int n_kv_heads, int n_tokens);
+cudaError_t launch_rope_mma(const Params& p, cudaStream_t s);
 
 // Record a status and message for kvc_last_error(); returns st.
 kvc_status report_error(kvc_status st, const char* fmt, ...);

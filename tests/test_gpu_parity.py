@@ -286,3 +286,32 @@ def test_latent_tensor_core_peaked():
     a = synth.lowrank_cache(c)
     a["q"] = synth.to_bf16_bits(synth.bf16_bits_to_f32(a["q"]) * 8)
     assert_close(run_decode(c, a, 4096), oracle(c, a, 4096), what="latent peaked")
+
+
+# ------------------------------------------------------------------ pre-RoPE keys on warp-level MMAs
+
+
+@pytest.mark.parametrize("rv,page,Hq,B,n,cap", [
+    (48, 0, 32, 2, 4096, 4096),       # C2 ranks, whole 64-token rotation groups
+    (48, 0, 32, 2, 4001, 4016),       # ragged last tile, partial rotation group
+    (48, 0, 32, 1, 1, 16),            # one token
+    (32, 16, 16, 3, 1234, 1248),      # paged, two query heads per KV head
+    (64, 0, 64, 2, 777, 784),         # eight query heads per KV head
+])
+def test_rope_mma_path(rv, page, Hq, B, n, cap):
+    """Pre-RoPE INT4 keys with a capacity that is a multiple of 16 run on the
+    warp-level kernel (reconstruction, rotation and scores on mma.sync); per-row
+    lengths force the generic kernel.  Both must match the oracle."""
+    c = synth.config("c2", B=B, Hq=Hq, T=cap, rv=rv, page=page, seed=21 + rv)
+    a = synth.lowrank_cache(c)
+    ref = oracle(c, a, n)
+    assert_close(run_decode(c, a, n, capacity=cap), ref, what=f"rope mma rv={rv} n={n}")
+    got = run_decode(c, a, n, capacity=cap, seq_lens=[n] * B)
+    assert_close(got, ref, what=f"generic rv={rv} n={n}")
+
+
+def test_rope_mma_peaked():
+    c = synth.config("c2", B=2, T=2048)
+    a = synth.lowrank_cache(c)
+    a["q"] = synth.to_bf16_bits(synth.bf16_bits_to_f32(a["q"]) * 8)
+    assert_close(run_decode(c, a, 2048), oracle(c, a, 2048), what="rope mma peaked")
