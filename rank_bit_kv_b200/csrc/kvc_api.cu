@@ -89,6 +89,10 @@ size_t ws_bytes(const kvc_layout* L, int n_tokens) {
     const int Sr = kvc::rope_mma_slots(L->d.batch, L->d.n_kv_heads, nt1);
     if (Sr > S) S = Sr;
   }
+  if (L->d.kind == KVC_VARRATE) {
+    const int Sv = kvc::varrate_warp_slots(L->d.batch, nt1);
+    if (Sv > S) S = Sv;
+  }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   size_t b = kWsHeader + round_up(rows * L->qdim * sizeof(float), 256);
   b += round_up((size_t)S * rows * (L->vdim + 2) * sizeof(float), 256);
@@ -472,6 +476,10 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
       p.seg_W = W;
       p.seg_tpu = tpu;
       p.seg_parts = parts;
+    } else if (kvc::varrate_warp_supported(p)) {
+      // fixed token splits per batch row (one partial per CTA)
+      kvc::varrate_warp_plan(p, &p.S, &p.split_len);
+      p.path = 5;
     }
   }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;

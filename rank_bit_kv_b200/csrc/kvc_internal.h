@@ -62,7 +62,8 @@ struct Params {
   // units of seg_tpu tiles (0 = split partials indexed by split)
   int seg_W, seg_tpu;
   int seg_parts;         // partials written per CTA and unit on that path
-  int path;              // split kernel: 0 generic, 1 rope_tc, 2 dense_tc, 3 latent_tc, 4 rope_mma
+  int path;              // split kernel: 0 generic, 1 rope_tc, 2 dense_tc, 3 latent_tc, 4 rope_mma,
+                         // 5 varrate_warp
   uint32_t* err;         // error word of the workspace (bounded waits that gave up)
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
   double rope_f[64];
@@ -125,6 +126,12 @@ bool rope_mma_supported(const Params& p);
 void rope_mma_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
 int rope_mma_slots(int batch, int n_kv_heads, int n_tokens);
 cudaError_t launch_rope_mma(const Params& p, cudaStream_t s);
+
+// variable-rate layout, one lane per (KV head, query head)
+bool varrate_warp_supported(const Params& p);
+void varrate_warp_plan(const Params& p, int* splits, int* split_len);
+int varrate_warp_slots(int batch, int n_tokens);
+cudaError_t launch_varrate_warp(const Params& p, cudaStream_t s);
 
 // Record a status and message for kvc_last_error(); returns st.
 kvc_status report_error(kvc_status st, const char* fmt, ...);

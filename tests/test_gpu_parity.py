@@ -315,3 +315,25 @@ def test_rope_mma_peaked():
     a = synth.lowrank_cache(c)
     a["q"] = synth.to_bf16_bits(synth.bf16_bits_to_f32(a["q"]) * 8)
     assert_close(run_decode(c, a, 2048), oracle(c, a, 2048), what="rope mma peaked")
+
+
+# ------------------------------------------------------------------ variable rate, one lane per head pair
+
+
+@pytest.mark.parametrize("B,n", [(1, 1), (1, 17), (2, 2049), (3, 5000)])
+def test_varrate_warp_path(B, n):
+    """Variable-rate records run on the lane-per-(KV head, query head) kernel;
+    per-row lengths force the generic kernel.  Both must match the oracle."""
+    c = synth.config("c4", B=B, T=n)
+    a = synth.varrate_cache(c)
+    ref = oracle(c, a, n)
+    assert_close(run_decode(c, a, n), ref, what=f"varrate warp B={B} n={n}")
+    assert_close(run_decode(c, a, n, seq_lens=[n] * B), ref, what=f"generic B={B} n={n}")
+
+
+def test_varrate_warp_single_rank_64():
+    """Every token at the top rank: the ragged layout degenerates to the uniform
+    rank-64 one (the path with two scale groups per record)."""
+    c = synth.config("c4", B=1, T=700)
+    a = synth.varrate_cache(c, ranks={"k": np.full((1, 700), 64), "v": np.full((1, 700), 64)})
+    assert_close(run_decode(c, a, 700), oracle(c, a, 700), what="varrate rank 64")
