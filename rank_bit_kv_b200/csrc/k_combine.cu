@@ -132,9 +132,13 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Params p) {
 // the signs) is issued before any arithmetic, so the row costs one round trip
 // to memory instead of one per step.  The residual accumulator is mapped back
 // with the in-register Hadamard transform of one warp.
-constexpr int kFastS = 64, kFastVals = 16;
+constexpr int kFastS = 160;
 
+// NV partial values per thread, NM maxima per lane of warp 0: a small instance
+// for few partials (low register use, several blocks per SM) and a large one
+template <int NV, int NM>
 __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
+  constexpr int kFastVals = NV, kFastM = NM;
   __shared__ float ws[kFastS];
   __shared__ float red[kThreads];
   __shared__ float acc[256];
@@ -154,15 +158,14 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
     nS = (int)(e / p.seg_W - a / p.seg_W + 1) * p.seg_parts;
   }
   // ---- issue every load
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-  if (tid < 32) {
-    if (lane < nS) {
-      m_a = part[(size_t)lane * rows * pst + vdim];
-      l_a = part[(size_t)lane * rows * pst + vdim + 1];
-    }
-    if (lane + 32 < nS) {
-      m_b = part[(size_t)(lane + 32) * rows * pst + vdim];
-      l_b = part[(size_t)(lane + 32) * rows * pst + vdim + 1];
+  float mm[kFastM], ll[kFastM];
+#pragma unroll
+  for (int k = 0; k < kFastM; ++k) {
+    mm[k] = -INFINITY;
+    ll[k] = 0.f;
+    if (tid < 32 && lane + 32 * k < nS) {
+      mm[k] = part[(size_t)(lane + 32 * k) * rows * pst + vdim];
+      ll[k] = part[(size_t)(lane + 32 * k) * rows * pst + vdim + 1];
     }
   }
   const int K = kThreads / vdim;         // partial groups per value index
@@ -184,12 +187,18 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
   const float sgn = p.resid ? (float)p.signs_v[oi] * rsqrtf((float)kResidDim) : 0.f;
   // ---- weights
   if (tid < 32) {
-    const float mx = warp_max(fmaxf(m_a, m_b));
-    const float wa = (mx == -INFINITY || m_a == -INFINITY) ? 0.f : exp2f(m_a - mx);
-    const float wb = (mx == -INFINITY || m_b == -INFINITY) ? 0.f : exp2f(m_b - mx);
-    if (lane < nS) ws[lane] = wa;
-    if (lane + 32 < nS) ws[lane + 32] = wb;
-    const float lt = warp_sum((wa != 0.f ? wa * l_a : 0.f) + (wb != 0.f ? wb * l_b : 0.f));
+    float mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kFastM; ++k) mx = fmaxf(mx, mm[k]);
+    mx = warp_max(mx);
+    float lt = 0.f;
+#pragma unroll
+    for (int k = 0; k < kFastM; ++k) {
+      const float w = (mx == -INFINITY || mm[k] == -INFINITY) ? 0.f : exp2f(mm[k] - mx);
+      if (lane + 32 * k < nS) ws[lane + 32 * k] = w;
+      if (w != 0.f) lt = fmaf(w, ll[k], lt);
+    }
+    lt = warp_sum(lt);
     if (lane == 0) lsum = lt;
   }
   __syncthreads();
@@ -246,10 +255,13 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
 cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   if (p.S > kMaxS) return cudaErrorInvalidValue;
   const int rows = p.L * p.B * p.Hq;
-  const bool fast = p.kind == KVC_LOWRANK && p.d == 128 && p.L == 1 &&
-                    p.vdim == p.rv + (p.resid ? kResidDim : 0) && p.rv >= 16 && p.rv <= 64 &&
-                    p.S <= kFastS &&
-                    (p.S + kThreads / p.vdim - 1) / (kThreads / p.vdim) <= kFastVals;
+  const bool lowrank = p.kind == KVC_LOWRANK && p.vdim == p.rv + (p.resid ? kResidDim : 0) &&
+                       p.rv >= 16 && p.rv <= 64;
+  const bool varrate = p.kind == KVC_VARRATE && p.vdim == 64 && p.rv == 64 && !p.resid;
+  const int per_thread = (lowrank || varrate) ? (p.S + kThreads / p.vdim - 1) / (kThreads / p.vdim) : 0;
+  const bool fast = (lowrank || varrate) && p.d == 128 && p.L == 1 && p.S <= kFastS &&
+                    per_thread <= 40;
+  const bool small = fast && p.S <= 64 && per_thread <= 16;
   const size_t bytes = ((size_t)p.vdim + p.S + kThreads) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(combine_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -264,7 +276,8 @@ cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (fast) return cudaLaunchKernelEx(&cfg, combine_lowrank_kernel, p);
+  if (small) return cudaLaunchKernelEx(&cfg, combine_lowrank_kernel<16, 2>, p);
+  if (fast) return cudaLaunchKernelEx(&cfg, combine_lowrank_kernel<40, 5>, p);
   return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 

@@ -47,9 +47,21 @@ __device__ __forceinline__ void cp_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// nibble k of w as a float (exact: 2^23 + c with the 2^23 removed)
-__device__ __forceinline__ float nib(uint32_t w, int k) {
-  return __int_as_float(0x4B000000u | ((w >> (4 * k)) & 15u)) - 8388608.f;
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// the 8 nibbles of w as floats (exact): each nibble is moved into the low byte
+// of the bit pattern 0x4B0000xx = 2^23 + c, and 2^23 is subtracted
+__device__ __forceinline__ void nib8(uint32_t w, float (&c)[8]) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    c[2 * j] = __int_as_float(prmt(lo, 0x4B000000u, 0x7650u + j)) - 8388608.f;
+    c[2 * j + 1] = __int_as_float(prmt(hi, 0x4B000000u, 0x7650u + j)) - 8388608.f;
+  }
 }
 
 __device__ __forceinline__ float2 h2f2(uint32_t x) {
@@ -65,19 +77,27 @@ __device__ __forceinline__ float score_r(const uint8_t* rec, const float (&q)[kV
     const uint32_t w = *reinterpret_cast<const uint16_t*>(rec);
     const float s = __half2float(*reinterpret_cast<const __half*>(rec + 2));
     const float z = __half2float(*reinterpret_cast<const __half*>(rec + 4));
-    float d = 0.f;
+    float c[8];
+    nib8(w, c);
+    float d = c[0] * q[0];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) d = fmaf(nib(w, k), q[k], d);
+    for (int k = 1; k < 4; ++k) d = fmaf(c[k], q[k], d);
     return fmaf(s, d, z * pre[0]);
   } else {
     constexpr int NW = R / 8;
-    float d[2] = {0.f, 0.f};
+    float dw[NW];                       // one chain per code word (short dependency chains)
 #pragma unroll
     for (int wi = 0; wi < NW; ++wi) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(rec + 4 * wi);
+      float c[8];
+      nib8(*reinterpret_cast<const uint32_t*>(rec + 4 * wi), c);
+      float a = c[0] * q[8 * wi];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) d[wi / 4] = fmaf(nib(w, k), q[8 * wi + k], d[wi / 4]);
+      for (int k = 1; k < 8; ++k) a = fmaf(c[k], q[8 * wi + k], a);
+      dw[wi] = a;
     }
+    float d[2] = {0.f, 0.f};
+#pragma unroll
+    for (int wi = 0; wi < NW; ++wi) d[wi / 4] += dw[wi];
     const float2 sz0 = h2f2(*reinterpret_cast<const uint32_t*>(rec + R / 2));
     constexpr int P = R == 8 ? 1 : R == 16 ? 2 : 3;     // prefix of group 0 up to min(R, 32)
     float s = fmaf(sz0.x, d[0], sz0.y * pre[P]);
@@ -96,8 +116,10 @@ __device__ __forceinline__ void value_r(const uint8_t* rec, float p, float (&acc
     const uint32_t w = *reinterpret_cast<const uint16_t*>(rec);
     const float ps = p * __half2float(*reinterpret_cast<const __half*>(rec + 2));
     const float pz = p * __half2float(*reinterpret_cast<const __half*>(rec + 4));
+    float c[8];
+    nib8(w, c);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = fmaf(ps, nib(w, k), acc[k] + pz);
+    for (int k = 0; k < 4; ++k) acc[k] = fmaf(ps, c[k], acc[k] + pz);
   } else {
     constexpr int NW = R / 8;
     float ps[2], pz[2];
@@ -115,11 +137,12 @@ __device__ __forceinline__ void value_r(const uint8_t* rec, float p, float (&acc
     }
 #pragma unroll
     for (int wi = 0; wi < NW; ++wi) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(rec + 4 * wi);
+      float c[8];
+      nib8(*reinterpret_cast<const uint32_t*>(rec + 4 * wi), c);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int i = 8 * wi + k;
-        acc[i] = fmaf(ps[wi / 4], nib(w, k), acc[i] + pz[wi / 4]);
+        acc[i] = fmaf(ps[wi / 4], c[k], acc[i] + pz[wi / 4]);
       }
     }
   }
