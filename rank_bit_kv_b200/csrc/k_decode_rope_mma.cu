@@ -6,7 +6,8 @@
 //     group) and reconstructs K = L Bk with mma.sync m16n8k16 (M = 16 tokens,
 //     N = 128 dims, K = the rank; f16 accumulate), the Bk fragments read from
 //     shared memory with ldmatrix.trans;
-//   - applies the rotation of the token's position inside its 64-token group,
+//   - applies the rotation of the token's position inside its group of 128 (or
+//     64) tokens,
 //     R_delta, in f16x2 (cos / sin of delta * omega_i from a per-CTA table);
 //     the group's own rotation R_t0 is folded into the queries once per group
 //     (R_t = R_t0 R_delta, rotate-half pairs (i, i + 64));
@@ -33,7 +34,10 @@ constexpr int kPThreads = 32 * kPWarps;
 constexpr int kPStages = 8;
 constexpr int kPDist = kPStages - 2;     // tiles in flight ahead of the one computed
 constexpr int kPRank = 32;               // key rank handled (one scale group)
-constexpr int kPGroup = 64;              // tokens sharing one query rotation
+// tokens sharing one query rotation: 128 where the rotation table fits next to
+// the rings (value rank <= 48), else 64
+template <int RV>
+constexpr int group_of() { return RV <= 48 ? 128 : 64; }
 constexpr int kPMaxHkv = 8;
 constexpr int kBkRow = 272;              // smem bytes per Bk row (128 f16 + 16 pad)
 constexpr int kBkHead = kPRank * kBkRow; // one KV head's factor
@@ -53,12 +57,14 @@ struct PStage {
   static constexpr int BYTES = LV + kPT * RV / 2;
   static constexpr int CHUNKS = BYTES / 16;
   static constexpr int CPL = (CHUNKS + 31) / 32;
+  static constexpr int GROUP = group_of<RV>();
   // dynamic shared memory: factors, rotation table, per-warp group rotation, rings
   static constexpr int OFF_ROPE = kPMaxHkv * kBkHead;
-  static constexpr int OFF_QTAB = OFF_ROPE + kPGroup * kRopeRow;
+  static constexpr int OFF_QTAB = OFF_ROPE + GROUP * kRopeRow;
   static constexpr int OFF_QROW = OFF_QTAB + kPWarps * kQTab;
   static constexpr int OFF_RING = OFF_QROW + kPWarps * kQRows;
   static constexpr int SMEM = OFF_RING + kPWarps * kPStages * BYTES;
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 struct PWork {
@@ -139,9 +145,9 @@ __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork 
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.bk + ((size_t)h * kPRank + rank) * 128) + ch);
     *reinterpret_cast<uint4*>(psm + h * kBkHead + row * kBkRow + ch * 16) = v;
   }
-  // rotation table: delta in [0, 64), entry (m, c4) holds (cos, sin) of
+  // rotation table: delta in [0, GROUP), entry (m, c4) holds (cos, sin) of
   // delta * omega_i for dims i = 8 nt + 2 c4 + {0, 1}, nt = 2m, 2m + 1, packed f16x2
-  for (int e = tid; e < kPGroup * 16; e += kPThreads) {
+  for (int e = tid; e < L::GROUP * 16; e += kPThreads) {
     const int dl = e >> 4, m = (e >> 2) & 3, c = e & 3;
     uint32_t w[4];
 #pragma unroll
@@ -246,10 +252,10 @@ __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork 
     cur_J = -1;
   };
 
-  // queries rotated by R_t0, t0 = 64 J, scaled by the softmax scale (log2 e
+  // queries rotated by R_t0, t0 = GROUP J, scaled by the softmax scale (log2 e
   // folded in), as the score MMA's B fragments
   auto rotate_q = [&](int J) {
-    const double t0 = (double)J * kPGroup;
+    const double t0 = (double)J * L::GROUP;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int i = lane + 32 * k;
@@ -368,7 +374,7 @@ __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork 
       }
     }
     // R_delta on pairs (i, i + 64): n-tiles nt and nt + 8, rows g and g + 8
-    const int dl0 = (kPT * jt) % kPGroup + g;
+    const int dl0 = (kPT * jt) % L::GROUP + g;
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const uint32_t tab = rope_s + (dl0 + 8 * r) * kRopeRow;
@@ -490,7 +496,7 @@ __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork 
     return st;
   };
   auto score_tile = [&](bool tail, const uint8_t* st, int jt, int nt, float (&s)[4]) {
-    const int J = (kPT * jt) / kPGroup;
+    const int J = (kPT * jt) / L::GROUP;
     if (J != cur_J) {
       rotate_q(J);
       cur_J = J;

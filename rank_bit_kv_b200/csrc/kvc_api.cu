@@ -115,7 +115,7 @@ extern "C" {
 
 const char* kvc_last_error(void) { return g_err.c_str(); }
 
-const char* kvc_version(void) { return "kvc 0.2 (sm_100a; decode kernels rev 10)"; }
+const char* kvc_version(void) { return "kvc 0.2 (sm_100a; decode kernels rev 11)"; }
 
 kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out) {
   if (!desc || !out) return fail(KVC_EINVAL, "kvc_create_layout: NULL argument");
