@@ -21,10 +21,14 @@
 //     query operand uses the same order), and so is the ordering of value rows
 //     (undone when the partials are written); both are chosen so that one
 //     32-bit shared-memory word feeds whole operand registers.
-//   - Online softmax with a lazily raised reference maximum (raised only when
-//     a score exceeds it by more than 8 in log2 units).
-// Shared-memory rows of 32 bytes are stored with tokens 4..7 (mod 8) swapped
-// pairwise, which makes the value-operand loads free of bank conflicts.
+//   - MMA row slot i holds token (i & 8) | ((i & 7) >> 1) | ((i & 1) << 2), so
+//     that the value operand's token slots read tokens c4, c4 + 4, c4 + 8,
+//     c4 + 12 of lane c4 (every shared-memory load is a per-thread base plus an
+//     immediate, conflict-free); the residual key rows are stored in slot order.
+//   - Scores are kept in units of 2^-24 log2; online softmax with a lazily
+//     raised reference maximum (raised only when a score exceeds it by more
+//     than 8 in log2 units); the scores of tile k + 1 are formed before the
+//     softmax and value update of tile k.
 #include <math.h>
 
 #include <type_traits>
