@@ -363,6 +363,7 @@ cudaError_t launch_split(const Params& p, cudaStream_t s) {
     case 3: return launch_latent_tc(p, s);
     case 4: return launch_rope_mma(p, s);
     case 5: return launch_varrate_warp(p, s);
+    case 6: return launch_block_mma(p, s);
     default: break;
   }
   const Geo g = geometry(p);

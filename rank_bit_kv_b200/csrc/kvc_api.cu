@@ -93,6 +93,10 @@ size_t ws_bytes(const kvc_layout* L, int n_tokens) {
     const int Sv = kvc::varrate_warp_slots(L->d.batch, nt1);
     if (Sv > S) S = Sv;
   }
+  if (L->d.kind == KVC_BLOCK_SHARED) {
+    const int Sb = kvc::block_mma_slots(L->d.batch, L->L, L->d.n_q_heads, nt1);
+    if (Sb > S) S = Sb;
+  }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   size_t b = kWsHeader + round_up(rows * L->qdim * sizeof(float), 256);
   b += round_up((size_t)S * rows * (L->vdim + 2) * sizeof(float), 256);
@@ -480,6 +484,9 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
       // fixed token splits per batch row (one partial per CTA)
       kvc::varrate_warp_plan(p, &p.S, &p.split_len);
       p.path = 5;
+    } else if (kvc::block_mma_supported(p)) {
+      kvc::block_mma_plan(p, &p.S, &p.split_len);
+      p.path = 6;
     }
   }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;

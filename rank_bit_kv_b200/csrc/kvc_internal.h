@@ -63,7 +63,7 @@ struct Params {
   int seg_W, seg_tpu;
   int seg_parts;         // partials written per CTA and unit on that path
   int path;              // split kernel: 0 generic, 1 rope_tc, 2 dense_tc, 3 latent_tc, 4 rope_mma,
-                         // 5 varrate_warp
+                         // 5 varrate_warp, 6 block_mma
   uint32_t* err;         // error word of the workspace (bounded waits that gave up)
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
   double rope_f[64];
@@ -132,6 +132,12 @@ bool varrate_warp_supported(const Params& p);
 void varrate_warp_plan(const Params& p, int* splits, int* split_len);
 int varrate_warp_slots(int batch, int n_tokens);
 cudaError_t launch_varrate_warp(const Params& p, cudaStream_t s);
+
+// block-shared latent, 32 absorbed queries per CTA on mma.sync
+bool block_mma_supported(const Params& p);
+void block_mma_plan(const Params& p, int* splits, int* split_len);
+int block_mma_slots(int batch, int n_layers, int n_q_heads, int n_tokens);
+cudaError_t launch_block_mma(const Params& p, cudaStream_t s);
 
 // Record a status and message for kvc_last_error(); returns st.
 kvc_status report_error(kvc_status st, const char* fmt, ...);

@@ -337,3 +337,18 @@ def test_varrate_warp_single_rank_64():
     c = synth.config("c4", B=1, T=700)
     a = synth.varrate_cache(c, ranks={"k": np.full((1, 700), 64), "v": np.full((1, 700), 64)})
     assert_close(run_decode(c, a, 700), oracle(c, a, 700), what="varrate rank 64")
+
+
+# ------------------------------------------------------------------ block-shared latent on warp-level MMAs
+
+
+@pytest.mark.parametrize("B,n", [(1, 1), (2, 300), (1, 2049)])
+def test_block_mma_path(B, n):
+    """The block-shared latent for 4 layers runs on the CTA-cooperative mma.sync
+    kernel (32 absorbed queries per CTA); per-row lengths force the generic
+    kernel.  Both must match the oracle."""
+    c = synth.config("c3", B=B, T=n)
+    a = synth.block_shared_cache(c)
+    ref = oracle(c, a, n)
+    assert_close(run_decode(c, a, n), ref, what=f"block mma B={B} n={n}")
+    assert_close(run_decode(c, a, n, seq_lens=[n] * B), ref, what=f"generic B={B} n={n}")
