@@ -177,7 +177,11 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
     if (jj >= n_tiles) return 0;
     const int u = t / wk.tpu, jt = t % wk.tpu;
     const int b = u / Hkv, kvh = u % Hkv;
-    if (p.page) return (__ldg(p.page_table + (size_t)b * npp + jt) * Hkv + kvh) * kLT;
+    if (p.page) {
+      // a page id outside the cache is clamped (never read out of bounds)
+      const int pg = min(max(__ldg(p.page_table + (size_t)b * npp + jt), 0), p.n_pages - 1);
+      return (pg * Hkv + kvh) * kLT;
+    }
     return u * p.tmax + jt * kLT;
   };
   int rows_cur = tile_row(lane), rows_next = tile_row(32 + lane);

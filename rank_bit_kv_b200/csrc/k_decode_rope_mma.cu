@@ -200,7 +200,9 @@ __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork 
     const int u = t / wk.tpu, jt = t % wk.tpu;
     if (p.page) {
       const int b = u / Hkv, kvh = u % Hkv;
-      return (__ldg(p.page_table + (size_t)b * (p.tmax / kPT) + jt) * Hkv + kvh) * kPT;
+      // a page id outside the cache is clamped (never read out of bounds)
+      const int pg = min(max(__ldg(p.page_table + (size_t)b * (p.tmax / kPT) + jt), 0), p.n_pages - 1);
+      return (pg * Hkv + kvh) * kPT;
     }
     return u * p.tmax + jt * kPT;
   };
