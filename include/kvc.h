@@ -10,7 +10,7 @@
  *   - INT4 latent with per-group fp16 scale and zero, min/max uniform rule:
  *     "BellowsKV Architecture: Block-Shared Cache Latents, Outlier-Free Low-Bit
  *     Storage, and Single-Decision Eviction ...", "Worked Example: Why the
- *     Latent Quantizes Flat" (function qerr);
+ *     Latent Quantizes Flat";
  *   - keys stored before RoPE and rotated on reconstruction: "JoLT:
  *     Near-Lossless KV Cache Compression", "Key findings";
  *   - a rotated low-bit residual of the truncation error: "A JoLT for the KV
@@ -32,8 +32,7 @@
  *     host-side layout handle.  No entry point allocates device memory.
  *   - Work is enqueued on the caller's stream (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream).  No entry point synchronizes the
- *     device, except that kvc_append copies host-side VARRATE ranks with
- *     cudaMemcpyAsync from pageable memory (see kvc_append).
+ *     device.
  *   - Every entry point returns a kvc_status and never throws or aborts.  On
  *     error nothing is launched and kvc_last_error() describes the problem
  *     (thread-local string, valid until the next call on the same thread).
@@ -139,6 +138,12 @@ typedef struct kvc_layout kvc_layout;  /* opaque, host-side */
  * n_tokens: tokens 0..n_tokens-1 of every row are attended.  seq_lens
  *   (optional, device int32 [B]) gives per-row lengths; values are clamped to
  *   [0, n_tokens].  A row of length 0 produces a zero output.
+ * status: optional device uint32 word.  kvc_append ORs KVC_DEV_* bits into it
+ *   for every token it had to skip because a device-side argument was invalid
+ *   (see kvc_append); the library never clears it.  NULL: skips go unreported.
+ * Page-table entries outside [0, n_pages) never make a kernel touch memory
+ *   outside the cache: decode kernels clamp them (the row then reads some
+ *   page's data), append skips the token and sets KVC_DEV_BAD_PAGE.
  */
 typedef struct {
   void* lk_codes;
@@ -163,7 +168,18 @@ typedef struct {
   const int32_t* seq_lens;
   int32_t n_tokens;
   int32_t _reserved;
+  uint32_t* status;
 } kvc_cache;
+
+/* Bits of the device-side status words: kvc_cache.status (append) and the
+ * workspace error word (decode, see kvc_decode_attn). */
+enum {
+  KVC_DEV_WAIT_TIMEOUT = 1u,   /* decode: a bounded wait gave up; output invalid  */
+  KVC_DEV_BAD_POS = 2u,        /* append: pos[b] outside [0, max_tokens - n_new]  */
+  KVC_DEV_BAD_RANK = 4u,       /* append: a VARRATE rank not in {4,8,16,32,64}    */
+  KVC_DEV_BAD_PAGE = 8u,       /* append: a page-table entry outside [0, n_pages)  */
+  KVC_DEV_BAD_OFFSET = 16u     /* append: a VARRATE record beyond its byte stream  */
+};
 
 /* Indices into the sizes[] array filled by kvc_buffer_sizes(). */
 enum {
@@ -176,60 +192,108 @@ enum {
 };
 
 /* Validate a description and create an immutable layout handle.  Host only.
+ * Defines the stored format of the pages' compressed caches: a low-rank latent
+ * times a factor ("BELT Connects KV-Cache Compression ...", section 3),
+ * optionally quantized per group (BellowsKV page, "Worked Example: Why the
+ * Latent Quantizes Flat"), with keys pre-RoPE ("JoLT: Near-Lossless KV Cache
+ * Compression", "Key findings"), a rotated low-bit residual ("A JoLT for the KV
+ * cache ...", "Abstract (arXiv)"), a block-shared latent (BellowsKV page,
+ * "Share the Input, Not the Cache") or a per-token rank ("VarRate ...",
+ * "Summary").  desc is read, not kept; *out receives a handle the caller
+ * releases with kvc_destroy_layout.
  * Errors: KVC_EINVAL (NULL, non-positive or inconsistent sizes),
  * KVC_EUNSUPPORTED (e.g. resid_bits > 0 with head_dim != 128, rope with a
  * kind other than LOWRANK, a VARRATE max rank other than 64). */
 kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out);
 
-/* Release a handle (NULL is ignored). */
+/* Release a handle (NULL is ignored).  No counterpart on the pages. */
 void kvc_destroy_layout(kvc_layout* layout);
 
 /* Bytes each cache buffer must have (0 = buffer unused by this layout), in the
- * KVC_BUF_* order.  These are the closed forms of the stored format: e.g. an
- * INT4 low-rank row costs rank/2 + 4*ceil(rank/group) bytes per component. */
+ * KVC_BUF_* order; sizes[] is caller-owned host memory of KVC_NBUF entries.
+ * These are the closed forms of the stored format -- an INT4 low-rank row costs
+ * rank/2 + 4*ceil(rank/group) bytes per component -- the byte arithmetic the
+ * BellowsKV page does in "The Cache That Outgrew the Weights" for the dense
+ * cache.  Errors: KVC_EINVAL on NULL. */
 kvc_status kvc_buffer_sizes(const kvc_layout* layout, size_t sizes[KVC_NBUF]);
 
-/* Compressed bytes a decode step reads for n_tokens tokens (cache rows only,
+/* Compressed bytes a decode step reads for n_tokens tokens (cache rows only;
  * VARRATE: the exact record bytes are data dependent, so the expected size at
- * the average record is returned).  Used for achieved-bandwidth figures. */
+ * the average record is returned).  Used for achieved-bandwidth figures: decode
+ * re-reads the whole cache every step (BellowsKV page, "The Cache That Outgrew
+ * the Weights").  Returns 0 for a NULL layout or n_tokens <= 0. */
 size_t kvc_step_bytes(const kvc_layout* layout, int32_t n_tokens);
 
-/* Device workspace bytes kvc_decode_attn needs for contexts up to n_tokens. */
+/* Device workspace bytes kvc_decode_attn needs for contexts up to n_tokens
+ * (error word, projected queries, split partials).  No counterpart on the
+ * pages (split-T partials are this library's design).  0 for NULL. */
 size_t kvc_workspace_bytes(const kvc_layout* layout, int32_t n_tokens);
 
 /* Number of kernel launches one kvc_decode_attn call makes for n_tokens. */
 int32_t kvc_decode_launches(const kvc_layout* layout, int32_t n_tokens);
 
-/* Append n_new tokens to every batch row.
+/* Append n_new tokens to every batch row: project each new pre-RoPE key and
+ * value onto the latent and quantize it into its slot.  Passages: the latent
+ * times factor representation ("BELT ...", section 3), the per-group min/max
+ * INT4 rule with fp16 scale and zero (BellowsKV page, "Worked Example: Why the
+ * Latent Quantizes Flat"), keys compressed before RoPE ("JoLT: Near-Lossless
+ * KV Cache Compression", "Key findings"), the rotated low-bit residual of the
+ * truncation error ("A JoLT for the KV cache ...", "Abstract (arXiv)"), ragged
+ * per-token ranks ("VarRate ...", "Summary").
  *   k_new, v_new: device bf16 [B, Hkv, n_new, d] pre-RoPE keys / values
  *     (DENSE with n_layers > 1: [n_layers, B, Hkv, n_new, d]);
  *     BLOCK_SHARED: k_new = the latent, bf16 [B, n_new, latent_dim]; v_new unused.
- *   pos: HOST int32 [B], slot of each row's first new token; the tokens go to
- *     slots pos[b] .. pos[b] + n_new - 1 (KVC_ECAPACITY beyond max_tokens).
- *   new_ranks: VARRATE only, HOST uint8 [2, B, n_new] (K ranks, then V ranks),
- *     each in {4, 8, 16, 32, 64}; they are copied into rank_k / rank_v with
- *     cudaMemcpyAsync (pageable source: the call returns once they are
- *     staged).  The records of row b are written from offset[b][pos[b]], which
+ *   pos: DEVICE int32 [B], slot of each row's first new token; the tokens go to
+ *     slots pos[b] .. pos[b] + n_new - 1.
+ *   new_ranks: VARRATE only, DEVICE uint8 [2, B, n_new] (K ranks, then V
+ *     ranks), each in {4, 8, 16, 32, 64}; the kernel stores them in rank_k /
+ *     rank_v.  The records of row b are written from offset[b][pos[b]], which
  *     must already be valid, and offset[b][pos[b] + 1 ..] are set.
- * LOWRANK append projects x onto the factor rows (l = x Bk^T), quantizes l per
- * group (codes = clamp(round_half_even((l - z) / s), 0, 15), s = fp16((max -
- * min)/15), z = fp16(min)); with a residual, y = Q (x - l_hat Bk) is stored as
- * 2-bit codes clamp(floor(y/s) + 2, 0, 3) with s = fp16(max|y| / 1.5).
- * BLOCK_SHARED: s = fp16(max|x|/7) per group, code = clamp(round(x/s),-7,7)+8.
- * fp16 latent layouts store l rounded to fp16. */
+ * All pointers are caller-owned device memory read or written on the stream.
+ * Host-detectable errors (NULL, misalignment, n_new < 1 or > max_tokens, a
+ * VARRATE call without new_ranks) return before anything is launched.  pos and
+ * the ranks live on the device, so the kernels check them: a row whose pos is
+ * outside [0, max_tokens - n_new] is skipped (KVC_DEV_BAD_POS), a token with a
+ * rank outside the set skips its row from that token on (KVC_DEV_BAD_RANK,
+ * offsets stay consistent), a token whose page-table entry is outside
+ * [0, n_pages) is skipped (KVC_DEV_BAD_PAGE), and a VARRATE record that would
+ * run past its stream is not written (KVC_DEV_BAD_OFFSET); the bits are ORed
+ * into cache->status when it is not NULL.  Nothing is written outside the
+ * cache buffers.
+ * Arithmetic: LOWRANK projects x onto the factor rows (l = x Bk^T, fp32),
+ * then per group z = fp16(min), s = fp16((max - min)/15) and each element is
+ * coded as the nearest step of s above z (IEEE fp32 division, ties to even,
+ * clamped to 0..15; code 0 when s = 0); with a residual, y = Q (x - l_hat Bk)
+ * is stored as 2-bit codes clamp(floor(y/s) + 2, 0, 3) with
+ * s = fp16(max|y| / 1.5).  BLOCK_SHARED: s = fp16(max|x|/7) per group, code =
+ * clamp(round(x/s), -7, 7) + 8.  fp16 latent layouts store l rounded to fp16. */
 kvc_status kvc_append(const kvc_layout* layout, const kvc_cache* cache,
                       const void* k_new, const void* v_new, const int32_t* pos,
                       int32_t n_new, const uint8_t* new_ranks, void* stream);
 
-/* Single-token decode attention over tokens [0, len_b) of every row.
+/* Single-token decode attention over tokens [0, len_b) of every row,
+ * evaluated directly over the stored factors without materializing dense K/V
+ * ("A JoLT for the KV cache ...", "Abstract (arXiv)", FlashJoLT; "BELT ...",
+ * section 4 on kernels over the compressed cache): latent-space scores
+ * q Bk^T . l_t, or keys reconstructed and rotated per tile when stored
+ * pre-RoPE ("JoLT: Near-Lossless KV Cache Compression", "Key findings"); one
+ * latent read by all layers of its block (BellowsKV page, "Share the Input,
+ * Not the Cache"); per-token ranks ("VarRate ...", "Summary").  The result is
+ * softmax(scale * q . k_t) . v_t over the dequantized, reconstructed k, v.
  *   q: device bf16 [B, Hq, d] (already rotated by the caller when rope = 1);
  *      BLOCK_SHARED / layered DENSE: [n_layers, B, Hq, d].
  *   out: device fp32 (or bf16 if out_bf16) with q's shape.
- *   workspace: device, >= kvc_workspace_bytes(layout, cache->n_tokens) bytes;
- *      its contents on entry do not matter.
+ *   workspace: device, >= kvc_workspace_bytes(layout, cache->n_tokens) bytes,
+ *      16-byte aligned, caller-owned; its contents on entry do not matter.
+ *      Bytes 0..3 hold the error word afterwards: the call zeroes it (on the
+ *      stream) before any kernel that can set it, and a kernel whose bounded
+ *      wait gave up ORs KVC_DEV_WAIT_TIMEOUT into it -- the output of such a
+ *      call is invalid.  Read it after the stream has completed.
+ * Host-detectable errors (NULL, misalignment, n_tokens beyond max_tokens, a
+ * small workspace, missing cache buffers) return before anything is enqueued.
  * Launches kvc_decode_launches() kernels: a query projection, the split-T
  * fused decode over the compressed tiles, and the split combine with the
- * up-projection. */
+ * up-projection (on some paths a zeroing of the error word precedes them). */
 kvc_status kvc_decode_attn(const kvc_layout* layout, const kvc_cache* cache,
                            const void* q, void* out, void* workspace,
                            size_t ws_bytes, void* stream);
@@ -256,15 +320,83 @@ kvc_status kvc_decode_attn_timed(const kvc_layout* layout, const kvc_cache* cach
  * for kvc_decode_attn, which this call runs with that array as the workspace.
  *   - Layouts whose kvc_workspace_bytes(layout, cache->n_tokens) exceeds
  *     KVC_STATIC_SCRATCH_BYTES are rejected with KVC_EWORKSPACE (nothing runs).
+ *     Every other host-detectable error is reported as by kvc_decode_attn,
+ *     also before anything is enqueued.
  *   - The first call on a device looks up the array's device address on the
  *     current device (once per device, with that device current); make that
  *     first call before any stream capture.
  *   - Every call on a device shares the one array and leaves its contents
- *     behind; the call clears what must start at zero (the error word) on the
- *     stream before the kernels run.  Calls that overlap on the GPU (other
- *     streams, other threads) race on the array: serialize them. */
+ *     behind; what must start at zero (the error word) is cleared on the
+ *     stream before the kernels that can set it.  Calls that overlap on the
+ *     GPU (other streams, other threads) race on the array: serialize them. */
 kvc_status kvc_decode_attn_static(const kvc_layout* layout, const kvc_cache* cache,
                                   const void* q, void* out, void* stream);
+
+/* Error word of the built-in scratch area on the current device (the
+ * workspace error word of the last kvc_decode_attn_static call, see
+ * kvc_decode_attn): enqueues a 4-byte copy of it to dst (device memory or
+ * pinned host memory, caller-owned) on the stream; read dst after the stream
+ * has completed.  No counterpart on the pages.  Errors: KVC_EINVAL on NULL dst,
+ * KVC_ECUDA if the copy cannot be enqueued. */
+kvc_status kvc_static_error_word(uint32_t* dst, void* stream);
+
+/* ---- Joint rank / residual-bit allocation (host only) -------------------
+ * "JoLT: Near-Lossless KV Cache Compression", section "How JoLT works": the
+ * layers are grouped, the keys and the values of each group are separate
+ * cells, and one Lagrangian multiplier picks every cell's ranks and residual
+ * bit-width under a shared byte budget; "A JoLT for the KV cache ...",
+ * "Abstract (arXiv)": a single Lagrangian dual under a global byte
+ * constraint.  The chosen (rank, bits) of a cell become the rank_k / rank_v and
+ * resid_bits of the layout that stores it. */
+#define KVC_MAX_RESID_BITS 8
+
+typedef struct {
+  int32_t rank;   /* latent rank of the option (1..spec_len)                  */
+  int32_t bits;   /* residual bits per coordinate, 0 = no residual (0..8)     */
+} kvc_rank_bits;
+
+/* Byte and distortion tables of every (cell, option), host arrays
+ * [n_cells, n_options] written by the call.  Per cell: spectra
+ * [n_cells, spec_len] squared singular values of its (rows x head_dim) data,
+ * descending; rows[c] stored token rows, heads[c] factors (one per KV head).
+ *   bytes(r, b) = rows * (ceil(r * latent_bits / 8) + 4 * ceil(r / group)
+ *                 [+ head_dim * b / 8 + 2 when b > 0])
+ *                 + heads * r * head_dim * 2 [+ heads * head_dim when b > 0]
+ *   distortion(r, b) = eta_latent * (sum of the first r squared singular
+ *                 values) + eta_resid[b] * (sum of the rest)
+ * (latent_bits 16: no scale/zero bytes).  eta_resid is indexed by the bit
+ * width (entries 0..KVC_MAX_RESID_BITS; eta_resid[0] = 1 means the truncated
+ * tail is lost).  The distortion model is this library's reading: the pages
+ * state the allocation, not the error model.  Errors: KVC_EINVAL (NULL,
+ * empty sizes, an option outside the spectrum or the bit range). */
+kvc_status kvc_rank_bit_tables(int32_t n_cells, int32_t spec_len, const double* spectra,
+                               const int64_t* rows, const int32_t* heads, int32_t n_options,
+                               const kvc_rank_bits* options, int32_t head_dim,
+                               int32_t latent_bits, int32_t group, double eta_latent,
+                               const double* eta_resid, double* bytes, double* distortion);
+
+/* One Lagrangian multiplier for all cells: each cell takes the option that
+ * minimises distortion + lambda * bytes (ties: fewer bytes, then the earlier
+ * option), and lambda is the smallest of the pairwise break points
+ * (D_a - D_b) / (B_b - B_a) (or 0) at which the total bytes fit the budget --
+ * found exactly, by a binary search over the sorted break points.  choice
+ * [n_cells] (host) receives the option index of every cell, *lambda (may be
+ * NULL) the multiplier.  Among all allocations that use no more bytes, the
+ * result has the least total distortion.  Errors: KVC_EINVAL (NULL, empty or
+ * non-finite tables), KVC_ECAPACITY (even the cheapest options exceed the
+ * budget). */
+kvc_status kvc_allocate_rank_bits(int32_t n_cells, int32_t n_options, const double* bytes,
+                                  const double* distortion, double budget, int32_t* choice,
+                                  double* lambda);
+
+/* Test switch (per calling thread, off by default): while on, decode calls
+ * whose split kernel has bounded waits (the tcgen05 pre-RoPE kernel) enqueue
+ * that kernel without its tile copies, so its waits run out after their limit
+ * (0.5 s), it sets KVC_DEV_WAIT_TIMEOUT in the workspace error word and exits
+ * cleanly; the output of such a call is invalid.  Used to test that a wait
+ * that gives up is reported and leaves the context usable.  No counterpart on
+ * the pages. */
+void kvc_test_skip_tile_copies(int32_t on);
 
 /* Thread-local description of the last error on this thread ("" if none). */
 const char* kvc_last_error(void);

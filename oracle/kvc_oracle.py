@@ -17,8 +17,10 @@ low-bit KV caches):
   quantizer is the min/max uniform rule of the worked example on the page
   "BellowsKV Architecture: Block-Shared Cache Latents, Outlier-Free Low-Bit
   Storage, and Single-Decision Eviction ..." (section "Worked Example: Why the
-  Latent Quantizes Flat", function ``qerr``): s = (hi - lo) / (2^bits - 1),
-  q = round((v - lo) / s) * s + lo, with Python's round (half to even).
+  Latent Quantizes Flat"): the range between a group's smallest and largest
+  value is cut into 2^bits - 1 equal steps, every value is replaced by its
+  nearest step counted from the minimum, ties going to the even step (the
+  rounding of the example's language).
 * Block-shared latents: one latent per block of n layers, every layer
   reconstructing its own keys and values through its own up-projection; the
   latent is quantized with one scale per group of adjacent coordinates and no
@@ -126,7 +128,7 @@ def n_groups(n, g):
 
 
 # ----------------------------------------------------------------------------
-# quantizers (BellowsKV page, "Worked Example", function qerr)
+# quantizers (BellowsKV page, "Worked Example: Why the Latent Quantizes Flat")
 # ----------------------------------------------------------------------------
 
 

@@ -8,9 +8,15 @@
 //   residual:       e = x - l_hat Bk, y = H (diag(signs) e) / sqrt(128),
 //                   s = fp16(max|y| / 1.5), code = clamp(floor(y / s) + 2, 0, 3)
 //   block-shared:   s = fp16(max|x| / 7), code = clamp(rint(x / s), -7, 7) + 8
-// This is the min/max rule of the BellowsKV worked example ("Worked Example:
-// Why the Latent Quantizes Flat", qerr: s = (hi - lo) / 15,
-// round((v - lo) / s)) with the scale and zero stored in fp16.
+// The INT4 rule is the per-group min/max uniform quantizer of the BellowsKV
+// page ("Worked Example: Why the Latent Quantizes Flat"): fifteen equal steps
+// between the group's extremes, each value coded by its nearest step, here with
+// the step and the offset stored in fp16.
+//
+// pos and the VARRATE ranks are device arrays, so the kernels validate them:
+// rows with a slot range outside the cache, tokens with a bad rank or page id,
+// and records that would run past their stream are skipped (never written out
+// of bounds) and reported by KVC_DEV_* bits in the optional status word.
 #include <math.h>
 
 #include "kvc_device.cuh"
@@ -19,6 +25,20 @@ namespace kvc {
 namespace {
 
 constexpr int kThreads = 128;
+
+__device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// First slot of row b's new tokens, or -1 when pos[b] leaves the cache.
+__device__ __forceinline__ int first_slot(const AppendParams& a, int b) {
+  const int p0 = a.pos[b];
+  return (p0 < 0 || p0 > a.p.tmax - a.n_new) ? -1 : p0;
+}
+
+__device__ __forceinline__ bool varrate_rank_ok(int r) {
+  return r == 4 || r == 8 || r == 16 || r == 32 || r == 64;
+}
 
 // Quantize lat[0..r) in groups of g into packed INT4 codes and (s, z) pairs.
 __device__ void quant_int4_asym(const float* lat, int r, int g, uint8_t* codes, __half* sz,
@@ -70,14 +90,28 @@ __global__ void __launch_bounds__(kThreads) append_lowrank_kernel(AppendParams a
   const int b = idx / p.Hkv;
   const int tid = threadIdx.x;
   const int d = p.d;
-  const int tok = a.pos[b] + i;
+  const int p0 = first_slot(a, b);
+  if (p0 < 0) {                       // whole block leaves before any barrier
+    if (tid == 0 && h == 0 && comp == 0 && i == 0) flag(a.status, KVC_DEV_BAD_POS);
+    return;
+  }
+  const int tok = p0 + i;
+  if (p.page) {
+    const int pp = p.page_table[(int64_t)b * (p.tmax / p.page) + tok / p.page];
+    if (pp < 0 || pp >= p.n_pages) {
+      if (tid == 0 && h == 0 && comp == 0) flag(a.status, KVC_DEV_BAD_PAGE);
+      return;
+    }
+  }
   const __nv_bfloat16* src = (comp == 0 ? a.k_new : a.v_new) + (((int64_t)b * p.Hkv + h) * a.n_new + i) * d;
   for (int j = tid; j < d; j += kThreads) xs[j] = bf2f(src[j]);
 
   int r;
   const __half* fac;
   if (p.kind == KVC_VARRATE) {
-    r = (comp == 0 ? p.rank_k : p.rank_v)[(int64_t)b * p.tmax + tok];
+    // stored by the offsets kernel: 0 when the token was skipped
+    r = (comp == 0 ? a.rank_k_w : a.rank_v_w)[(int64_t)b * p.tmax + tok];
+    if (!varrate_rank_ok(r)) return;
     fac = (comp == 0 ? p.bk : p.bv) + (int64_t)h * 64 * d;
   } else {
     r = comp == 0 ? p.rk : p.rv;
@@ -95,7 +129,12 @@ __global__ void __launch_bounds__(kThreads) append_lowrank_kernel(AppendParams a
   if (p.kind == KVC_VARRATE) {
     const int* off = comp == 0 ? a.off_k_w : a.off_v_w;
     uint8_t* stream = (comp == 0 ? a.lk_w : a.lv_w) + (size_t)b * p.stream_bytes;
-    uint8_t* rec = stream + off[(int64_t)b * (p.tmax + 1) + tok] + h * varrate_head_bytes(r);
+    const int64_t o = (int64_t)off[(int64_t)b * (p.tmax + 1) + tok] + h * varrate_head_bytes(r);
+    if (o < 0 || o + varrate_head_bytes(r) > (int64_t)p.stream_bytes) {
+      if (tid == 0) flag(a.status, KVC_DEV_BAD_OFFSET);
+      return;
+    }
+    uint8_t* rec = stream + o;
     quant_int4_asym(lat, r, 32, rec, reinterpret_cast<__half*>(rec + r / 2), nullptr, tid);
     return;
   }
@@ -145,24 +184,51 @@ __global__ void __launch_bounds__(kThreads) append_lowrank_kernel(AppendParams a
   }
 }
 
-// VARRATE: offsets of the new records, offset[pos + i + 1] = offset[pos + i] + size.
+// VARRATE: ranks and offsets of the new records, offset[pos + i + 1] =
+// offset[pos + i] + size.  A token whose K or V rank is outside the set, or
+// whose record would run past the stream, is stored as an empty record of
+// rank 0 (the append kernel then skips it and decode ignores it).
 __global__ void varrate_offsets_kernel(AppendParams a) {
   const Params& p = a.p;
   const int comp = blockIdx.x % 2, b = blockIdx.x / 2;
   if (threadIdx.x != 0) return;
+  const int p0 = first_slot(a, b);
+  if (p0 < 0) {
+    if (comp == 0) flag(a.status, KVC_DEV_BAD_POS);
+    return;
+  }
   int* off = (comp == 0 ? a.off_k_w : a.off_v_w) + (int64_t)b * (p.tmax + 1);
-  const uint8_t* rank = (comp == 0 ? p.rank_k : p.rank_v) + (int64_t)b * p.tmax;
-  int o = off[a.pos[b]];
+  uint8_t* rank = (comp == 0 ? a.rank_k_w : a.rank_v_w) + (int64_t)b * p.tmax;
+  const uint8_t* nk = a.new_ranks + (int64_t)b * a.n_new;
+  const uint8_t* nv = a.new_ranks + ((int64_t)p.B + b) * a.n_new;
+  int64_t o = off[p0];
+  bool dead = o < 0 || o > (int64_t)p.stream_bytes;
+  if (dead) flag(a.status, KVC_DEV_BAD_OFFSET);
   for (int i = 0; i < a.n_new; ++i) {
-    o += p.Hkv * varrate_head_bytes(rank[a.pos[b] + i]);
-    off[a.pos[b] + i + 1] = o;
+    const int rk = nk[i], rv = nv[i];
+    const bool ok = varrate_rank_ok(rk) && varrate_rank_ok(rv);
+    if (!ok && comp == 0) flag(a.status, KVC_DEV_BAD_RANK);
+    int size = (ok && !dead) ? p.Hkv * varrate_head_bytes(comp == 0 ? rk : rv) : 0;
+    if (size && o + size > (int64_t)p.stream_bytes) {
+      dead = true;
+      size = 0;
+      flag(a.status, KVC_DEV_BAD_OFFSET);
+    }
+    rank[p0 + i] = size ? (uint8_t)(comp == 0 ? rk : rv) : 0;
+    o += size;
+    off[p0 + i + 1] = (int)o;
   }
 }
 
 __global__ void __launch_bounds__(kThreads) append_block_kernel(AppendParams a) {
   const Params& p = a.p;
   const int i = blockIdx.x % a.n_new, b = blockIdx.x / a.n_new;
-  const int tok = a.pos[b] + i;
+  const int p0 = first_slot(a, b);
+  if (p0 < 0) {
+    if (threadIdx.x == 0 && i == 0) flag(a.status, KVC_DEV_BAD_POS);
+    return;
+  }
+  const int tok = p0 + i;
   const int D = p.D, g = p.g, ng = D / g;
   const __nv_bfloat16* src = a.k_new + ((int64_t)b * a.n_new + i) * D;
   const int64_t mi = (int64_t)b * p.tmax + tok;
@@ -202,8 +268,13 @@ __global__ void append_dense_kernel(AppendParams a) {
   const int b = idx % p.B;
   const int l = idx / p.B;
   const int d = p.d;
+  const int p0 = first_slot(a, b);
+  if (p0 < 0) {
+    if (threadIdx.x == 0 && i == 0 && h == 0 && l == 0) flag(a.status, KVC_DEV_BAD_POS);
+    return;
+  }
   const int64_t src = ((((int64_t)l * p.B + b) * p.Hkv + h) * a.n_new + i) * d;
-  const int64_t dst = ((((int64_t)l * p.B + b) * p.Hkv + h) * p.tmax + a.pos[b] + i) * d;
+  const int64_t dst = ((((int64_t)l * p.B + b) * p.Hkv + h) * p.tmax + p0 + i) * d;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
     a.kd_w[dst + j] = a.k_new[src + j];
     a.vd_w[dst + j] = a.v_new[src + j];

@@ -216,7 +216,10 @@ __global__ void __launch_bounds__(kThreads, 1) rope_tc_kernel(Params p, Work wk,
     // multicast) completing on the stage's full barrier
     int issued_upto = 0;  // tiles issued
     TileCursor cur(t_first, wk.tpu);
-    for (int jj = 0; jj < n_tiles && !*abort; ++jj, cur.next()) {
+    // (test switch: with no copies issued, every consumer's bounded wait runs
+    // out and the CTA takes its abort path)
+    const int n_issue = p.test_no_copies ? 0 : n_tiles;
+    for (int jj = 0; jj < n_issue && !*abort; ++jj, cur.next()) {
       const int s = slot_of<kStagesLog2>(jj);
       if (!mbar_wait(&bars.empty[s], phase_of<kStagesLog2>(jj) ^ 1, abort, err)) break;
       const int nt = cur.valid_rows(p.n_tokens);

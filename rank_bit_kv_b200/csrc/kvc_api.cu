@@ -24,6 +24,7 @@ struct kvc_layout {
 namespace {
 
 thread_local std::string g_err;
+thread_local int g_test_no_copies = 0;   // kvc_test_skip_tile_copies
 
 kvc_status fail(kvc_status st, const char* fmt, ...) {
   char buf[512];
@@ -118,6 +119,8 @@ kvc_status kvc::report_error(kvc_status st, const char* fmt, ...) {
 extern "C" {
 
 const char* kvc_last_error(void) { return g_err.c_str(); }
+
+void kvc_test_skip_tile_copies(int32_t on) { g_test_no_copies = on ? 1 : 0; }
 
 const char* kvc_version(void) { return "kvc 0.2 (sm_100a; decode kernels rev 11)"; }
 
@@ -454,6 +457,7 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
   kvc_status st = fill_params(L, c, &p);
   if (st != KVC_OK) return st;
   p.q = (const __nv_bfloat16*)q;
+  p.test_no_copies = g_test_no_copies;
   p.out = out;
   p.out_bf16 = L->d.out_bf16;
   plan(L, c->n_tokens, &p.S, &p.split_len);
@@ -496,6 +500,11 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
   p.part = (float*)(ws + kWsHeader + round_up(rows * L->qdim * sizeof(float), 256));
   cudaStream_t s = (cudaStream_t)stream;
   cudaGetLastError();  // clear a stale error so it is not reported as ours
+  if (kvc::path_sets_error_word(p)) {
+    // the workspace's previous contents do not matter: start the word at zero
+    st = launch_status(cudaMemsetAsync(p.err, 0, sizeof(uint32_t), s), "error word reset");
+    if (st != KVC_OK) return st;
+  }
   if (kvc::needs_qproj(p)) {
     st = launch_status(kvc::launch_qproj(p, s), "qproj launch");
     if (st != KVC_OK) return st;
@@ -521,22 +530,17 @@ extern "C" kvc_status kvc_append(const kvc_layout* L, const kvc_cache* c, const 
   if (!L || !c || !pos) return fail(KVC_EINVAL, "kvc_append: NULL argument");
   const kvc_layout_desc& d = L->d;
   if (n_new < 1) return fail(KVC_EINVAL, "n_new %d < 1", n_new);
+  if (n_new > d.max_tokens)
+    return fail(KVC_ECAPACITY, "n_new %d > max_tokens %d", n_new, d.max_tokens);
   if (!k_new || (d.kind != KVC_BLOCK_SHARED && !v_new))
     return fail(KVC_EINVAL, "kvc_append: k_new / v_new is NULL");
-  if (!aligned16(k_new) || (v_new && !aligned16(v_new)))
-    return fail(KVC_EALIGN, "k_new / v_new must be 16-byte aligned");
-  for (int b = 0; b < d.batch; ++b) {
-    if (pos[b] < 0 || (int64_t)pos[b] + n_new > d.max_tokens)
-      return fail(KVC_ECAPACITY, "row %d: slots %d..%d beyond max_tokens %d", b, pos[b],
-                  pos[b] + n_new - 1, d.max_tokens);
-  }
+  if (!aligned16(k_new) || (v_new && !aligned16(v_new)) || !aligned16(pos))
+    return fail(KVC_EALIGN, "k_new / v_new / pos must be 16-byte aligned");
+  if (c->status && (reinterpret_cast<uintptr_t>(c->status) & 3u))
+    return fail(KVC_EALIGN, "cache.status must be 4-byte aligned");
   if (d.kind == KVC_VARRATE) {
     if (!new_ranks) return fail(KVC_EINVAL, "VARRATE append needs new_ranks");
-    for (int64_t i = 0; i < 2LL * d.batch * n_new; ++i) {
-      const int r = new_ranks[i];
-      if (r != 4 && r != 8 && r != 16 && r != 32 && r != 64)
-        return fail(KVC_EINVAL, "rank %d not in {4, 8, 16, 32, 64}", r);
-    }
+    if (!aligned16(new_ranks)) return fail(KVC_EALIGN, "new_ranks must be 16-byte aligned");
   }
   kvc::AppendParams* a = new (std::nothrow) kvc::AppendParams();
   if (!a) return fail(KVC_EINVAL, "out of host memory");
@@ -550,7 +554,9 @@ extern "C" kvc_status kvc_append(const kvc_layout* L, const kvc_cache* c, const 
   a->k_new = (const __nv_bfloat16*)k_new;
   a->v_new = (const __nv_bfloat16*)v_new;
   a->n_new = n_new;
-  for (int b = 0; b < d.batch; ++b) a->pos[b] = pos[b];
+  a->pos = pos;
+  a->new_ranks = new_ranks;
+  a->status = c->status;
   a->lk_w = (uint8_t*)c->lk_codes;
   a->lksz_w = (__half*)c->lk_sz;
   a->lv_w = (uint8_t*)c->lv_codes;
@@ -563,20 +569,11 @@ extern "C" kvc_status kvc_append(const kvc_layout* L, const kvc_cache* c, const 
   a->vd_w = (__nv_bfloat16*)c->v_dense;
   a->off_k_w = c->offset_k;
   a->off_v_w = c->offset_v;
+  a->rank_k_w = c->rank_k;
+  a->rank_v_w = c->rank_v;
   cudaStream_t s = (cudaStream_t)stream;
   cudaGetLastError();
-  if (d.kind == KVC_VARRATE) {
-    for (int comp = 0; comp < 2 && st == KVC_OK; ++comp) {
-      uint8_t* dst = comp == 0 ? c->rank_k : c->rank_v;
-      for (int b = 0; b < d.batch && st == KVC_OK; ++b) {
-        cudaError_t e = cudaMemcpyAsync(dst + (size_t)b * d.max_tokens + pos[b],
-                                        new_ranks + ((size_t)comp * d.batch + b) * n_new,
-                                        n_new, cudaMemcpyHostToDevice, s);
-        st = launch_status(e, "rank copy");
-      }
-    }
-  }
-  if (st == KVC_OK) st = launch_status(kvc::launch_append(*a, s), "append launch");
+  st = launch_status(kvc::launch_append(*a, s), "append launch");
   delete a;
   if (st != KVC_OK) return st;
   return ok();

@@ -18,12 +18,16 @@ __device__ __forceinline__ int row_len(const Params& p, int b) {
   return n;
 }
 
+// Physical page of token t of batch row b, clamped to the pool so that a bad
+// page-table entry never sends a read outside the cache.
+__device__ __forceinline__ int page_of(const Params& p, int b, int t) {
+  const int pp = p.page_table[(int64_t)b * (p.tmax / p.page) + t / p.page];
+  return min(max(pp, 0), p.n_pages - 1);
+}
+
 // Row index of (batch row b, KV head h, token t) in a low-rank component.
 __device__ __forceinline__ int64_t lowrank_row(const Params& p, int b, int h, int t) {
-  if (p.page) {
-    const int pp = p.page_table[(int64_t)b * (p.tmax / p.page) + t / p.page];
-    return ((int64_t)pp * p.Hkv + h) * p.page + (t % p.page);
-  }
+  if (p.page) return ((int64_t)page_of(p, b, t) * p.Hkv + h) * p.page + (t % p.page);
   return ((int64_t)b * p.Hkv + h) * p.tmax + t;
 }
 

@@ -65,6 +65,7 @@ struct Params {
   int path;              // split kernel: 0 generic, 1 rope_tc, 2 dense_tc, 3 latent_tc, 4 rope_mma,
                          // 5 varrate_warp, 6 block_mma
   uint32_t* err;         // error word of the workspace (bounded waits that gave up)
+  int test_no_copies;    // test switch: the tcgen05 producer issues no tile copies
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
   double rope_f[64];
 };
@@ -85,7 +86,9 @@ struct AppendParams {
   const __nv_bfloat16* k_new;
   const __nv_bfloat16* v_new;
   int n_new;
-  int pos[kMaxBatch];
+  const int* pos;              // device [B]: slot of each row's first new token
+  const uint8_t* new_ranks;    // device [2, B, n_new] (VARRATE)
+  uint32_t* status;            // optional device word for skipped tokens (KVC_DEV_*)
   uint8_t* lk_w;
   __half* lksz_w;
   uint8_t* lv_w;
@@ -98,6 +101,8 @@ struct AppendParams {
   __nv_bfloat16* vd_w;
   int* off_k_w;
   int* off_v_w;
+  uint8_t* rank_k_w;
+  uint8_t* rank_v_w;
 };
 
 // tensor-core decode of pre-RoPE INT4 low-rank caches; every CTA writes one
@@ -153,5 +158,9 @@ __host__ __device__ inline bool needs_qproj(const Params& p) {
   return p.kind == KVC_VARRATE || p.kind == KVC_BLOCK_SHARED ||
          (p.kind == KVC_LOWRANK && !p.rope);
 }
+
+// Whether the chosen split kernel has bounded waits that can set the
+// workspace error word (the call zeroes the word first only then).
+__host__ __device__ inline bool path_sets_error_word(const Params& p) { return p.path == 1; }
 
 }  // namespace kvc

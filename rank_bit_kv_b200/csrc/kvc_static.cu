@@ -55,10 +55,21 @@ extern "C" kvc_status kvc_decode_attn_static(const kvc_layout* layout, const kvc
   void* ws = nullptr;
   kvc_status st = scratch_of_current_device(&ws);
   if (st != KVC_OK) return st;
-  // the array keeps the previous call's contents: the error word starts at zero
-  cudaError_t e = cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream);
-  if (e != cudaSuccess)
-    return kvc::report_error(KVC_ECUDA, "clearing the scratch error word: %s",
-                             cudaGetErrorString(e));
+  // Every other check, and the zeroing of the error word where the chosen
+  // kernel can set it, happens inside kvc_decode_attn before it enqueues
+  // anything, so a call that fails launches nothing.
   return kvc_decode_attn(layout, cache, q, out, ws, kScratchBytes, stream);
+}
+
+extern "C" kvc_status kvc_static_error_word(uint32_t* dst, void* stream) {
+  if (!dst) return kvc::report_error(KVC_EINVAL, "kvc_static_error_word: NULL dst");
+  void* ws = nullptr;
+  kvc_status st = scratch_of_current_device(&ws);
+  if (st != KVC_OK) return st;
+  cudaError_t e = cudaMemcpyAsync(dst, ws, sizeof(uint32_t), cudaMemcpyDefault,
+                                  (cudaStream_t)stream);
+  if (e != cudaSuccess)
+    return kvc::report_error(KVC_ECUDA, "copying the scratch error word: %s",
+                             cudaGetErrorString(e));
+  return KVC_OK;
 }

@@ -37,7 +37,17 @@ class CacheDesc(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in BUFS[:15]] + [
         ("offset_k", C.c_void_p), ("offset_v", C.c_void_p), ("rank_k", C.c_void_p),
         ("rank_v", C.c_void_p), ("seq_lens", C.c_void_p), ("n_tokens", C.c_int32),
-        ("_reserved", C.c_int32)]
+        ("_reserved", C.c_int32), ("status", C.c_void_p)]
+
+# bits of the device-side status words (include/kvc.h, KVC_DEV_*)
+DEV_WAIT_TIMEOUT, DEV_BAD_POS, DEV_BAD_RANK, DEV_BAD_PAGE, DEV_BAD_OFFSET = 1, 2, 4, 8, 16
+
+
+class RankBits(C.Structure):
+    _fields_ = [("rank", C.c_int32), ("bits", C.c_int32)]
+
+
+MAX_RESID_BITS = 8   # KVC_MAX_RESID_BITS
 
 
 class KvcError(RuntimeError):
@@ -69,8 +79,7 @@ def lib():
         L.kvc_workspace_bytes.restype = sz
         L.kvc_decode_launches.argtypes = [vp, i32]
         L.kvc_decode_launches.restype = i32
-        L.kvc_append.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, C.POINTER(i32), i32,
-                                 C.POINTER(C.c_uint8), vp]
+        L.kvc_append.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, vp, i32, vp, vp]
         L.kvc_append.restype = C.c_int
         L.kvc_decode_attn.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, vp, sz, vp]
         L.kvc_decode_attn.restype = C.c_int
@@ -78,6 +87,17 @@ def lib():
         L.kvc_decode_attn_timed.restype = C.c_int
         L.kvc_decode_attn_static.argtypes = [vp, C.POINTER(CacheDesc), vp, vp, vp]
         L.kvc_decode_attn_static.restype = C.c_int
+        L.kvc_static_error_word.argtypes = [vp, vp]
+        L.kvc_static_error_word.restype = C.c_int
+        dp = C.POINTER(C.c_double)
+        L.kvc_rank_bit_tables.argtypes = [i32, i32, dp, C.POINTER(C.c_int64), C.POINTER(i32), i32,
+                                          C.POINTER(RankBits), i32, i32, i32, C.c_double, dp, dp,
+                                          dp]
+        L.kvc_rank_bit_tables.restype = C.c_int
+        L.kvc_allocate_rank_bits.argtypes = [i32, i32, dp, dp, C.c_double, C.POINTER(i32), dp]
+        L.kvc_allocate_rank_bits.restype = C.c_int
+        L.kvc_test_skip_tile_copies.argtypes = [i32]
+        L.kvc_test_skip_tile_copies.restype = None
         L.kvc_last_error.argtypes = []
         L.kvc_last_error.restype = C.c_char_p
         L.kvc_version.argtypes = []
@@ -174,6 +194,7 @@ class Cache:
                 self.bufs[name] = torch.zeros(int(nbytes), dtype=torch.uint8, device=device)
         self.n_tokens = 0
         self.seq_lens = None
+        self.status = None        # optional device int32 [1] for append's KVC_DEV_* bits
         if fill:
             self.upload(fill)
 
@@ -198,6 +219,7 @@ class Cache:
             setattr(c, name, t.data_ptr())
         c.seq_lens = None if self.seq_lens is None else self.seq_lens.data_ptr()
         c.n_tokens = int(self.n_tokens)
+        c.status = None if self.status is None else self.status.data_ptr()
         return c
 
 
@@ -269,15 +291,76 @@ def decode_static(layout: Layout, cache: Cache, q, out, stream=None):
     check(lib().kvc_decode_attn_static(layout.h, C.byref(cs), _ptr(q), _ptr(out), st))
 
 
+def static_error_word(dst, stream=None):
+    """kvc_static_error_word: enqueue a copy of the built-in scratch area's
+    error word into dst (a torch int32 tensor on the device or in pinned host
+    memory)."""
+    st = stream if stream is not None else current_stream_ptr()
+    check(lib().kvc_static_error_word(_ptr(dst), st))
+
+
+def _device_array(x, dtype, device):
+    """x as a device tensor (torch tensors on the device pass through)."""
+    import torch
+
+    if isinstance(x, torch.Tensor) and x.is_cuda:
+        return x
+    return torch.as_tensor(np.ascontiguousarray(np.asarray(x, dtype=dtype))).to(device)
+
+
 def append(layout: Layout, cache: Cache, k_new, v_new, pos, n_new, new_ranks=None,
            stream=None):
-    """kvc_append: k_new / v_new torch bf16 device tensors, pos host ints [B]."""
+    """kvc_append: k_new / v_new torch bf16 device tensors; pos [B] and the
+    VARRATE ranks [2, B, n_new] as device tensors (host sequences are copied to
+    the device first)."""
+    dev = k_new.device
+    pos_d = _device_array(pos, np.int32, dev)
+    nr_d = None if new_ranks is None else _device_array(new_ranks, np.uint8, dev)
     cs = cache.struct()
-    posa = (C.c_int32 * len(pos))(*[int(x) for x in pos])
-    rk = None
-    if new_ranks is not None:
-        nr = np.ascontiguousarray(np.asarray(new_ranks, dtype=np.uint8))
-        rk = nr.ctypes.data_as(C.POINTER(C.c_uint8))
     st = stream if stream is not None else current_stream_ptr()
-    check(lib().kvc_append(layout.h, C.byref(cs), _ptr(k_new), _ptr(v_new), posa, int(n_new),
-                           rk, st))
+    check(lib().kvc_append(layout.h, C.byref(cs), _ptr(k_new), _ptr(v_new), _ptr(pos_d),
+                           int(n_new), _ptr(nr_d), st))
+    # keep the marshalled arrays alive until the stream has used them
+    cache._append_args = (pos_d, nr_d)
+
+
+# --------------------------------------------------------------------------- rank / bit allocation
+
+
+def _dbl(a):
+    a = np.ascontiguousarray(np.asarray(a, np.float64))
+    return a, a.ctypes.data_as(C.POINTER(C.c_double))
+
+
+def rank_bit_tables(spectra, rows, heads, options, head_dim, eta_latent, eta_resid,
+                    latent_bits=4, group=32):
+    """kvc_rank_bit_tables: (bytes, distortion) numpy [cells, options].
+    options: sequence of (rank, bits); eta_resid: dict bits -> factor."""
+    spectra, sp = _dbl(spectra)
+    n_cells, spec_len = spectra.shape
+    rows_a = np.ascontiguousarray(np.asarray(rows, np.int64))
+    heads_a = np.ascontiguousarray(np.asarray(heads, np.int32))
+    opts = (RankBits * len(options))(*[RankBits(int(r), int(b)) for r, b in options])
+    eta = np.zeros(MAX_RESID_BITS + 1)
+    for b, v in eta_resid.items():
+        eta[int(b)] = v
+    eta, ep = _dbl(eta)
+    B = np.zeros((n_cells, len(options)))
+    D = np.zeros((n_cells, len(options)))
+    check(lib().kvc_rank_bit_tables(
+        n_cells, spec_len, sp, rows_a.ctypes.data_as(C.POINTER(C.c_int64)),
+        heads_a.ctypes.data_as(C.POINTER(C.c_int32)), len(options), opts, int(head_dim),
+        int(latent_bits), int(group), float(eta_latent), ep,
+        B.ctypes.data_as(C.POINTER(C.c_double)), D.ctypes.data_as(C.POINTER(C.c_double))))
+    return B, D
+
+
+def allocate_rank_bits(bytes_, distortion, budget):
+    """kvc_allocate_rank_bits: (choice [cells] int, lambda)."""
+    B, bp = _dbl(bytes_)
+    D, dp = _dbl(distortion)
+    n_cells, n_opt = B.shape
+    ch = (C.c_int32 * n_cells)()
+    lam = C.c_double()
+    check(lib().kvc_allocate_rank_bits(n_cells, n_opt, bp, dp, float(budget), ch, C.byref(lam)))
+    return np.array(list(ch), np.int64), lam.value

@@ -35,8 +35,9 @@ def test_exports_every_declared_symbol(lib):
 
 def test_struct_sizes_match_header(lib):
     # kvc_layout_desc: 17 int32 + float + double = 80 bytes; kvc_cache: 20 pointers + 2 int32
+    # + the status pointer
     assert C.sizeof(kvc.LayoutDesc) == 80
-    assert C.sizeof(kvc.CacheDesc) == 20 * 8 + 8
+    assert C.sizeof(kvc.CacheDesc) == 20 * 8 + 8 + 8
 
 
 @pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5"])
@@ -141,30 +142,65 @@ def test_decode_host_errors_launch_nothing(lib):
 
 
 def test_append_host_errors(lib):
+    """kvc_append takes pos (and the VARRATE ranks) as device arrays: the host
+    checks pointers, alignment and sizes and returns before any CUDA call;
+    the values themselves are the kernels' to check (tested on the GPU)."""
     lay, c = _layout_c2()
     cs = kvc.CacheDesc()
-    fake = 0x10000
+    fake = 0x10000                   # 16-byte aligned, never dereferenced
     for n in ("lk_codes", "lk_sz", "lv_codes", "lv_sz", "bk", "bv"):
         setattr(cs, n, fake)
-    pos = (C.c_int32 * 2)(60, 0)
-    st = lib.kvc_append(lay.h, C.byref(cs), C.c_void_p(fake), C.c_void_p(fake), pos, 5, None, None)
-    assert kvc.STATUS[st] == "KVC_ECAPACITY"
-    pos = (C.c_int32 * 2)(-1, 0)
-    st = lib.kvc_append(lay.h, C.byref(cs), C.c_void_p(fake), C.c_void_p(fake), pos, 1, None, None)
-    assert kvc.STATUS[st] == "KVC_ECAPACITY"
-    st = lib.kvc_append(lay.h, C.byref(cs), C.c_void_p(fake), C.c_void_p(fake), pos, 0, None, None)
-    assert kvc.STATUS[st] == "KVC_EINVAL"
-    # VARRATE rank outside {4, 8, 16, 32, 64}
+    f = C.c_void_p(fake)
+    st = lib.kvc_append(lay.h, C.byref(cs), f, f, None, 1, None, None)
+    assert kvc.STATUS[st] == "KVC_EINVAL"                   # NULL pos
+    st = lib.kvc_append(lay.h, C.byref(cs), f, f, C.c_void_p(fake + 4), 1, None, None)
+    assert kvc.STATUS[st] == "KVC_EALIGN"                   # pos not 16-byte aligned
+    st = lib.kvc_append(lay.h, C.byref(cs), f, f, f, 65, None, None)
+    assert kvc.STATUS[st] == "KVC_ECAPACITY"                # n_new > max_tokens (64)
+    st = lib.kvc_append(lay.h, C.byref(cs), f, f, f, 0, None, None)
+    assert kvc.STATUS[st] == "KVC_EINVAL"                   # n_new < 1
+    st = lib.kvc_append(lay.h, C.byref(cs), f, None, f, 1, None, None)
+    assert kvc.STATUS[st] == "KVC_EINVAL"                   # v_new NULL
+    cs.status = fake + 2
+    st = lib.kvc_append(lay.h, C.byref(cs), f, f, f, 1, None, None)
+    assert kvc.STATUS[st] == "KVC_EALIGN" and b"status" in lib.kvc_last_error()
+    cs.status = None
+    cs.lk_sz = None
+    st = lib.kvc_append(lay.h, C.byref(cs), f, f, f, 1, None, None)
+    assert kvc.STATUS[st] == "KVC_EINVAL" and b"lk_sz" in lib.kvc_last_error()
+    # VARRATE: the ranks are required and must be aligned
     c4 = synth.config("c4", T=16)
     lay4 = kvc.Layout(kvc.desc_from_config(c4))
     cs4 = kvc.CacheDesc()
     for n in ("lk_codes", "lv_codes", "offset_k", "offset_v", "rank_k", "rank_v", "bk", "bv"):
         setattr(cs4, n, fake)
-    ranks = np.array([[[4]], [[12]]], dtype=np.uint8)
-    pos1 = (C.c_int32 * 1)(0)
-    st = lib.kvc_append(lay4.h, C.byref(cs4), C.c_void_p(fake), C.c_void_p(fake), pos1, 1,
-                        ranks.ctypes.data_as(C.POINTER(C.c_uint8)), None)
-    assert kvc.STATUS[st] == "KVC_EINVAL" and b"rank 12" in lib.kvc_last_error()
+    st = lib.kvc_append(lay4.h, C.byref(cs4), f, f, f, 1, None, None)
+    assert kvc.STATUS[st] == "KVC_EINVAL" and b"new_ranks" in lib.kvc_last_error()
+    st = lib.kvc_append(lay4.h, C.byref(cs4), f, f, f, 1, C.c_void_p(fake + 1), None)
+    assert kvc.STATUS[st] == "KVC_EALIGN"
+
+
+def test_static_entry_points_validate_before_enqueueing(lib):
+    """The workspace-free decode refuses bad calls without touching the GPU:
+    its scratch lookup and every enqueue come after the host checks."""
+    lay, c = _layout_c2()
+    cs = kvc.CacheDesc()
+    st = lib.kvc_decode_attn_static(None, C.byref(cs), None, None, None)
+    assert kvc.STATUS[st] == "KVC_EINVAL"
+    st = lib.kvc_static_error_word(None, None)
+    assert kvc.STATUS[st] == "KVC_EINVAL"
+
+
+def test_header_cites_a_passage_beside_each_operation():
+    """Each entry point that computes part of the method names the page and
+    section that define it in its own comment."""
+    src = open(os.path.join(ROOT, "include", "kvc.h")).read()
+    for fn in ("kvc_create_layout", "kvc_append", "kvc_decode_attn", "kvc_buffer_sizes",
+               "kvc_step_bytes"):
+        i = re.search(rf"^[\w ]+\*?\s*\b{fn}\(", src, re.M).start()   # the declaration
+        j = src.rindex("/*", 0, i)
+        comment = src[j:i]
+        assert re.search(r'"[^"]+"', comment), fn          # a quoted page or section title
 
 
 def test_library_has_no_oracle_dependency():

@@ -203,8 +203,11 @@ def test_residual_off_equals_plain_lowrank():
 
 def test_int4_asym_matches_page_formula_on_fp16_exact_groups():
     """When lo and (hi-lo)/15 are already fp16 values the codes and the
-    dequantized values are exactly the worked example's
-    round((v - lo) / s) * s + lo with Python's round."""
+    dequantized values are exactly the worked example's rule (BellowsKV page,
+    "Worked Example: Why the Latent Quantizes Flat"): the nearest of the
+    fifteen equal steps above the minimum, ties to the even step -- evaluated
+    here in exact rational arithmetic, independently of the oracle's floats."""
+    from fractions import Fraction
     rng = np.random.default_rng(14)
     for _ in range(200):
         lo = float(np.float16(rng.uniform(-3, 0)))
@@ -215,7 +218,8 @@ def test_int4_asym_matches_page_formula_on_fp16_exact_groups():
         x = np.concatenate([[lo, hi], rng.uniform(lo, hi, 30)])
         codes, sc, zc = O.quantize_int4_asym(x, 32)
         assert sc[0] == s and zc[0] == lo
-        page = [round((v - lo) / s) * s + lo for v in x]          # the printed rule
+        steps = [round(Fraction(v) / Fraction(s) - Fraction(lo) / Fraction(s)) for v in x]
+        page = [float(Fraction(lo) + k * Fraction(s)) for k in steps]
         np.testing.assert_array_equal(codes * s + lo, page)
         np.testing.assert_array_equal(O.dequant_int4_asym(codes, sc, zc, 32), page)
         assert codes[0] == 0 and codes[1] == 15

@@ -34,8 +34,10 @@ def _setup(cfg):
 
 
 @pytest.mark.parametrize("name,over", [
-    ("c2", {}),                                  # Llama-8B layer, 32K context (tensor-core path)
-    ("c5", {"B": 2, "T": 1000}),                 # paged, rotated residual (generic path)
+    ("c2", {}),                     # Llama-8B layer, 32K context: warp-level pre-RoPE kernel
+    ("c2", {"B": 2, "T": 1000}),    # capacity not a multiple of 16: tcgen05 pre-RoPE kernel,
+                                    # the one whose bounded waits use the error word
+    ("c5", {"B": 2, "T": 1000}),    # paged, rotated residual: warp-level latent-space kernel
 ])
 def test_static_scratch_decode_matches_workspace_decode(name, over):
     cfg = synth.config(name, **over)
@@ -46,11 +48,14 @@ def test_static_scratch_decode_matches_workspace_decode(name, over):
     kvc.decode(lay, cache, q, ref, ws)
     torch.cuda.synchronize()
     ref = ref.cpu().numpy()
+    word = torch.full((4,), -1, dtype=torch.int32, device="cuda")
     for call in range(2):
         out = torch.full(q.shape, float("nan"), device="cuda")
         kvc.decode_static(lay, cache, q, out)
+        kvc.static_error_word(word)
         torch.cuda.synchronize()
         assert_close(out.cpu().numpy(), ref, MAX_ABS, REL_L2, what=f"{name} static call {call}")
+        assert int(word[0].item()) == 0, "the built-in scratch area reports an aborted wait"
 
 
 def test_static_scratch_refuses_layouts_beyond_its_size():
