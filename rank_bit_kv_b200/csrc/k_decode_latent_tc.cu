@@ -126,6 +126,17 @@ __device__ __forceinline__ uint32_t field2(uint32_t x, uint32_t x6, int mu) {
 }
 constexpr uint32_t kN0 = 0x000F000Fu;    // nibble 0 of both halves (eps 1)
 constexpr uint32_t kN1 = 0x00F000F0u;    // nibble 1 of both halves (eps 16)
+// Code centring, exact in f16 subnormals: an INT4 value operand c * eps * 2^-24
+// becomes (c - 8) * eps * 2^-24.  The long fp32 MMA accumulations then hold sums
+// near the result instead of a large common part that the zero terms cancel
+// afterwards, so the rounding of the tensor-core accumulation (which is not
+// round-to-nearest) is not amplified.  (The 2-bit residual values, a tenth of
+// the latent's in size, keep their plain codes.)
+constexpr uint32_t kC0 = 0x00080008u;    // 8 * 2^-24 in both halves (eps 1)
+constexpr uint32_t kC1 = 0x00800080u;    // 8 * 16 * 2^-24 (eps 16)
+__device__ __forceinline__ uint32_t hsub_u32(uint32_t x, uint32_t c) {
+  return h2u(__hsub2(*reinterpret_cast<__half2*>(&x), *reinterpret_cast<__half2*>(&c)));
+}
 
 template <int RV, bool RES>
 __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork wk) {
@@ -471,7 +482,11 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         if (!ok0) sz_0 = __float2half2_rn(0.f);
         if (!ok1) sz_1 = __float2half2_rn(0.f);
       }
-      const __half2 zt = __hfma2(hp23, __high2half2(sz_1), __hmul2(hp01, __high2half2(sz_0)));
+      // zero term of the centred codes: p * (z + 8 s)
+      const __half2 k8 = __float2half2_rn(8.f);
+      const __half2 zc0 = __hfma2(__low2half2(sz_0), k8, __high2half2(sz_0));
+      const __half2 zc1 = __hfma2(__low2half2(sz_1), k8, __high2half2(sz_1));
+      const __half2 zt = __hfma2(hp23, zc1, __hmul2(hp01, zc0));
       const float2 ztf = __half22float2(zt);
       zs[v][0] += ztf.x;
       zs[v][1] += ztf.y;
@@ -483,12 +498,14 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
       const uint32_t xA = prmt(lds32(lv), lds32(lv + 4 * RVB), sel);
       const uint32_t xB = prmt(lds32(lv + 8 * RVB), lds32(lv + 12 * RVB), sel);
       {
-        const uint32_t a[4] = {xA & kN0, xA & kN1, xB & kN0, xB & kN1};
+        const uint32_t a[4] = {hsub_u32(xA & kN0, kC0), hsub_u32(xA & kN1, kC1),
+                               hsub_u32(xB & kN0, kC0), hsub_u32(xB & kN1, kC1)};
         mma16816(accV[2 * v], a, b0, b1);
       }
       if (!half) {
         const uint32_t yA = xA >> 8, yB = xB >> 8;
-        const uint32_t a[4] = {yA & kN0, yA & kN1, yB & kN0, yB & kN1};
+        const uint32_t a[4] = {hsub_u32(yA & kN0, kC0), hsub_u32(yA & kN1, kC1),
+                               hsub_u32(yB & kN0, kC0), hsub_u32(yB & kN1, kC1)};
         mma16816(accV[2 * v + 1], a, b0, b1);
       }
     }
@@ -500,9 +517,10 @@ __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork
         if (!ok1) rs_1 = __float2half2_rn(0.f);
       }
       const __half2 q01 = __hmul2(hp01, rs_0), q23 = __hmul2(hp23, rs_1);
-      const float2 qs = __half22float2(__hadd2(q01, q23));
-      sR[0] += qs.x;
-      sR[1] += qs.y;
+      // the sum of the very operands the MMA uses, in fp32
+      const float2 qa = __half22float2(q01), qb = __half22float2(q23);
+      sR[0] += qa.x + qb.x;
+      sR[1] += qa.y + qb.y;
       const uint32_t b0 = movmatrix_trans(h2u(q01));
       const uint32_t b1 = movmatrix_trans(h2u(q23));
       const uint32_t wA0 = lds32(st + o_rv), wA1 = lds32(st + o_rv + 128);

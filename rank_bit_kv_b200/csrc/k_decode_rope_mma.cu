@@ -4,8 +4,8 @@
 // per tile:
 //   - dequantises the key latents into f16 operands (x = c s + z per token and
 //     group) and reconstructs K = L Bk with mma.sync m16n8k16 (M = 16 tokens,
-//     N = 128 dims, K = the rank; f16 accumulate), the Bk fragments read from
-//     shared memory with ldmatrix.trans;
+//     N = 128 dims, K = the rank; fp32 accumulate, each sum rounded to f16
+//     once), the Bk fragments read from shared memory with ldmatrix.trans;
 //   - applies the rotation of the token's position inside its group of 128 (or
 //     64) tokens,
 //     R_delta, in f16x2 (cos / sin of delta * omega_i from a per-CTA table);
@@ -92,16 +92,6 @@ __device__ __forceinline__ uint32_t lds32(const uint8_t* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
-// D (f16x2 x 2) += A B, f16 accumulate
-__device__ __forceinline__ void mma_f16acc(uint32_t (&d)[2], const uint32_t (&a)[4], uint32_t b0,
-                                           uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f16.f16.f16.f16 {%0,%1}, {%2,%3,%4,%5}, {%6,%7}, "
-      "{%0,%1};"
-      : "+r"(d[0]), "+r"(d[1])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -119,6 +109,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 constexpr uint32_t kN0 = 0x000F000Fu;    // nibble 0 of both halves
 constexpr uint32_t kN1 = 0x00F000F0u;    // nibble 1 of both halves (x 16)
 constexpr uint32_t kMagic = 0x64006400u; // f16 1024 in both halves
+// Value codes enter the MMA centred, (c - 8) * eps * 2^-24 (exact in f16
+// subnormals), so the long fp32 accumulation holds a sum near the result rather
+// than a large common part that the zero term cancels afterwards.
+constexpr uint32_t kC0 = 0x00080008u;    // 8 * 2^-24 in both halves (eps 1)
+constexpr uint32_t kC1 = 0x00800080u;    // 8 * 16 * 2^-24 (eps 16)
 
 // Rank held by k-slot kappa (0..15) of k-step ks of the reconstruction MMA:
 // thread c4 turns word c4 of a latent row (ranks 8 c4 .. 8 c4 + 7) into its
@@ -360,34 +355,37 @@ __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork 
         a[ks][3] = deq(x1 >> 4, s1, z1);
       }
     }
-    // reconstruction K = L Bk: 16 n-tiles of 8 dims, f16 accumulate
+    // reconstruction K = L Bk (16 n-tiles of 8 dims) with fp32 accumulators,
+    // one RoPE pair of n-tile couples at a time: n-tiles 2m, 2m + 1 hold dims
+    // i and n-tiles 2m + 8, 2m + 9 dims i + 64.  Each sum is rounded to f16 once,
+    // then R_delta rotates the pair (rows g and g + 8) in f16x2.
     uint32_t kf[16][2];
     const uint32_t bk_s = sm_s + kvh * kBkHead + ldsm_off;
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) kf[nt][0] = kf[nt][1] = 0u;
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {
-        uint32_t b[4];
-        ldsm_x4_trans(b, bk_s + ks * 16 * kBkRow + np * 32);
-        mma_f16acc(kf[2 * np], a[ks], b[0], b[1]);
-        mma_f16acc(kf[2 * np + 1], a[ks], b[2], b[3]);
-      }
-    }
-    // R_delta on pairs (i, i + 64): n-tiles nt and nt + 8, rows g and g + 8
     const int dl0 = (kPT * jt) % L::GROUP + g;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const uint32_t tab = rope_s + (dl0 + 8 * r) * kRopeRow;
+    for (int m = 0; m < 4; ++m) {
+      float c[4][4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const uint4 t = lds128(tab + 64 * m);
+      for (int x = 0; x < 4; ++x) c[x][0] = c[x][1] = c[x][2] = c[x][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        uint32_t b[4];
+        ldsm_x4_trans(b, bk_s + ks * 16 * kBkRow + m * 32);
+        mma16816(c[0], a[ks], b[0], b[1]);
+        mma16816(c[1], a[ks], b[2], b[3]);
+        ldsm_x4_trans(b, bk_s + ks * 16 * kBkRow + (m + 4) * 32);
+        mma16816(c[2], a[ks], b[0], b[1]);
+        mma16816(c[3], a[ks], b[2], b[3]);
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const uint4 t = lds128(rope_s + (dl0 + 8 * r) * kRopeRow + 64 * m);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int nt = 2 * m + h;
           const __half2 cs = u2h2(h ? t.z : t.x), sn = u2h2(h ? t.w : t.y);
-          const __half2 lo = u2h2(kf[nt][r]), hi = u2h2(kf[nt + 8][r]);
+          const __half2 lo = __floats2half2_rn(c[h][2 * r], c[h][2 * r + 1]);
+          const __half2 hi = __floats2half2_rn(c[2 + h][2 * r], c[2 + h][2 * r + 1]);
           kf[nt][r] = h2u(__hfma2(lo, cs, __hneg2(__hmul2(hi, sn))));
           kf[nt + 8][r] = h2u(__hfma2(hi, cs, __hmul2(lo, sn)));
         }
@@ -456,7 +454,11 @@ __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork 
         if (!ok0) sz_0 = __float2half2_rn(0.f);
         if (!ok1) sz_1 = __float2half2_rn(0.f);
       }
-      const __half2 zt = __hfma2(hp23, __high2half2(sz_1), __hmul2(hp01, __high2half2(sz_0)));
+      // zero term of the centred codes: p * (z + 8 s)
+      const __half2 k8 = __float2half2_rn(8.f);
+      const __half2 zc0 = __hfma2(__low2half2(sz_0), k8, __high2half2(sz_0));
+      const __half2 zc1 = __hfma2(__low2half2(sz_1), k8, __high2half2(sz_1));
+      const __half2 zt = __hfma2(hp23, zc1, __hmul2(hp01, zc0));
       const float2 ztf = __half22float2(zt);
       zs[v][0] += ztf.x;
       zs[v][1] += ztf.y;
@@ -467,13 +469,16 @@ __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork 
       const uint32_t sel = half ? sel_h : sel_v;
       const uint32_t xA = prmt(lds32(lv), lds32(lv + RVB), sel);
       const uint32_t xB = prmt(lds32(lv + 8 * RVB), lds32(lv + 9 * RVB), sel);
+      auto cen = [](uint32_t x, uint32_t c) { return h2u(__hsub2(u2h2(x), u2h2(c))); };
       {
-        const uint32_t av[4] = {xA & kN0, xA & kN1, xB & kN0, xB & kN1};
+        const uint32_t av[4] = {cen(xA & kN0, kC0), cen(xA & kN1, kC1), cen(xB & kN0, kC0),
+                                cen(xB & kN1, kC1)};
         mma16816(accV[2 * v], av, b0, b1);
       }
       if (!half) {
         const uint32_t yA = xA >> 8, yB = xB >> 8;
-        const uint32_t av[4] = {yA & kN0, yA & kN1, yB & kN0, yB & kN1};
+        const uint32_t av[4] = {cen(yA & kN0, kC0), cen(yA & kN1, kC1), cen(yB & kN0, kC0),
+                                cen(yB & kN1, kC1)};
         mma16816(accV[2 * v + 1], av, b0, b1);
       }
     }

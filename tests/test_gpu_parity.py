@@ -171,35 +171,50 @@ def test_per_row_lengths():
 
 
 def test_bf16_output():
+    """bf16 output is held to the same tolerance as fp32 output: the combine
+    rounds once, from fp32, after the division by the softmax sum."""
     c = synth.config("c2", B=1, T=500)
     a = synth.lowrank_cache(c)
     got = run_decode(c, a, 500, out_bf16=1)
     ref = oracle(c, a, 500)
-    # bf16 output rounding adds up to 2^-9 relative per element
-    assert_close(got, ref, max_abs=1e-2, rel_l2=5e-3, what="bf16 out")
+    assert_close(got, ref, what="bf16 out")
+
+
+def test_bf16_output_full_size_c2():
+    """bf16 output on the benchmark workload (all 8 rows) within the stated
+    tolerance."""
+    from tests import full_size as F
+
+    ex, futs = F.submit_rows("c2", "uniform", list(range(8)))
+    c, a = F.build_arrays("c2", "uniform")
+    got = run_decode(c, a, c["T"], out_bf16=1)
+    rows = F.collect(ex, futs)
+    ref = np.stack([rows[b] for b in range(c["B"])])
+    assert_close(got, ref, what="c2 full bf16 out")
 
 
 # ------------------------------------------------------------------ full-size workloads
 
 
-def test_c2_full_size_sampled():
-    c = synth.config("c2")
-    a = synth.lowrank_cache(c)
-    got = run_decode(c, a, c["T"])
-    for b in (0, 5):
-        sub = sub_batch(a, [b], ("q", "lk_codes", "lk_sz", "lv_codes", "lv_sz"))
-        assert_close(got[b:b + 1], oracle(dict(c, B=1), sub, c["T"]), what=f"c2 full b={b}")
+@pytest.mark.parametrize("variant", ["uniform", "gaussian"])
+@pytest.mark.parametrize("name", ["c2", "c5"])
+def test_full_size_every_row(name, variant):
+    """The full workloads in the launch configuration the benchmark times,
+    every batch row compared with the oracle.  The warp-level kernels cut
+    equal byte ranges across (row, KV head) units, so a unit boundary can fall
+    inside any warp's range: every row is checked, not a sample.  `gaussian`
+    uses codes quantized from N(0,1) latents, as the configurations state."""
+    from tests import full_size as F
 
-
-def test_c5_full_size_sampled():
-    c = synth.config("c5")
-    a = synth.lowrank_cache(c)
+    c0 = synth.config(name)
+    ex, futs = F.submit_rows(name, variant, list(range(c0["B"])))   # oracle overlaps the GPU
+    c, a = F.build_arrays(name, variant)
     got = run_decode(c, a, c["T"])
-    for b in (3,):
-        sub = dict(a)
-        sub["q"] = a["q"][[b]]
-        sub["page_table"] = a["page_table"][[b]]
-        assert_close(got[b:b + 1], oracle(dict(c, B=1), sub, c["T"]), what=f"c5 full b={b}")
+    rows = F.collect(ex, futs)
+    for b in range(c["B"]):
+        assert_close(got[b:b + 1], rows[b][None], what=f"{name} {variant} full b={b}")
+    ref = np.stack([rows[b] for b in range(c["B"])])
+    assert_close(got, ref, what=f"{name} {variant} full, all rows")
 
 
 def test_c4_full_size():
