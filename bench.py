@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-others", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -60,11 +61,13 @@ def parse():
 
 
 def measured_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, which): the driver's measured peaks, else
+    the fallback figures of earlier measurements on this hardware."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
 
 
 def profiled_traffic(version):
@@ -183,7 +186,87 @@ def dense_step(torch, kvc, synth, device, steps, warmup):
     return {"us_per_step": round(us, 2), "bytes_per_step": byts, "GB/s": round(byts / us / 1e3, 1)}
 
 
+OTHER_WORKLOADS = {
+    "c3": "block-shared latent, 4 layers x 32 q heads, latent 512 INT4/g64 sym, B=4, T=65536",
+    "c4": "variable rank per token {4..64}, ragged INT4 records, B=1, T=131072",
+    "c5": "low rank K32/V64 INT4 + 2-bit rotated residual, 16-token pages, B=16, T=65536, "
+          "one kvc_append of a new token per step then decode",
+}
+
+
+def other_workloads(torch, kvc, synth, device, steps, peak_gbs, peak_tflops):
+    """The other configured workloads, each timed the same way: a 512 MiB
+    write flushes L2 before every step, CUDA events around the step (for C5
+    the append of one new token at slot T-1 of every row, then the decode) and,
+    recorded by the library, around the split-T kernel; medians over the
+    steps."""
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    n = max(5, min(steps, 20))
+    res = {}
+    for name, what in OTHER_WORKLOADS.items():
+        c = synth.config(name)
+        lay = kvc.Layout(kvc.desc_from_config(c))
+        fill = (synth.block_shared_cache(c) if name == "c3" else
+                synth.varrate_cache(c) if name == "c4" else synth.lowrank_cache(c))
+        cache = kvc.Cache(lay, device=device, fill=fill)
+        cache.n_tokens = c["T"]
+        q = torch.from_numpy(np.ascontiguousarray(fill["q"]).view(np.int16)).to(device).view(
+            torch.bfloat16)
+        del fill
+        out = torch.empty(q.shape, device=device)
+        ws = torch.empty(lay.workspace_bytes(c["T"]), dtype=torch.uint8, device=device)
+        app = None
+        if name == "c5":
+            kn, vn = synth.new_tokens(c, 1)
+            app = (torch.from_numpy(kn.view(np.int16)).to(device).view(torch.bfloat16),
+                   torch.from_numpy(vn.view(np.int16)).to(device).view(torch.bfloat16),
+                   torch.full((c["B"],), c["T"] - 1, dtype=torch.int32, device=device))
+
+        def step(ev=None):
+            if app is not None:
+                kvc.append(lay, cache, app[0], app[1], app[2], 1)
+            kvc.decode(lay, cache, q, out, ws, events=ev)
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        evs = [(kvc.RawEvent(), kvc.RawEvent()) for _ in range(n)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        st_us, k_us = [], []
+        for i in range(n):
+            flush.fill_(i & 255)
+            e0.record()
+            step(evs[i])
+            e1.record()
+            torch.cuda.synchronize()
+            st_us.append(e0.elapsed_time(e1) * 1e3)
+            k_us.append(evs[i][0].elapsed_ms(evs[i][1]) * 1e3)
+        byts = lay.step_bytes(c["T"])
+        su, ku = statistics.median(st_us), statistics.median(k_us)
+        r = {"what": what, "steps": n, "step_us": round(su, 2), "kernel_us": round(ku, 2),
+             "bytes_per_step": byts, "step_GBps": round(byts / su / 1e3, 1),
+             "kernel_GBps": round(byts / ku / 1e3, 1),
+             "kernel_frac_of_measured_hbm": round(byts / ku / 1e3 / peak_gbs, 4),
+             "finite": bool(torch.isfinite(out).all().item()),
+             "launches_per_step": lay.decode_launches(c["T"]) + (1 if app is not None else 0)}
+        if name == "c3":
+            flops = 2 * 2 * c["L"] * c["Hq"] * c["D"] * c["T"] * c["B"]
+            r["flops_per_step"] = flops
+            r["kernel_TFLOPs"] = round(flops / ku / 1e6, 1)
+            r["kernel_frac_of_measured_bf16"] = round(flops / ku / 1e6 / peak_tflops, 4)
+            r["bound"] = "tensor"
+        else:
+            r["bound"] = "hbm"
+        res[name] = r
+        del cache, q, out, ws, app
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def _oracle_threads():
+    """BLAS threads numpy would use (the oracle's matrix products)."""
     try:
         from threadpoolctl import threadpool_info
         return max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
@@ -191,78 +274,116 @@ def _oracle_threads():
         return 1
 
 
-def _oracle_unit(a, c, b, h, n_tok):
-    """Oracle decode of one (batch row, KV head) unit over its first n_tok tokens."""
+def _cpu_model():
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.startswith("Model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def _oracle_slice(a, c, n_tok):
+    """The fp64 oracle on the whole batch (all rows and KV heads) over the first
+    n_tok tokens of every row: the workload's step on a shorter context."""
     from oracle import kvc_oracle as O
 
-    sub = {n: a[n][[b]][:, [h]] for n in ("lk_codes", "lk_sz", "lv_codes", "lv_sz")}
-    sub["q"] = a["q"][[b]][:, h * 4:(h + 1) * 4]
-    sub["bk"], sub["bv"] = a["bk"][[h]], a["bv"][[h]]
-    return O.decode_from_storage(dict(c, B=1, Hkv=1, Hq=4), sub, n_tok)
+    return O.decode_from_storage(c, a, n_tok)
 
 
-def _unit_bytes(c, n_tok):
+def _slice_bytes(c, n_tok):
     from oracle import kvc_oracle as O
 
-    return O.lowrank_bytes_per_token_head(c["rk"], c["rv"], c["bits"], c["g"]) * n_tok
+    per = O.lowrank_bytes_per_token_head(c["rk"], c["rv"], c["bits"], c["g"])
+    return per * n_tok * c["B"] * c["Hkv"]
 
 
-def cpu_oracle_rate(a, c, seconds):
-    """Time the fp64 oracle on a bounded sample of the workload: whole
-    (batch row, KV head) units at the full context, until `seconds` elapse."""
+def _sized_slice(a, c, seconds):
+    """Tokens per row such that one whole-batch oracle call takes about
+    `seconds` (calibrated on a 1024-token call), a multiple of 256."""
+    t0 = time.perf_counter()
+    _oracle_slice(a, c, 1024)
+    per_tok = (time.perf_counter() - t0) / 1024
+    n = int(seconds / max(per_tok, 1e-9)) // 256 * 256
+    return int(min(c["T"], max(256, n)))
+
+
+def _time_slices(a, c, n_tok, seconds):
     done, t0 = 0, time.perf_counter()
-    units = [(b, h) for b in range(c["B"]) for h in range(c["Hkv"])]
     while True:
-        b, h = units[done % len(units)]
-        _oracle_unit(a, c, b, h, c["T"])
+        _oracle_slice(a, c, n_tok)
         done += 1
         el = time.perf_counter() - t0
         if el >= seconds:
-            break
-    gbs = done * _unit_bytes(c, c["T"]) / el / 1e9
-    return {"value": round(gbs, 4), "unit": "GB/s", "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"{done} unit decodes cycling over the {len(units)} (batch row, KV head) units at T={c['T']} "
-                      f"({done * _unit_bytes(c, c['T'])} compressed bytes) in {el:.1f} s, "
-                      f"fp64 numpy"}
+            return done, el
+
+
+def cpu_oracle_rate(a, c, seconds):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload: the
+    whole batch (all 64 (row, KV head) units) over the first n tokens of every
+    row, repeated for about `seconds`, once with numpy's default threads and
+    once limited to one thread."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        threadpool_limits = None
+    n_tok = _sized_slice(a, c, seconds / 4)
+    done, el = _time_slices(a, c, n_tok, seconds / 2)
+    gbs = done * _slice_bytes(c, n_tok) / el / 1e9
+    one = None
+    if threadpool_limits is not None:
+        with threadpool_limits(1):
+            d1, e1 = _time_slices(a, c, n_tok, seconds / 2)
+        one = round(d1 * _slice_bytes(c, n_tok) / e1 / 1e9, 5)
+    return {"value": round(gbs, 5), "unit": "GB/s", "cores": _oracle_threads(), "kind": "oracle",
+            "value_1_core": one, "host_cpus": os.cpu_count(), "cpu_model": _cpu_model(),
+            "sample": f"{done} whole-batch oracle calls over the first {n_tok} of {c['T']} "
+                      f"tokens of all {c['B'] * c['Hkv']} (row, KV head) units "
+                      f"({_slice_bytes(c, n_tok)} compressed bytes each) in {el:.1f} s, fp64 "
+                      f"numpy; the oracle's numpy calls use up to `cores` BLAS threads, "
+                      f"value_1_core limits them to one"}
 
 
 # --------------------------------------------------------------------------- arms
 
 
 def run_reference(args, rank, world):
-    """Reference arm: the fp64 CPU oracle on the host cores (rank 0 only).
-    Each step is a bounded sample of the workload: the first n tokens of one
-    (batch row, KV head) unit, n sized so that the whole run stays near two
-    minutes; the rate is in the workload's unit (compressed GB/s)."""
+    """Reference arm: the fp64 CPU oracle, as it stands, on the host cores
+    (rank 0 only; other ranks exit without work).  Each step is the whole
+    batch -- every (batch row, KV head) unit -- over the first n tokens of
+    every row, n sized so that the --warmup + --steps calls end within about
+    three minutes (the full 32K context when the host is fast enough).
+    ms_per_step is the measured time of that call; value is its compressed
+    bytes over that time (GB/s, the workload's unit)."""
     if rank != 0:
         return
     from rank_bit_kv_b200 import synth
 
     c = synth.config(WORKLOAD)
     a = synth.lowrank_cache(c)
+    n_tok = _sized_slice(a, c, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        _oracle_slice(a, c, n_tok)
     t0 = time.perf_counter()
-    _oracle_unit(a, c, 0, 0, 4096)
-    per_tok = (time.perf_counter() - t0) / 4096
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    n_tok = int(min(c["T"], max(256, budget / per_tok)))
-    units = [(b, h) for b in range(c["B"]) for h in range(c["Hkv"])]
-    for i in range(args.warmup):
-        _oracle_unit(a, c, *units[i % len(units)], n_tok)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        _oracle_unit(a, c, *units[i % len(units)], n_tok)
+    for _ in range(args.steps):
+        _oracle_slice(a, c, n_tok)
     el = time.perf_counter() - t0
-    gbs = args.steps * _unit_bytes(c, n_tok) / el / 1e9
-    full_step = _unit_bytes(c, c["T"]) * c["B"] * c["Hkv"]
-    us = full_step / (gbs * 1e9) * 1e6
+    per_step = _slice_bytes(c, n_tok)
+    gbs = args.steps * per_step / el / 1e9
+    ms = el / args.steps * 1e3
     cb = {"value": round(gbs, 5), "unit": "GB/s", "cores": _oracle_threads(), "kind": "oracle",
-          "sample": f"per step: first {n_tok} of {c['T']} tokens of one (batch row, KV head) "
-                    f"unit ({_unit_bytes(c, n_tok)} compressed bytes), fp64 numpy"}
+          "host_cpus": os.cpu_count(), "cpu_model": _cpu_model(),
+          "sample": f"per step: all {c['B'] * c['Hkv']} (row, KV head) units over the first "
+                    f"{n_tok} of {c['T']} tokens of every row ({per_step} compressed bytes), "
+                    f"fp64 numpy"}
     line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 5), "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(us / 1e3, 3), "us_per_step": round(us, 1),
+            "ms_per_step": round(ms, 3), "us_per_step": round(ms * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(c, "n/a (host)"),
+            "data": "synthetic", "config": workload_config(c),
+            "tokens_per_row_per_step": n_tok, "bytes_per_step": per_step,
             "cpu_baseline": cb,
             "e2e": {"value": round(gbs, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -284,11 +405,13 @@ def job_rate(world, step_bytes, steps, ms):
     return world * step_bytes * steps / (ms / 1e3) / 1e9
 
 
-def workload_config(c, l2):
+def workload_config(c):
     return {"workload": WORKLOAD_NAME, "batch": c["B"], "q_heads": c["Hq"], "kv_heads": c["Hkv"],
             "head_dim": c["d"], "context": c["T"], "rank_k": c["rk"], "rank_v": c["rv"],
             "latent_bits": c["bits"], "group": c["g"], "rope_theta": c["theta"],
-            "keys": "pre-RoPE", "l2": l2}
+            "keys": "pre-RoPE",
+            "l2": "inputs larger than L2: consecutive GPU steps rotate over cache copies "
+                  "whose total exceeds the 126 MB L2"}
 
 
 def run_kvc(args, rank, world, torch, dist):
@@ -361,10 +484,14 @@ def run_kvc(args, rank, world, torch, dist):
     dense = None
     if not args.no_dense:
         dense = dense_step(torch, kvc, synth, device, K, 3)
+    others = None
+    if not args.no_others:
+        others = other_workloads(torch, kvc, synth, device, K, measured_peaks()[0],
+                                 measured_peaks()[1])
 
     if rank != 0:
         return
-    peak, peak_kind = measured_peaks()
+    peak, peak_tf, peak_kind = measured_peaks()
     achieved = step_bytes / (hot_us * 1e-6) / 1e9
     version = kvc.lib().kvc_version().decode()
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -380,11 +507,11 @@ def run_kvc(args, rank, world, torch, dist):
             "us_per_step": round(ms_per_step * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic",
-            "config": workload_config(c, f"{n} rotating cache copies of {step_bytes} B "
-                                         f"({n * step_bytes} B > 126 MiB L2)"),
+            "config": workload_config(c),
+            "cache_copies": {"n": n, "bytes_each": step_bytes, "total": n * step_bytes},
             "bytes_per_step": step_bytes, "gpu_launches": K * launches,
             "kernel_version": version, "clocks": clocks, "roofline": roof, "e2e": e2e,
-            "dense_bf16_same_step": dense, "cpu_baseline": cpu}
+            "dense_bf16_same_step": dense, "workloads": others, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
 
 
