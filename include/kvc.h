@@ -81,9 +81,15 @@ typedef enum {
  * KVC_VARRATE: rank_k = rank_v = max rank (64); per-token ranks from
  *   {4, 8, 16, 32, 64}; latent_bits = 4, group_size = 32.
  * KVC_BLOCK_SHARED: n_layers layers share one latent of latent_dim values per
- *   token, INT4 symmetric (x = (code - 8) * scale) with one fp16 scale per
- *   group_size values; per-layer fp16 up-projections W_k, W_v
- *   [n_layers, latent_dim, n_kv_heads * head_dim].
+ *   token, symmetric integer codes (x = (code - 2^(b-1)) * scale, codes from
+ *   round(x / scale) with scale = max|x| / (2^(b-1) - 1) per group) with one
+ *   fp16 scale per group_size values; latent_bits b in {4 (0 means 4), 8, 3};
+ *   value_bits 0: the one latent feeds the keys and the values of every layer;
+ *   value_bits in {2, 3, 4, 8}: a second latent at that width feeds the values
+ *   (the key latent at latent_bits feeds the keys) -- the operating points of
+ *   the BellowsKV page ("Reading the Retention Table": n = 2 with INT8, n = 4
+ *   with INT4, INT3, a 3-bit key / 2-bit value variant); per-layer fp16
+ *   up-projections W_k, W_v [n_layers, latent_dim, n_kv_heads * head_dim].
  * KVC_DENSE_BF16: bf16 K/V; n_layers >= 1 layers stored.
  */
 typedef struct {
@@ -104,6 +110,7 @@ typedef struct {
   int32_t page_size;      /* 0 (contiguous) or 16 (LOWRANK)                   */
   int32_t n_pages;        /* physical pages in the pool when paged            */
   int32_t out_bf16;       /* 0: fp32 output, 1: bf16 output                   */
+  int32_t value_bits;     /* BLOCK_SHARED: 0 (shared) or a value latent's width */
   float softmax_scale;    /* 0 means 1/sqrt(head_dim)                         */
   double rope_theta;      /* RoPE base (500000 for Llama-3.1)                 */
 } kvc_layout_desc;
@@ -132,12 +139,18 @@ typedef struct kvc_layout kvc_layout;  /* opaque, host-side */
  *   r = rank[b][t]; offset_k/offset_v int32 [B, max_tokens + 1] (offset[b][0]
  *   must be 0), rank_k/rank_v uint8 [B, max_tokens]; bk, bv fp16 [Hkv, 64, d]
  *   of which a token uses its first r rows.
- * KVC_BLOCK_SHARED: lk_codes uint8 [B, max_tokens, latent_dim/2],
- *   lk_sz fp16 [B, max_tokens, latent_dim/group_size]; bk = W_k, bv = W_v.
+ * KVC_BLOCK_SHARED: lk_codes uint8 [B, max_tokens, latent_dim * latent_bits / 8]
+ *   (element i in bits [b i, b i + b) of the row's little-endian bit stream),
+ *   lk_sz fp16 [B, max_tokens, latent_dim/group_size]; with value_bits > 0 the
+ *   value latent likewise in lv_codes / lv_sz; bk = W_k, bv = W_v.
  * KVC_DENSE_BF16: k_dense, v_dense bf16 [n_layers, B, Hkv, max_tokens, d].
  * n_tokens: tokens 0..n_tokens-1 of every row are attended.  seq_lens
  *   (optional, device int32 [B]) gives per-row lengths; values are clamped to
  *   [0, n_tokens].  A row of length 0 produces a zero output.
+ * layer: BLOCK_SHARED and layered DENSE decode: 0 decodes all n_layers layers
+ *   at once (q, out [n_layers, B, Hq, d]); l + 1 decodes layer l alone (q, out
+ *   [B, Hq, d]) -- a layer of a block run on its own, reading the same shared
+ *   latent.  Ignored by the other kinds and by kvc_append.
  * status: optional device uint32 word.  kvc_append ORs KVC_DEV_* bits into it
  *   for every token it had to skip because a device-side argument was invalid
  *   (see kvc_append); the library never clears it.  NULL: skips go unreported.
@@ -167,7 +180,7 @@ typedef struct {
   uint8_t* rank_v;
   const int32_t* seq_lens;
   int32_t n_tokens;
-  int32_t _reserved;
+  int32_t layer;
   uint32_t* status;
 } kvc_cache;
 
@@ -242,7 +255,8 @@ int32_t kvc_decode_launches(const kvc_layout* layout, int32_t n_tokens);
  * per-token ranks ("VarRate ...", "Summary").
  *   k_new, v_new: device bf16 [B, Hkv, n_new, d] pre-RoPE keys / values
  *     (DENSE with n_layers > 1: [n_layers, B, Hkv, n_new, d]);
- *     BLOCK_SHARED: k_new = the latent, bf16 [B, n_new, latent_dim]; v_new unused.
+ *     BLOCK_SHARED: k_new = the (key) latent, bf16 [B, n_new, latent_dim]; v_new
+ *     the value latent of the same shape when value_bits > 0, else unused.
  *   pos: DEVICE int32 [B], slot of each row's first new token; the tokens go to
  *     slots pos[b] .. pos[b] + n_new - 1.
  *   new_ranks: VARRATE only, DEVICE uint8 [2, B, n_new] (K ranks, then V
@@ -340,6 +354,106 @@ kvc_status kvc_decode_attn_static(const kvc_layout* layout, const kvc_cache* cac
  * KVC_ECUDA if the copy cannot be enqueued. */
 kvc_status kvc_static_error_word(uint32_t* dst, void* stream);
 
+/* ---- Bulk prefill compression: per-head factors by randomized SVD -------
+ * "A JoLT for the KV cache ...", "Abstract (arXiv)": FlashJoLT replaces the
+ * exact token-mode SVD with a randomized approximation; "JoLT: Near-Lossless
+ * KV Cache Compression", "How JoLT works" and "Key findings": only the token
+ * and feature axes are truncated (a factor per KV head), keys before RoPE.
+ * The factor of KV head h (rank x 128) spans the top right singular subspace
+ * of the head's token-major prefill matrix (the n_rows first tokens of every
+ * batch row); kvc_append with n_new = the prefill length then projects and
+ * quantizes every token onto it.  Method: the randomized range finder with
+ * the caller's Gaussian test matrix omega and power_iters power iterations,
+ * then the exact SVD of the small projection -- computed through the Gram
+ * matrix X^T X (one tensor-core pass over x, fp32 accumulation) and fp64 dense
+ * algebra on it (orthonormalisation, Cholesky, Jacobi eigensolver).  Factor
+ * rows come largest singular value first, each scaled by +-1 so that its entry
+ * of largest magnitude is positive, and are stored as fp16.  No call
+ * synchronizes; nothing is allocated. */
+
+/* Device workspace bytes kvc_fit_factors needs for n_kv_heads heads. */
+size_t kvc_fit_workspace_bytes(int32_t n_kv_heads);
+
+/* x: device bf16 [batch, n_kv_heads, capacity, head_dim] prefill keys (pre-RoPE)
+ *   or values (the layout kvc_append reads with n_new = capacity);
+ * omega: device fp32 [n_kv_heads, head_dim, k] test matrices (N(0,1) draws);
+ * k: sketch width, even, 2..96 (rank + oversampling); rank <= k;
+ * factor: device fp16 [n_kv_heads, rank, head_dim] (the layout's bk / bv);
+ * sigma2: device fp32 [n_kv_heads, k] or NULL: the squared singular values of
+ *   the projection, largest first (the spectrum kvc_rank_bit_tables takes);
+ * workspace: device, >= kvc_fit_workspace_bytes(n_kv_heads), caller-owned.
+ * All pointers 16-byte aligned.  Errors (before anything is enqueued):
+ * KVC_EINVAL (NULL, sizes), KVC_EUNSUPPORTED (head_dim != 128), KVC_EALIGN,
+ * KVC_EWORKSPACE; KVC_ECUDA if a launch fails. */
+kvc_status kvc_fit_factors(const void* x, int32_t batch, int32_t n_kv_heads, int32_t capacity,
+                           int32_t n_rows, int32_t head_dim, const float* omega, int32_t k,
+                           int32_t rank, int32_t power_iters, void* factor, float* sigma2,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- Token importance: query salience, ranks by salience, block eviction --
+ * "VarRate: Training-Free Variable-Rate KV Cache Compression for Long-Context
+ * LLMs", "Summary" / "Method": every token gets a low-rank budget chosen by its
+ * query salience and keeps a nonzero rank.  "BellowsKV Architecture ...",
+ * "Three Measurements, Three Operators": the layers of a block agree on which
+ * tokens matter, so one importance decision per block, from all n layers'
+ * scores, is applied once to the shared latent.  Readings (the pages give no
+ * formulas): the salience of token t is the attention probability it receives
+ * from a window of queries, summed over the window and over all query heads;
+ * ranks go by salience quantiles; a block's importance is the sum of its
+ * layers' saliences and the decision keeps the `keep` most important tokens.
+ * Ties in the ordering go to the lower position. */
+
+/* Device workspace bytes kvc_window_salience needs. */
+size_t kvc_salience_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                    int32_t window, int32_t n_tokens);
+
+/* salience[b][t] = sum over query heads h and window queries w of
+ * softmax_t(scale * q[b][h][w] . keys[b][h / G][t]) over t < n_tokens.
+ *   q_window: device bf16 [batch, n_q_heads, window, 128] (as the attention
+ *     sees them, i.e. rotated when the model uses RoPE);
+ *   keys: device bf16 [batch, n_kv_heads, capacity, 128] prefill keys (rotated);
+ *   salience: device fp32 [batch, n_tokens] (written); softmax_scale 0 means
+ *     1/sqrt(128).  (n_q_heads / n_kv_heads) * window <= 128.
+ * Two tensor-core passes over the keys (bf16 in, fp32 accumulate).  Errors
+ * before anything is enqueued: KVC_EINVAL, KVC_EUNSUPPORTED (head_dim, too
+ * many window rows), KVC_EALIGN, KVC_EWORKSPACE. */
+kvc_status kvc_window_salience(const void* q_window, const void* keys, int32_t batch,
+                               int32_t n_q_heads, int32_t n_kv_heads, int32_t window,
+                               int32_t capacity, int32_t n_tokens, int32_t head_dim,
+                               float softmax_scale, float* salience, void* workspace,
+                               size_t ws_bytes, void* stream);
+
+/* Ranks by salience: in each batch row, tokens in descending salience (ties:
+ * lower position first) take rung_ranks[0] for the first rung_counts[0]
+ * tokens, rung_ranks[1] for the next rung_counts[1], ...; the last rung takes
+ * every remaining token, so no token is left without a rank.  Exact ordering
+ * (a radix select on 64-bit keys), so the counts are exact.
+ *   salience: device fp32 [batch, n_tokens];
+ *   rung_ranks: host int32 [n_rungs] in {4, 8, 16, 32, 64} (1..8 rungs);
+ *   rung_counts: host int32 [n_rungs - 1];
+ *   ranks: device uint8 [2, batch, n_tokens] (written): K ranks then V ranks
+ *     (equal), the new_ranks layout of kvc_append. */
+kvc_status kvc_ranks_by_salience(const float* salience, int32_t batch, int32_t n_tokens,
+                                 int32_t n_rungs, const int32_t* rung_ranks,
+                                 const int32_t* rung_counts, uint8_t* ranks, void* stream);
+
+/* One keep decision per block: importance[b][t] = sum over the block's layers
+ * of salience_layers[l][b][t]; kept[b] (device int32 [batch, keep], written)
+ * lists the positions of the `keep` most important tokens of row b in
+ * ascending order.  salience_layers: device fp32 [n_layers, batch, n_tokens];
+ * importance: device fp32 [batch, n_tokens] (written).  keep <= n_tokens. */
+kvc_status kvc_block_keep(const float* salience_layers, int32_t n_layers, int32_t batch,
+                          int32_t n_tokens, int32_t keep, float* importance, int32_t* kept,
+                          void* stream);
+
+/* Apply a keep decision once to a block-shared latent: row i of batch row b of
+ * dst receives row kept[b][i] of src (codes and scales), i < keep.  Both
+ * layouts are KVC_BLOCK_SHARED with the same batch and latent format; dst's
+ * capacity holds keep tokens.  The caller sets dst->n_tokens = keep afterwards. */
+kvc_status kvc_block_compact(const kvc_layout* src_layout, const kvc_cache* src,
+                             const kvc_layout* dst_layout, const kvc_cache* dst,
+                             const int32_t* kept, int32_t keep, void* stream);
+
 /* ---- Joint rank / residual-bit allocation (host only) -------------------
  * "JoLT: Near-Lossless KV Cache Compression", section "How JoLT works": the
  * layers are grouped, the keys and the values of each group are separate
@@ -397,6 +511,15 @@ kvc_status kvc_allocate_rank_bits(int32_t n_cells, int32_t n_options, const doub
  * that gives up is reported and leaves the context usable.  No counterpart on
  * the pages. */
 void kvc_test_skip_tile_copies(int32_t on);
+
+/* Kernel choice for pre-RoPE INT4 layouts (per calling thread): 0 (default)
+ * and 1 run the warp-level kernel (reconstruction on mma.sync, fp32
+ * accumulate; the faster of the two on the benchmark layout as measured), 2
+ * the warpgroup kernel with the reconstruction on tcgen05 (fp32 accumulator in
+ * TMEM) where the layout allows it.  Both compute the same decode; the switch
+ * exists so that either can be tested and timed.  No counterpart on the
+ * pages. */
+void kvc_select_rope_kernel(int32_t which);
 
 /* Thread-local description of the last error on this thread ("" if none). */
 const char* kvc_last_error(void);

@@ -193,6 +193,62 @@ def quantize_int4_sym(x, g):
     return codes, s_out
 
 
+def quantize_sym(x, g, bits):
+    """Group-wise symmetric quantizer of width `bits` (BellowsKV-Quant at the
+    page's other operating points: INT8, INT3 and a 2-bit value latent).
+
+    Per group: s = fp16(max|x| / (2^(bits-1) - 1)); code = clamp(round_half_even
+    (x / s), -(2^(bits-1) - 1), 2^(bits-1) - 1) + 2^(bits-1) (offset binary);
+    code = 2^(bits-1) when s == 0.  bits = 4 is quantize_int4_sym."""
+    x = np.asarray(x, dtype=np.float64)
+    qmax, off = 2 ** (bits - 1) - 1, 2 ** (bits - 1)
+    n = x.shape[-1]
+    ng = n_groups(n, g)
+    codes = np.empty(x.shape, dtype=np.int64)
+    s_out = np.empty(x.shape[:-1] + (ng,), dtype=np.float64)
+    for j in range(ng):
+        sl = x[..., j * g : min((j + 1) * g, n)]
+        s = fp16_rn(np.abs(sl).max(axis=-1) / qmax)
+        safe = np.where(s > 0, s, 1.0)
+        c = np.clip(np.rint(sl / safe[..., None]), -qmax, qmax) + off
+        c = np.where((s > 0)[..., None], c, off)
+        codes[..., j * g : min((j + 1) * g, n)] = c.astype(np.int64)
+        s_out[..., j] = s
+    return codes, s_out
+
+
+def dequant_sym(codes, scale, g, bits):
+    """x_hat = (code - 2^(bits-1)) * s."""
+    c = np.asarray(codes, dtype=np.float64)
+    grp = np.arange(c.shape[-1]) // g
+    return (c - 2.0 ** (bits - 1)) * np.asarray(scale, np.float64)[..., grp]
+
+
+def pack_bits(c, bits):
+    """Codes [..., n] -> bytes [..., n * bits / 8]: element i in bits
+    [bits i, bits i + bits) of the little-endian bit stream (n * bits % 8 == 0)."""
+    c = np.asarray(c, dtype=np.int64)
+    n = c.shape[-1]
+    out = np.zeros(c.shape[:-1] + (n * bits // 8,), dtype=np.uint8)
+    for i in range(n):
+        for k in range(bits):
+            bit = (c[..., i] >> k) & 1
+            pos = bits * i + k
+            out[..., pos // 8] |= (bit << (pos % 8)).astype(np.uint8)
+    return out
+
+
+def unpack_bits(codes, n, bits):
+    """Inverse of pack_bits: bytes [..., n * bits / 8] -> codes [..., n]."""
+    b = np.asarray(codes, dtype=np.int64)
+    out = np.zeros(b.shape[:-1] + (n,), dtype=np.int64)
+    for i in range(n):
+        for k in range(bits):
+            pos = bits * i + k
+            out[..., i] |= ((b[..., pos // 8] >> (pos % 8)) & 1) << k
+    return out
+
+
 def dequant_int4_sym(codes, scale, g):
     """x_hat = (code - 8) * s."""
     c = np.asarray(codes, dtype=np.float64)
@@ -354,16 +410,18 @@ def decode_varrate(q, lat_k, lat_v, rank_k, rank_v, bk, bv, scale):
     return out
 
 
-def decode_block_shared(q, latent, wk, wv, n_kv_heads, scale):
+def decode_block_shared(q, latent, wk, wv, n_kv_heads, scale, latent_v=None):
     """One latent per block of layers.  q [L, B, Hq, d]; latent [B, T, D];
     wk, wv [L, D, Hkv*d].  Layer l reconstructs K_l = latent W_k^l and
-    V_l = latent W_v^l, then runs GQA attention.  Returns [L, B, Hq, d]."""
+    V_l = latent W_v^l (latent_v W_v^l when a separate value latent is given),
+    then runs GQA attention.  Returns [L, B, Hq, d]."""
+    lat_v = latent if latent_v is None else latent_v
     nl, bsz, hq, d = q.shape
     out = np.empty((nl, bsz, hq, d))
     for l in range(nl):
         for b in range(bsz):
             K = (latent[b] @ wk[l]).reshape(-1, n_kv_heads, d).transpose(1, 0, 2)
-            V = (latent[b] @ wv[l]).reshape(-1, n_kv_heads, d).transpose(1, 0, 2)
+            V = (lat_v[b] @ wv[l]).reshape(-1, n_kv_heads, d).transpose(1, 0, 2)
             out[l, b] = gqa_decode(q[l, b], K, V, scale)
     return out
 
@@ -533,10 +591,20 @@ def decode_from_storage(desc, arrays, n_tokens):
                               f16_to_f64(arrays["bk"]), f16_to_f64(arrays["bv"]), scale)
     if kind == "block_shared":
         D, g = desc["D"], desc["g"]
-        codes = unpack_int4(np.asarray(arrays["lk_codes"])[:, :n_tokens], D)
-        lat = dequant_int4_sym(codes, f16_to_f64(np.asarray(arrays["lk_sz"])[:, :n_tokens]), g)
-        return decode_block_shared(q, lat, f16_to_f64(arrays["wk"]), f16_to_f64(arrays["wv"]),
-                                   desc["Hkv"], scale)
+        bits, vbits = desc.get("bits", 4), desc.get("vbits", 0)
+
+        def latent_of(codes_name, sz_name, b):
+            codes = unpack_bits(np.asarray(arrays[codes_name])[:, :n_tokens], D, b)
+            return dequant_sym(codes, f16_to_f64(np.asarray(arrays[sz_name])[:, :n_tokens]), g, b)
+
+        lat = latent_of("lk_codes", "lk_sz", bits)
+        lat_v = latent_of("lv_codes", "lv_sz", vbits) if vbits else None
+        wk, wv = f16_to_f64(arrays["wk"]), f16_to_f64(arrays["wv"])
+        layer = desc.get("layer", 0)
+        if layer:                      # one layer of the block: q [B, Hq, d]
+            return decode_block_shared(q[None], lat, wk[layer - 1:layer], wv[layer - 1:layer],
+                                       desc["Hkv"], scale, latent_v=lat_v)[0]
+        return decode_block_shared(q, lat, wk, wv, desc["Hkv"], scale, latent_v=lat_v)
     if kind == "dense":
         K = bf16_bits_to_f64(arrays["k_dense"])[..., :n_tokens, :]
         V = bf16_bits_to_f64(arrays["v_dense"])[..., :n_tokens, :]

@@ -7,7 +7,8 @@
 //                   round half to even; code 0 when s == 0)
 //   residual:       e = x - l_hat Bk, y = H (diag(signs) e) / sqrt(128),
 //                   s = fp16(max|y| / 1.5), code = clamp(floor(y / s) + 2, 0, 3)
-//   block-shared:   s = fp16(max|x| / 7), code = clamp(rint(x / s), -7, 7) + 8
+//   block-shared:   b-bit symmetric, s = fp16(max|x| / (2^(b-1) - 1)),
+//                   code = clamp(rint(x / s), -(2^(b-1) - 1), 2^(b-1) - 1) + 2^(b-1)
 // The INT4 rule is the per-group min/max uniform quantizer of the BellowsKV
 // page ("Worked Example: Why the Latent Quantizes Flat"): fifteen equal steps
 // between the group's extremes, each value coded by its nearest step, here with
@@ -222,38 +223,47 @@ __global__ void varrate_offsets_kernel(AppendParams a) {
 
 __global__ void __launch_bounds__(kThreads) append_block_kernel(AppendParams a) {
   const Params& p = a.p;
-  const int i = blockIdx.x % a.n_new, b = blockIdx.x / a.n_new;
+  // grid: ((b * n_new + i) * ncomp + comp); comp 1 is the separate value latent
+  const int ncomp = p.vbits ? 2 : 1;
+  int idx = blockIdx.x;
+  const int comp = idx % ncomp;
+  idx /= ncomp;
+  const int i = idx % a.n_new, b = idx / a.n_new;
   const int p0 = first_slot(a, b);
   if (p0 < 0) {
-    if (threadIdx.x == 0 && i == 0) flag(a.status, KVC_DEV_BAD_POS);
+    if (threadIdx.x == 0 && i == 0 && comp == 0) flag(a.status, KVC_DEV_BAD_POS);
     return;
   }
   const int tok = p0 + i;
   const int D = p.D, g = p.g, ng = D / g;
-  const __nv_bfloat16* src = a.k_new + ((int64_t)b * a.n_new + i) * D;
+  const int bits = comp ? p.vbits : p.bits;
+  const int qmax = (1 << (bits - 1)) - 1, zero_code = 1 << (bits - 1);
+  const __nv_bfloat16* src = (comp ? a.v_new : a.k_new) + ((int64_t)b * a.n_new + i) * D;
   const int64_t mi = (int64_t)b * p.tmax + tok;
-  uint8_t* codes = a.lk_w + mi * (D / 2);
-  __half* sc = a.lksz_w + mi * ng;
+  uint8_t* codes = (comp ? a.lv_w : a.lk_w) + mi * (D * bits / 8);
+  __half* sc = (comp ? a.lvsz_w : a.lksz_w) + mi * ng;
   __shared__ float gsc[64];
   for (int gi = threadIdx.x; gi < ng; gi += kThreads) {
     float m = 0.f;
     for (int j = gi * g; j < (gi + 1) * g; ++j) m = fmaxf(m, fabsf(bf2f(src[j])));
-    const __half sh = __float2half_rn(m / 7.f);
+    const __half sh = __float2half_rn(m / (float)qmax);
     sc[gi] = sh;
     gsc[gi] = __half2float(sh);
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < D / 2; j += kThreads) {
-    int c2[2];
+  // eight codes per thread: element e in bits [bits e, bits e + bits) of the row
+  for (int j = threadIdx.x; j < D / 8; j += kThreads) {
+    uint64_t word = 0;
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int e = 2 * j + k;
+    for (int k = 0; k < 8; ++k) {
+      const int e = 8 * j + k;
       const float s = gsc[e / g];
-      int c = 8;
-      if (s > 0.f) c = (int)fminf(fmaxf(rintf(bf2f(src[e]) / s), -7.f), 7.f) + 8;
-      c2[k] = c;
+      int c = zero_code;
+      if (s > 0.f)
+        c = (int)fminf(fmaxf(rintf(bf2f(src[e]) / s), (float)-qmax), (float)qmax) + zero_code;
+      word |= (uint64_t)c << (bits * k);
     }
-    codes[j] = (uint8_t)(c2[0] | (c2[1] << 4));
+    for (int k = 0; k < bits; ++k) codes[(size_t)j * bits + k] = (uint8_t)(word >> (8 * k));
   }
 }
 
@@ -294,7 +304,7 @@ cudaError_t launch_append(const AppendParams& a, cudaStream_t s) {
       append_lowrank_kernel<<<p.B * p.Hkv * 2 * a.n_new, kThreads, 0, s>>>(a);
       break;
     case KVC_BLOCK_SHARED:
-      append_block_kernel<<<p.B * a.n_new, kThreads, 0, s>>>(a);
+      append_block_kernel<<<p.B * a.n_new * (p.vbits ? 2 : 1), kThreads, 0, s>>>(a);
       break;
     default:
       append_dense_kernel<<<p.L * p.B * p.Hkv * a.n_new, 128, 0, s>>>(a);

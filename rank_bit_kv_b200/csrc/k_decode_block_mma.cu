@@ -304,7 +304,8 @@ __global__ void __launch_bounds__(kXThreads, 2) block_mma_kernel(Params p) {
 }  // namespace
 
 bool block_mma_supported(const Params& p) {
-  return p.kind == KVC_BLOCK_SHARED && p.D == kXD && p.g == kXG && p.d == 128 &&
+  return p.kind == KVC_BLOCK_SHARED && p.bits == 4 && p.vbits == 0 && p.D == kXD &&
+         p.g == kXG && p.d == 128 &&
          (p.L * p.Hq) % kXQ == 0 && !p.seq_lens && p.n_tokens > 0 && p.qdim == kXD &&
          p.vdim == kXD;
 }

@@ -53,7 +53,7 @@ __host__ __device__ inline Geo geometry(const Params& p) {
       g.nq = kBlockQueries;
       g.kd = p.D;
       g.vd = p.D;
-      g.alias_v = true;
+      g.alias_v = p.vbits == 0;     // one latent feeds keys and values
       break;
     default:
       g.nq = p.G;
@@ -254,14 +254,18 @@ __global__ void __launch_bounds__(kThreads) split_generic_kernel(Params p) {
       }
     } else if (p.kind == KVC_BLOCK_SHARED) {
       const int D = p.D, ng = D / p.g;
+      const int kb = D * p.bits / 8, vb = D * p.vbits / 8;
       for (int e = tid; e < g.tt * D; e += kThreads) {
         const int t = e / D, c = e % D;
-        float v = 0.f;
+        float v = 0.f, w = 0.f;
         if (t < nt) {
           const int64_t mi = (int64_t)b * p.tmax + t0 + t;
-          v = ((float)int4_at(p.lk + mi * (D / 2), c) - 8.f) * h2f(p.lksz[mi * ng + c / p.g]);
+          v = (float)sym_level_at(p.lk + mi * kb, c, p.bits) * h2f(p.lksz[mi * ng + c / p.g]);
+          if (p.vbits)
+            w = (float)sym_level_at(p.lv + mi * vb, c, p.vbits) * h2f(p.lvsz[mi * ng + c / p.g]);
         }
         kt[t * kstr + c] = v;
+        if (p.vbits) vt[t * vstr + c] = w;
       }
     } else {  // dense bf16
       const int d = p.d;
@@ -362,6 +366,7 @@ cudaError_t launch_split(const Params& p, cudaStream_t s) {
     case 2: return launch_dense_tc(p, s);
     case 3: return launch_latent_tc(p, s);
     case 4: return launch_rope_mma(p, s);
+    case 7: return launch_rope_wg(p, s);
     case 5: return launch_varrate_warp(p, s);
     case 6: return launch_block_mma(p, s);
     default: break;

@@ -25,6 +25,7 @@ namespace {
 
 thread_local std::string g_err;
 thread_local int g_test_no_copies = 0;   // kvc_test_skip_tile_copies
+thread_local int g_rope_kernel = 0;      // kvc_select_rope_kernel
 
 kvc_status fail(kvc_status st, const char* fmt, ...) {
   char buf[512];
@@ -89,6 +90,8 @@ size_t ws_bytes(const kvc_layout* L, int n_tokens) {
     if (Sl > S) S = Sl;
     const int Sr = kvc::rope_mma_slots(L->d.batch, L->d.n_kv_heads, nt1);
     if (Sr > S) S = Sr;
+    const int Sw = kvc::rope_wg_slots(L->d.batch, L->d.n_kv_heads, nt1);
+    if (Sw > S) S = Sw;
   }
   if (L->d.kind == KVC_VARRATE) {
     const int Sv = kvc::varrate_warp_slots(L->d.batch, nt1);
@@ -122,7 +125,9 @@ const char* kvc_last_error(void) { return g_err.c_str(); }
 
 void kvc_test_skip_tile_copies(int32_t on) { g_test_no_copies = on ? 1 : 0; }
 
-const char* kvc_version(void) { return "kvc 0.2 (sm_100a; decode kernels rev 11)"; }
+void kvc_select_rope_kernel(int32_t which) { g_rope_kernel = which == 2 ? 2 : 0; }
+
+const char* kvc_version(void) { return "kvc 0.3 (sm_100a; decode kernels rev 12)"; }
 
 kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out) {
   if (!desc || !out) return fail(KVC_EINVAL, "kvc_create_layout: NULL argument");
@@ -247,8 +252,24 @@ kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out) {
         st = KVC_EUNSUPPORTED, why = "n_layers * n_q_heads must be a multiple of 32";
         break;
       }
-      L->sizes[KVC_BUF_LK_CODES] = B * T * d.latent_dim / 2;
-      L->sizes[KVC_BUF_LK_SZ] = B * T * (d.latent_dim / d.group_size) * 2;
+      if (d.latent_bits == 0) d.latent_bits = 4;
+      if (d.latent_bits != 3 && d.latent_bits != 4 && d.latent_bits != 8) {
+        st = KVC_EUNSUPPORTED, why = "block-shared latent_bits must be 3, 4 or 8";
+        break;
+      }
+      if (d.value_bits != 0 && d.value_bits != 2 && d.value_bits != 3 && d.value_bits != 4 &&
+          d.value_bits != 8) {
+        st = KVC_EUNSUPPORTED, why = "value_bits must be 0 (shared latent) or 2, 3, 4, 8";
+        break;
+      }
+      L->d.latent_bits = d.latent_bits;
+      const size_t ngs = d.latent_dim / d.group_size;
+      L->sizes[KVC_BUF_LK_CODES] = B * T * d.latent_dim * d.latent_bits / 8;
+      L->sizes[KVC_BUF_LK_SZ] = B * T * ngs * 2;
+      if (d.value_bits) {
+        L->sizes[KVC_BUF_LV_CODES] = B * T * d.latent_dim * d.value_bits / 8;
+        L->sizes[KVC_BUF_LV_SZ] = B * T * ngs * 2;
+      }
       L->sizes[KVC_BUF_BK] = L->sizes[KVC_BUF_BV] =
           (size_t)d.n_layers * d.latent_dim * Hkv * hd * 2;
       L->qdim = d.latent_dim;
@@ -296,8 +317,12 @@ size_t kvc_step_bytes(const kvc_layout* L, int32_t n) {
       const double ef = 0.4 * 6 + 0.25 * 8 + 0.2 * 12 + 0.1 * 20 + 0.05 * 40;
       return (size_t)((double)rowsB * 2 * ef) + (size_t)d.batch * n * 10;
     }
-    case KVC_BLOCK_SHARED:
-      return (size_t)d.batch * n * (d.latent_dim / 2 + 2 * (d.latent_dim / d.group_size));
+    case KVC_BLOCK_SHARED: {
+      const size_t scales = 2 * (d.latent_dim / d.group_size);
+      size_t per = d.latent_dim * d.latent_bits / 8 + scales;
+      if (d.value_bits) per += d.latent_dim * d.value_bits / 8 + scales;
+      return (size_t)d.batch * n * per;
+    }
     case KVC_DENSE_BF16:
       return (size_t)d.n_layers * rowsB * d.head_dim * 2 * 2;
   }
@@ -336,6 +361,7 @@ static kvc_status fill_params(const kvc_layout* L, const kvc_cache* c, kvc::Para
   p->rk = d.rank_k;
   p->rv = d.rank_v;
   p->bits = d.latent_bits;
+  p->vbits = d.kind == KVC_BLOCK_SHARED ? d.value_bits : 0;
   p->g = d.group_size;
   p->ngk = L->ngk;
   p->ngv = L->ngv;
@@ -416,6 +442,10 @@ static kvc_status fill_params(const kvc_layout* L, const kvc_cache* c, kvc::Para
     case KVC_BLOCK_SHARED:
       need[nn++] = {c->lk_codes, "lk_codes"};
       need[nn++] = {c->lk_sz, "lk_sz"};
+      if (d.value_bits) {
+        need[nn++] = {c->lv_codes, "lv_codes (value latent)"};
+        need[nn++] = {c->lv_sz, "lv_sz (value latent)"};
+      }
       need[nn++] = {c->bk, "bk (W_k)"};
       need[nn++] = {c->bv, "bv (W_v)"};
       break;
@@ -456,6 +486,23 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
   kvc::Params p;
   kvc_status st = fill_params(L, c, &p);
   if (st != KVC_OK) return st;
+  if (c->layer < 0 || c->layer > L->L)
+    return fail(KVC_EINVAL, "cache.layer %d outside 0..%d", c->layer, L->L);
+  if (c->layer > 0 && L->L > 1) {
+    // one layer of the block: the shared cache with that layer's projections
+    // (block-shared) or that layer's slice of the dense cache
+    const size_t lo = (size_t)(c->layer - 1);
+    if (L->d.kind == KVC_BLOCK_SHARED) {
+      const size_t wsz = (size_t)L->d.latent_dim * L->d.n_kv_heads * L->d.head_dim;
+      p.bk += lo * wsz;
+      p.bv += lo * wsz;
+    } else if (L->d.kind == KVC_DENSE_BF16) {
+      const size_t lsz = (size_t)L->d.batch * L->d.n_kv_heads * L->d.max_tokens * L->d.head_dim;
+      p.kd += lo * lsz;
+      p.vd += lo * lsz;
+    }
+    p.L = 1;
+  }
   p.q = (const __nv_bfloat16*)q;
   p.test_no_copies = g_test_no_copies;
   p.out = out;
@@ -465,7 +512,11 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
     // the warp- / CTA-level tensor-core kernels run equal contiguous tile
     // ranges (seg_W tiles of the flattened (unit, tile) space per warp or CTA)
     int grid = 0, W = 0, tpu = 0, slots = 0, parts = 1;
-    if (kvc::rope_mma_supported(p)) {
+    if (kvc::rope_wg_supported(p) && g_rope_kernel == 2) {
+      kvc::rope_wg_plan(p, &grid, &W, &tpu, &slots);
+      p.path = 7;
+      parts = kvc::kRopeWgParts;
+    } else if (kvc::rope_mma_supported(p)) {
       kvc::rope_mma_plan(p, &grid, &W, &tpu, &slots);
       p.path = 4;
     } else if (kvc::rope_tc_supported(p)) {
@@ -532,7 +583,7 @@ extern "C" kvc_status kvc_append(const kvc_layout* L, const kvc_cache* c, const 
   if (n_new < 1) return fail(KVC_EINVAL, "n_new %d < 1", n_new);
   if (n_new > d.max_tokens)
     return fail(KVC_ECAPACITY, "n_new %d > max_tokens %d", n_new, d.max_tokens);
-  if (!k_new || (d.kind != KVC_BLOCK_SHARED && !v_new))
+  if (!k_new || ((d.kind != KVC_BLOCK_SHARED || d.value_bits) && !v_new))
     return fail(KVC_EINVAL, "kvc_append: k_new / v_new is NULL");
   if (!aligned16(k_new) || (v_new && !aligned16(v_new)) || !aligned16(pos))
     return fail(KVC_EALIGN, "k_new / v_new / pos must be 16-byte aligned");
@@ -575,6 +626,173 @@ extern "C" kvc_status kvc_append(const kvc_layout* L, const kvc_cache* c, const 
   cudaGetLastError();
   st = launch_status(kvc::launch_append(*a, s), "append launch");
   delete a;
+  if (st != KVC_OK) return st;
+  return ok();
+}
+
+extern "C" size_t kvc_fit_workspace_bytes(int32_t n_kv_heads) {
+  return n_kv_heads > 0 ? kvc::fit_workspace_bytes(n_kv_heads) : 0;
+}
+
+extern "C" kvc_status kvc_fit_factors(const void* x, int32_t batch, int32_t n_kv_heads,
+                                      int32_t capacity, int32_t n_rows, int32_t head_dim,
+                                      const float* omega, int32_t k, int32_t rank,
+                                      int32_t power_iters, void* factor, float* sigma2,
+                                      void* workspace, size_t ws_size, void* stream) {
+  if (!x || !omega || !factor || !workspace)
+    return fail(KVC_EINVAL, "kvc_fit_factors: NULL argument");
+  if (head_dim != 128) return fail(KVC_EUNSUPPORTED, "kvc_fit_factors: head_dim %d (128)", head_dim);
+  if (batch < 1 || n_kv_heads < 1 || capacity < 1 || n_rows < 1 || n_rows > capacity)
+    return fail(KVC_EINVAL, "kvc_fit_factors: batch %d, heads %d, rows %d of capacity %d", batch,
+                n_kv_heads, n_rows, capacity);
+  if (k < 2 || k > kvc::kFitMaxK || k % 2 || rank < 1 || rank > k)
+    return fail(KVC_EINVAL, "kvc_fit_factors: sketch width %d (even, 2..%d) and rank %d (<= k)",
+                k, kvc::kFitMaxK, rank);
+  if (power_iters < 0 || power_iters > 16)
+    return fail(KVC_EINVAL, "kvc_fit_factors: power_iters %d (0..16)", power_iters);
+  if (!aligned16(x) || !aligned16(omega) || !aligned16(factor) || !aligned16(workspace) ||
+      (sigma2 && !aligned16(sigma2)))
+    return fail(KVC_EALIGN, "kvc_fit_factors: pointers must be 16-byte aligned");
+  const size_t need = kvc::fit_workspace_bytes(n_kv_heads);
+  if (ws_size < need) return fail(KVC_EWORKSPACE, "workspace %zu bytes < %zu needed", ws_size, need);
+  kvc::FitParams f;
+  f.x = (const __nv_bfloat16*)x;
+  f.B = batch;
+  f.Hkv = n_kv_heads;
+  f.cap = capacity;
+  f.n_rows = n_rows;
+  f.omega = omega;
+  f.k = k;
+  f.rank = rank;
+  f.power_iters = power_iters;
+  f.factor = (__half*)factor;
+  f.sigma2 = sigma2;
+  f.workspace = workspace;
+  cudaGetLastError();
+  kvc_status st = launch_status(kvc::launch_fit(f, (cudaStream_t)stream), "factor fit launch");
+  if (st != KVC_OK) return st;
+  return ok();
+}
+
+extern "C" size_t kvc_salience_workspace_bytes(int32_t batch, int32_t n_q_heads,
+                                               int32_t n_kv_heads, int32_t window,
+                                               int32_t n_tokens) {
+  if (batch < 1 || n_q_heads < 1 || n_kv_heads < 1 || window < 1 || n_tokens < 1) return 0;
+  return kvc::salience_workspace_bytes(batch, n_q_heads, n_kv_heads, window, n_tokens);
+}
+
+extern "C" kvc_status kvc_window_salience(const void* q_window, const void* keys, int32_t batch,
+                                          int32_t n_q_heads, int32_t n_kv_heads, int32_t window,
+                                          int32_t capacity, int32_t n_tokens, int32_t head_dim,
+                                          float softmax_scale, float* salience, void* workspace,
+                                          size_t ws_size, void* stream) {
+  if (!q_window || !keys || !salience || !workspace)
+    return fail(KVC_EINVAL, "kvc_window_salience: NULL argument");
+  if (head_dim != 128) return fail(KVC_EUNSUPPORTED, "kvc_window_salience: head_dim %d (128)", head_dim);
+  if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads || window < 1 ||
+      n_tokens < 1 || n_tokens > capacity)
+    return fail(KVC_EINVAL, "kvc_window_salience: bad sizes");
+  if ((n_q_heads / n_kv_heads) * window > kvc::kSalMaxRows)
+    return fail(KVC_EUNSUPPORTED, "kvc_window_salience: %d query heads per KV head x window %d > %d",
+                n_q_heads / n_kv_heads, window, kvc::kSalMaxRows);
+  if (!aligned16(q_window) || !aligned16(keys) || !aligned16(salience) || !aligned16(workspace))
+    return fail(KVC_EALIGN, "kvc_window_salience: pointers must be 16-byte aligned");
+  const size_t need = kvc::salience_workspace_bytes(batch, n_q_heads, n_kv_heads, window, n_tokens);
+  if (ws_size < need) return fail(KVC_EWORKSPACE, "workspace %zu bytes < %zu needed", ws_size, need);
+  kvc::SalienceCall c;
+  c.q = (const __nv_bfloat16*)q_window;
+  c.k = (const __nv_bfloat16*)keys;
+  c.B = batch;
+  c.Hq = n_q_heads;
+  c.Hkv = n_kv_heads;
+  c.W = window;
+  c.cap = capacity;
+  c.T = n_tokens;
+  c.scale = softmax_scale > 0 ? softmax_scale : 1.0f / sqrtf((float)head_dim);
+  c.sal = salience;
+  c.workspace = workspace;
+  cudaGetLastError();
+  kvc_status st = launch_status(kvc::launch_salience(c, (cudaStream_t)stream), "salience launch");
+  if (st != KVC_OK) return st;
+  return ok();
+}
+
+extern "C" kvc_status kvc_ranks_by_salience(const float* salience, int32_t batch,
+                                            int32_t n_tokens, int32_t n_rungs,
+                                            const int32_t* rung_ranks, const int32_t* rung_counts,
+                                            uint8_t* ranks, void* stream) {
+  if (!salience || !rung_ranks || !ranks || (n_rungs > 1 && !rung_counts))
+    return fail(KVC_EINVAL, "kvc_ranks_by_salience: NULL argument");
+  if (batch < 1 || n_tokens < 1 || n_rungs < 1 || n_rungs > 8)
+    return fail(KVC_EINVAL, "kvc_ranks_by_salience: batch %d, tokens %d, rungs %d (1..8)", batch,
+                n_tokens, n_rungs);
+  kvc::RankLadder lad;
+  memset(&lad, 0, sizeof(lad));
+  lad.n = n_rungs;
+  for (int i = 0; i < n_rungs; ++i) {
+    const int r = rung_ranks[i];
+    if (r != 4 && r != 8 && r != 16 && r != 32 && r != 64)
+      return fail(KVC_EINVAL, "rung %d: rank %d not in {4, 8, 16, 32, 64}", i, r);
+    lad.rank[i] = r;
+    if (i + 1 < n_rungs) {
+      if (rung_counts[i] < 0) return fail(KVC_EINVAL, "rung %d: negative count", i);
+      lad.count[i] = rung_counts[i];
+    }
+  }
+  if (!aligned16(salience) || !aligned16(ranks))
+    return fail(KVC_EALIGN, "kvc_ranks_by_salience: pointers must be 16-byte aligned");
+  cudaGetLastError();
+  kvc_status st = launch_status(kvc::launch_ranks(nullptr, 0, const_cast<float*>(salience), batch,
+                                                  n_tokens, lad, ranks, (cudaStream_t)stream),
+                                "ranks launch");
+  if (st != KVC_OK) return st;
+  return ok();
+}
+
+extern "C" kvc_status kvc_block_keep(const float* salience_layers, int32_t n_layers,
+                                     int32_t batch, int32_t n_tokens, int32_t keep,
+                                     float* importance, int32_t* kept, void* stream) {
+  if (!salience_layers || !importance || !kept)
+    return fail(KVC_EINVAL, "kvc_block_keep: NULL argument");
+  if (n_layers < 1 || batch < 1 || n_tokens < 1 || keep < 1 || keep > n_tokens)
+    return fail(KVC_EINVAL, "kvc_block_keep: layers %d, batch %d, keep %d of %d tokens", n_layers,
+                batch, keep, n_tokens);
+  if (!aligned16(salience_layers) || !aligned16(importance) || !aligned16(kept))
+    return fail(KVC_EALIGN, "kvc_block_keep: pointers must be 16-byte aligned");
+  cudaGetLastError();
+  kvc_status st = launch_status(kvc::launch_keep(salience_layers, n_layers, importance, batch,
+                                                 n_tokens, keep, kept, (cudaStream_t)stream),
+                                "keep launch");
+  if (st != KVC_OK) return st;
+  return ok();
+}
+
+extern "C" kvc_status kvc_block_compact(const kvc_layout* src_layout, const kvc_cache* src,
+                                        const kvc_layout* dst_layout, const kvc_cache* dst,
+                                        const int32_t* kept, int32_t keep, void* stream) {
+  if (!src_layout || !src || !dst_layout || !dst || !kept)
+    return fail(KVC_EINVAL, "kvc_block_compact: NULL argument");
+  const kvc_layout_desc& a = src_layout->d;
+  const kvc_layout_desc& b = dst_layout->d;
+  if (a.kind != KVC_BLOCK_SHARED || b.kind != KVC_BLOCK_SHARED)
+    return fail(KVC_EUNSUPPORTED, "kvc_block_compact: block-shared layouts only");
+  if (a.batch != b.batch || a.latent_dim != b.latent_dim || a.group_size != b.group_size)
+    return fail(KVC_EINVAL, "kvc_block_compact: the two layouts differ in batch or latent format");
+  if (keep < 1 || keep > b.max_tokens || keep > src->n_tokens)
+    return fail(KVC_ECAPACITY, "kvc_block_compact: keep %d (source %d tokens, destination holds %d)",
+                keep, src->n_tokens, b.max_tokens);
+  if (!src->lk_codes || !src->lk_sz || !dst->lk_codes || !dst->lk_sz)
+    return fail(KVC_EINVAL, "kvc_block_compact: cache buffers are NULL");
+  if (!aligned16(src->lk_codes) || !aligned16(dst->lk_codes) || !aligned16(kept) ||
+      !aligned16(src->lk_sz) || !aligned16(dst->lk_sz))
+    return fail(KVC_EALIGN, "kvc_block_compact: pointers must be 16-byte aligned");
+  cudaGetLastError();
+  kvc_status st = launch_status(
+      kvc::launch_compact((const uint8_t*)src->lk_codes, (const __half*)src->lk_sz,
+                          (uint8_t*)dst->lk_codes, (__half*)dst->lk_sz, kept, a.batch,
+                          a.max_tokens, b.max_tokens, keep, a.latent_dim / 2,
+                          a.latent_dim / a.group_size, (cudaStream_t)stream),
+      "compact launch");
   if (st != KVC_OK) return st;
   return ok();
 }

@@ -37,6 +37,16 @@ __device__ __forceinline__ int int4_at(const uint8_t* row, int r) {
   return (r & 1) ? (byte >> 4) : (byte & 15);
 }
 
+// Signed level of the symmetric code of width `bits` at element i of a row:
+// element i occupies bits [bits * i, bits * i + bits) of the row's
+// little-endian bit stream; level = code - 2^(bits - 1).
+__device__ __forceinline__ int sym_level_at(const uint8_t* row, int i, int bits) {
+  const int o = i * bits, byte = o >> 3, sh = o & 7;
+  int v = row[byte] >> sh;
+  if (sh + bits > 8) v |= row[byte + 1] << (8 - sh);
+  return (v & ((1 << bits) - 1)) - (1 << (bits - 1));
+}
+
 // 2-bit element i of a row: element 4j+k in bits 2k..2k+1 of byte j.
 __device__ __forceinline__ int int2_at(const uint8_t* row, int i) {
   return (row[i >> 2] >> (2 * (i & 3))) & 3;

@@ -20,6 +20,7 @@ struct Params {
   // shape
   int kind, B, Hq, Hkv, G, d, L;
   int rk, rv, bits, g, ngk, ngv;
+  int vbits;             // block-shared: width of the separate value latent (0 = shared)
   int resid, rope, page, tmax, n_pages;
   int D;                 // block-shared latent width
   int n_tokens;
@@ -63,7 +64,7 @@ struct Params {
   int seg_W, seg_tpu;
   int seg_parts;         // partials written per CTA and unit on that path
   int path;              // split kernel: 0 generic, 1 rope_tc, 2 dense_tc, 3 latent_tc, 4 rope_mma,
-                         // 5 varrate_warp, 6 block_mma
+                         // 5 varrate_warp, 6 block_mma, 7 rope_wg
   uint32_t* err;         // error word of the workspace (bounded waits that gave up)
   int test_no_copies;    // test switch: the tcgen05 producer issues no tile copies
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
@@ -132,6 +133,14 @@ void rope_mma_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
 int rope_mma_slots(int batch, int n_kv_heads, int n_tokens);
 cudaError_t launch_rope_mma(const Params& p, cudaStream_t s);
 
+// pre-RoPE INT4 low-rank caches, warpgroup-autonomous, reconstruction on
+// tcgen05 (fp32 TMEM accumulator); four partials per warpgroup and unit
+constexpr int kRopeWgParts = 4;
+bool rope_wg_supported(const Params& p);
+void rope_wg_plan(const Params& p, int* grid, int* W, int* tpu, int* slots);
+int rope_wg_slots(int batch, int n_kv_heads, int n_tokens);
+cudaError_t launch_rope_wg(const Params& p, cudaStream_t s);
+
 // variable-rate layout, one lane per (KV head, query head)
 bool varrate_warp_supported(const Params& p);
 void varrate_warp_plan(const Params& p, int* splits, int* split_len);
@@ -143,6 +152,47 @@ bool block_mma_supported(const Params& p);
 void block_mma_plan(const Params& p, int* splits, int* split_len);
 int block_mma_slots(int batch, int n_layers, int n_q_heads, int n_tokens);
 cudaError_t launch_block_mma(const Params& p, cudaStream_t s);
+
+// factor fit by randomized SVD (bulk prefill compression)
+constexpr int kFitChunks = 64;        // Gram partials (CTAs) per KV head
+constexpr int kFitMaxK = 96;          // largest sketch width (rank + oversampling)
+constexpr int kFitSweeps = 10;        // Jacobi sweeps of the small eigenproblem
+struct FitParams {
+  const __nv_bfloat16* x;             // [B, Hkv, cap, 128] prefill keys or values
+  int B, Hkv, cap, n_rows;
+  const float* omega;                 // [Hkv, 128, k]
+  int k, rank, power_iters;
+  __half* factor;                     // [Hkv, rank, 128]
+  float* sigma2;                      // [Hkv, k] or null
+  void* workspace;
+};
+size_t fit_workspace_bytes(int n_kv_heads);
+cudaError_t launch_fit(const FitParams& f, cudaStream_t s);
+
+// token-importance producers (salience, ranks by salience, block keep decision)
+constexpr int kSalMaxRows = 128;      // query heads per KV head x window queries
+struct SalienceCall {
+  const __nv_bfloat16* q;             // [B, Hq, W, 128]
+  const __nv_bfloat16* k;             // [B, Hkv, cap, 128]
+  int B, Hq, Hkv, W, cap, T;
+  float scale;
+  float* sal;                         // [B, T]
+  void* workspace;
+};
+struct RankLadder {
+  int n;                              // rungs (<= 8)
+  int rank[8];                        // rank of each rung, most salient first
+  int count[8];                       // tokens of each rung but the last (the last takes the rest)
+};
+size_t salience_workspace_bytes(int B, int Hq, int Hkv, int W, int T);
+cudaError_t launch_salience(const SalienceCall& c, cudaStream_t s);
+cudaError_t launch_ranks(const float* part_sal, int Hkv, float* sal, int B, int T,
+                         const RankLadder& lad, uint8_t* ranks, cudaStream_t s);
+cudaError_t launch_keep(const float* sal_layers, int n_layers, float* importance, int B, int T,
+                        int keep, int* kept, cudaStream_t s);
+cudaError_t launch_compact(const uint8_t* src_codes, const __half* src_scales, uint8_t* dst_codes,
+                           __half* dst_scales, const int* kept, int B, int cap_src, int cap_dst,
+                           int keep, int code_bytes, int n_scales, cudaStream_t s);
 
 // Record a status and message for kvc_last_error(); returns st.
 kvc_status report_error(kvc_status st, const char* fmt, ...);
@@ -161,6 +211,8 @@ __host__ __device__ inline bool needs_qproj(const Params& p) {
 
 // Whether the chosen split kernel has bounded waits that can set the
 // workspace error word (the call zeroes the word first only then).
-__host__ __device__ inline bool path_sets_error_word(const Params& p) { return p.path == 1; }
+__host__ __device__ inline bool path_sets_error_word(const Params& p) {
+  return p.path == 1 || p.path == 7;
+}
 
 }  // namespace kvc

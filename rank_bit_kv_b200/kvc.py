@@ -29,15 +29,15 @@ class LayoutDesc(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "kind", "batch", "n_q_heads", "n_kv_heads", "head_dim", "max_tokens", "n_layers",
         "rank_k", "rank_v", "latent_bits", "group_size", "latent_dim", "rope", "resid_bits",
-        "page_size", "n_pages", "out_bf16")] + [("softmax_scale", C.c_float),
-                                                 ("rope_theta", C.c_double)]
+        "page_size", "n_pages", "out_bf16", "value_bits")] + [("softmax_scale", C.c_float),
+                                                               ("rope_theta", C.c_double)]
 
 
 class CacheDesc(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in BUFS[:15]] + [
         ("offset_k", C.c_void_p), ("offset_v", C.c_void_p), ("rank_k", C.c_void_p),
         ("rank_v", C.c_void_p), ("seq_lens", C.c_void_p), ("n_tokens", C.c_int32),
-        ("_reserved", C.c_int32), ("status", C.c_void_p)]
+        ("layer", C.c_int32), ("status", C.c_void_p)]
 
 # bits of the device-side status words (include/kvc.h, KVC_DEV_*)
 DEV_WAIT_TIMEOUT, DEV_BAD_POS, DEV_BAD_RANK, DEV_BAD_PAGE, DEV_BAD_OFFSET = 1, 2, 4, 8, 16
@@ -96,6 +96,26 @@ def lib():
         L.kvc_rank_bit_tables.restype = C.c_int
         L.kvc_allocate_rank_bits.argtypes = [i32, i32, dp, dp, C.c_double, C.POINTER(i32), dp]
         L.kvc_allocate_rank_bits.restype = C.c_int
+        L.kvc_fit_workspace_bytes.argtypes = [i32]
+        L.kvc_fit_workspace_bytes.restype = sz
+        L.kvc_fit_factors.argtypes = [vp, i32, i32, i32, i32, i32, vp, i32, i32, i32, vp, vp, vp,
+                                      sz, vp]
+        L.kvc_fit_factors.restype = C.c_int
+        L.kvc_salience_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        L.kvc_salience_workspace_bytes.restype = sz
+        L.kvc_window_salience.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, C.c_float,
+                                          vp, vp, sz, vp]
+        L.kvc_window_salience.restype = C.c_int
+        L.kvc_ranks_by_salience.argtypes = [vp, i32, i32, i32, C.POINTER(i32), C.POINTER(i32), vp,
+                                            vp]
+        L.kvc_ranks_by_salience.restype = C.c_int
+        L.kvc_block_keep.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
+        L.kvc_block_keep.restype = C.c_int
+        L.kvc_block_compact.argtypes = [vp, C.POINTER(CacheDesc), vp, C.POINTER(CacheDesc), vp,
+                                        i32, vp]
+        L.kvc_block_compact.restype = C.c_int
+        L.kvc_select_rope_kernel.argtypes = [i32]
+        L.kvc_select_rope_kernel.restype = None
         L.kvc_test_skip_tile_copies.argtypes = [i32]
         L.kvc_test_skip_tile_copies.restype = None
         L.kvc_last_error.argtypes = []
@@ -140,7 +160,8 @@ def desc_from_config(c, capacity=None, out_bf16=0):
     if kind == "block_shared":
         return make_desc("block_shared", batch=c["B"], n_q_heads=c["Hq"], n_kv_heads=c["Hkv"],
                          head_dim=c["d"], max_tokens=cap, n_layers=c["L"], latent_dim=c["D"],
-                         group_size=c["g"], out_bf16=out_bf16)
+                         group_size=c["g"], latent_bits=c.get("bits", 4),
+                         value_bits=c.get("vbits", 0), out_bf16=out_bf16)
     if kind == "dense":
         return make_desc("dense", batch=c["B"], n_q_heads=c["Hq"], n_kv_heads=c["Hkv"],
                          head_dim=c["d"], max_tokens=cap, n_layers=c.get("L", 1),
@@ -195,6 +216,7 @@ class Cache:
         self.n_tokens = 0
         self.seq_lens = None
         self.status = None        # optional device int32 [1] for append's KVC_DEV_* bits
+        self.layer = 0            # block-shared / layered dense: 0 all layers, l + 1 layer l
         if fill:
             self.upload(fill)
 
@@ -220,6 +242,7 @@ class Cache:
         c.seq_lens = None if self.seq_lens is None else self.seq_lens.data_ptr()
         c.n_tokens = int(self.n_tokens)
         c.status = None if self.status is None else self.status.data_ptr()
+        c.layer = int(self.layer)
         return c
 
 
@@ -364,3 +387,80 @@ def allocate_rank_bits(bytes_, distortion, budget):
     lam = C.c_double()
     check(lib().kvc_allocate_rank_bits(n_cells, n_opt, bp, dp, float(budget), ch, C.byref(lam)))
     return np.array(list(ch), np.int64), lam.value
+
+
+# --------------------------------------------------------------------------- factor fit
+
+
+def fit_factors(x, omega, rank, power_iters, n_rows=None, stream=None, with_sigma2=True):
+    """kvc_fit_factors on torch tensors: x bf16 [B, Hkv, cap, 128], omega fp32
+    [Hkv, 128, k].  Returns (factor fp16 [Hkv, rank, 128], sigma2 fp32 [Hkv, k])."""
+    import torch
+
+    B, Hkv, cap, d = x.shape
+    k = omega.shape[-1]
+    factor = torch.empty((Hkv, rank, d), dtype=torch.float16, device=x.device)
+    sigma2 = torch.empty((Hkv, k), dtype=torch.float32, device=x.device) if with_sigma2 else None
+    ws = torch.empty(int(lib().kvc_fit_workspace_bytes(Hkv)), dtype=torch.uint8, device=x.device)
+    st = stream if stream is not None else current_stream_ptr()
+    check(lib().kvc_fit_factors(_ptr(x), B, Hkv, cap, int(n_rows or cap), d, _ptr(omega), k,
+                                int(rank), int(power_iters), _ptr(factor), _ptr(sigma2),
+                                _ptr(ws), ws.numel(), st))
+    factor._fit_ws = ws        # keep the workspace alive until the stream has used it
+    return factor, sigma2
+
+
+# --------------------------------------------------------------------------- token importance
+
+
+def window_salience(q_window, keys, n_tokens=None, scale=0.0, stream=None):
+    """kvc_window_salience: q_window bf16 [B, Hq, W, 128], keys bf16 [B, Hkv, cap, 128]
+    -> salience fp32 [B, n_tokens]."""
+    import torch
+
+    B, Hq, W, d = q_window.shape
+    Hkv, cap = keys.shape[1], keys.shape[2]
+    T = int(n_tokens or cap)
+    sal = torch.empty((B, T), dtype=torch.float32, device=keys.device)
+    ws = torch.empty(int(lib().kvc_salience_workspace_bytes(B, Hq, Hkv, W, T)),
+                     dtype=torch.uint8, device=keys.device)
+    st = stream if stream is not None else current_stream_ptr()
+    check(lib().kvc_window_salience(_ptr(q_window), _ptr(keys), B, Hq, Hkv, W, cap, T, d,
+                                    float(scale), _ptr(sal), _ptr(ws), ws.numel(), st))
+    sal._ws = ws
+    return sal
+
+
+def ranks_by_salience(salience, rung_ranks, rung_counts, stream=None):
+    """kvc_ranks_by_salience -> uint8 [2, B, T] (K ranks, V ranks)."""
+    import torch
+
+    B, T = salience.shape
+    ranks = torch.empty((2, B, T), dtype=torch.uint8, device=salience.device)
+    rr = (C.c_int32 * len(rung_ranks))(*[int(x) for x in rung_ranks])
+    rc = (C.c_int32 * max(1, len(rung_counts)))(*[int(x) for x in rung_counts])
+    st = stream if stream is not None else current_stream_ptr()
+    check(lib().kvc_ranks_by_salience(_ptr(salience), B, T, len(rung_ranks), rr, rc, _ptr(ranks),
+                                      st))
+    return ranks
+
+
+def block_keep(salience_layers, keep, stream=None):
+    """kvc_block_keep: salience_layers fp32 [L, B, T] -> (importance [B, T], kept int32 [B, keep])."""
+    import torch
+
+    L, B, T = salience_layers.shape
+    imp = torch.empty((B, T), dtype=torch.float32, device=salience_layers.device)
+    kept = torch.empty((B, int(keep)), dtype=torch.int32, device=salience_layers.device)
+    st = stream if stream is not None else current_stream_ptr()
+    check(lib().kvc_block_keep(_ptr(salience_layers), L, B, T, int(keep), _ptr(imp), _ptr(kept), st))
+    return imp, kept
+
+
+def block_compact(src_layout, src_cache, dst_layout, dst_cache, kept, stream=None):
+    """kvc_block_compact: copy the kept latent rows of src into dst."""
+    a, b = src_cache.struct(), dst_cache.struct()
+    st = stream if stream is not None else current_stream_ptr()
+    check(lib().kvc_block_compact(src_layout.h, C.byref(a), dst_layout.h, C.byref(b), _ptr(kept),
+                                  int(kept.shape[1]), st))
+    dst_cache.n_tokens = int(kept.shape[1])

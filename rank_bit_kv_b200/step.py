@@ -36,6 +36,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--time", action="store_true")
+    ap.add_argument("--rope-kernel", type=int, default=0,
+                    help="pre-RoPE layouts: 0 / 1 warp-level mma.sync kernel, 2 tcgen05 warpgroup kernel")
     args = ap.parse_args(argv)
 
     import numpy as np
@@ -44,6 +46,7 @@ def main(argv=None):
     from rank_bit_kv_b200 import kvc, synth
 
     over = {} if args.batch is None else {"B": args.batch}
+    kvc.lib().kvc_select_rope_kernel(args.rope_kernel)
     c = synth.config(args.config, **over)
     lay, cache, fill = _cache(kvc, synth, c)
     q = torch.from_numpy(np.ascontiguousarray(fill["q"]).view(np.int16)).cuda().view(torch.bfloat16)

@@ -192,19 +192,26 @@ def dense_cache(B, Hq, Hkv, d, T, seed, n_layers=1, capacity=None):
 
 
 def block_shared_cache(c, T=None, capacity=None, rng=None):
-    """q uint16 [L, B, Hq, d]; codes uint8 [B, cap, D/2]; scales fp16 [B, cap, D/g];
-    wk, wv fp16 [L, D, Hkv*d] ~ N(0, 1/D)."""
+    """q uint16 [L, B, Hq, d]; codes uint8 [B, cap, D * bits / 8]; scales fp16
+    [B, cap, D/g] (scaled so that the latent's spread is the same at every
+    width); wk, wv fp16 [L, D, Hkv*d] ~ N(0, 1/D); with c['vbits'] > 0 a value
+    latent lv_codes / lv_sz at that width."""
     rng = rng or np.random.default_rng(c["seed"])
     T = c["T"] if T is None else T
     cap = capacity or T
     L, B, Hq, Hkv, d, D, g = c["L"], c["B"], c["Hq"], c["Hkv"], c["d"], c["D"], c["g"]
-    return dict(
+    bits, vbits = c.get("bits", 4), c.get("vbits", 0)
+    out = dict(
         q=to_bf16_bits(rng.standard_normal((L, B, Hq, d))),
         wk=(rng.standard_normal((L, D, Hkv * d)) / np.sqrt(D)).astype(np.float16),
         wv=(rng.standard_normal((L, D, Hkv * d)) / np.sqrt(D)).astype(np.float16),
-        lk_codes=uniform_codes(rng, (B, cap, D // 2)),
-        lk_sz=rng.uniform(0.30, 0.45, size=(B, cap, D // g)).astype(np.float16),
+        lk_codes=uniform_codes(rng, (B, cap, D * bits // 8)),
+        lk_sz=(rng.uniform(0.30, 0.45, size=(B, cap, D // g)) * 8 / 2 ** (bits - 1)).astype(np.float16),
     )
+    if vbits:
+        out["lv_codes"] = uniform_codes(rng, (B, cap, D * vbits // 8))
+        out["lv_sz"] = (rng.uniform(0.30, 0.45, size=(B, cap, D // g)) * 8 / 2 ** (vbits - 1)).astype(np.float16)
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -258,3 +265,32 @@ def varrate_cache(c, T=None, capacity=None, rng=None, ranks=None):
         out[f"offset_{comp}"] = off.astype(np.int32)
         out[f"{comp}stream"] = stream
     return out
+
+
+# --------------------------------------------------------------------------
+# prefill keys / values and test matrices for the factor fit
+# --------------------------------------------------------------------------
+
+
+def prefill_kv(c, T, rng=None, decay=0.06, noise=0.02):
+    """Pre-RoPE keys and values of a prefill, bf16 bits [B, Hkv, T, d]: per KV
+    head a random orthonormal basis with an exponentially decaying spectrum
+    (component i scaled by exp(-decay * i), as the low effective rank of cached
+    keys and values), plus a small isotropic part."""
+    rng = rng or np.random.default_rng(c["seed"] + 4000)
+    B, Hkv, d = c["B"], c["Hkv"], c["d"]
+    out = []
+    for _ in range(2):
+        x = np.empty((B, Hkv, T, d), np.float32)
+        scale = np.exp(-decay * np.arange(d))
+        for h in range(Hkv):
+            basis, _ = np.linalg.qr(rng.standard_normal((d, d)))
+            z = rng.standard_normal((B, T, d)) * scale
+            x[:, h] = (z @ basis.T + noise * rng.standard_normal((B, T, d))).astype(np.float32)
+        out.append(to_bf16_bits(x))
+    return out[0], out[1]
+
+
+def gaussian_test_matrix(n_heads, d, k, seed):
+    """N(0, 1) test matrices [n_heads, d, k] (fp32) of the randomized range finder."""
+    return np.random.default_rng(seed).standard_normal((n_heads, d, k)).astype(np.float32)

@@ -306,30 +306,58 @@ def test_latent_tensor_core_peaked():
 # ------------------------------------------------------------------ pre-RoPE keys on warp-level MMAs
 
 
+@pytest.fixture(params=["tcgen05_wg", "mma_sync"])
+def rope_kernel(request):
+    """Runs a test on both pre-RoPE kernels: the warp-level mma.sync kernel (the
+    default) and the tcgen05 warpgroup kernel."""
+    from rank_bit_kv_b200 import kvc
+
+    kvc.lib().kvc_select_rope_kernel(1 if request.param == "mma_sync" else 2)
+    yield request.param
+    kvc.lib().kvc_select_rope_kernel(0)
+
+
 @pytest.mark.parametrize("rv,page,Hq,B,n,cap", [
-    (48, 0, 32, 2, 4096, 4096),       # C2 ranks, whole 64-token rotation groups
-    (48, 0, 32, 2, 4001, 4016),       # ragged last tile, partial rotation group
+    (48, 0, 32, 2, 4096, 4096),       # C2 ranks, whole 128-token tiles
+    (48, 0, 32, 2, 4001, 4016),       # ragged last tile, capacity not a multiple of 128
     (48, 0, 32, 1, 1, 16),            # one token
     (32, 16, 16, 3, 1234, 1248),      # paged, two query heads per KV head
     (64, 0, 64, 2, 777, 784),         # eight query heads per KV head
+    (48, 16, 32, 3, 2049, 2064),      # paged, C2 ranks, a unit boundary inside most ranges
 ])
-def test_rope_mma_path(rv, page, Hq, B, n, cap):
+def test_rope_mma_path(rope_kernel, rv, page, Hq, B, n, cap):
     """Pre-RoPE INT4 keys with a capacity that is a multiple of 16 run on the
-    warp-level kernel (reconstruction, rotation and scores on mma.sync); per-row
-    lengths force the generic kernel.  Both must match the oracle."""
+    tensor-core kernels (tcgen05 reconstruction in TMEM, or reconstruction on
+    mma.sync); per-row lengths force the generic kernel.  All match the oracle."""
     c = synth.config("c2", B=B, Hq=Hq, T=cap, rv=rv, page=page, seed=21 + rv)
     a = synth.lowrank_cache(c)
     ref = oracle(c, a, n)
-    assert_close(run_decode(c, a, n, capacity=cap), ref, what=f"rope mma rv={rv} n={n}")
+    assert_close(run_decode(c, a, n, capacity=cap), ref, what=f"{rope_kernel} rv={rv} n={n}")
     got = run_decode(c, a, n, capacity=cap, seq_lens=[n] * B)
     assert_close(got, ref, what=f"generic rv={rv} n={n}")
 
 
-def test_rope_mma_peaked():
+def test_rope_mma_peaked(rope_kernel):
     c = synth.config("c2", B=2, T=2048)
     a = synth.lowrank_cache(c)
     a["q"] = synth.to_bf16_bits(synth.bf16_bits_to_f32(a["q"]) * 8)
-    assert_close(run_decode(c, a, 2048), oracle(c, a, 2048), what="rope mma peaked")
+    assert_close(run_decode(c, a, 2048), oracle(c, a, 2048), what=f"{rope_kernel} peaked")
+
+
+def test_rope_kernels_agree_at_full_size():
+    """The two pre-RoPE tensor-core kernels on the benchmark workload (every
+    row): both within the tolerance of each other's oracle-checked result."""
+    from rank_bit_kv_b200 import kvc
+
+    c = synth.config("c2")
+    a = synth.lowrank_cache(c)
+    got_mma = run_decode(c, a, c["T"])
+    kvc.lib().kvc_select_rope_kernel(2)
+    try:
+        got_wg = run_decode(c, a, c["T"])
+    finally:
+        kvc.lib().kvc_select_rope_kernel(0)
+    assert_close(got_wg, got_mma, what="tcgen05 vs mma.sync, full size")
 
 
 # ------------------------------------------------------------------ variable rate, one lane per head pair
