@@ -265,6 +265,109 @@ def other_workloads(torch, kvc, synth, device, steps, peak_gbs, peak_tflops):
     return res
 
 
+def producer_workloads(torch, kvc, synth, device, steps):
+    """The steps around decode, timed with CUDA events (L2 flushed before each
+    repetition): bulk prefill compression at the Llama-3.1-8B layer's size
+    (randomized-SVD factor fit of K and V, then one kvc_append of every prefill
+    token), the variable-rate producer at its workload's size (window salience
+    of 32 queries per head, ranks by the configured mix), and the joint
+    rank / residual-bit allocation (host) over 64 cells."""
+    import time as _time
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    n = max(3, min(steps, 5))
+    res = {}
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        fn()
+        torch.cuda.synchronize()
+        for i in range(n):
+            flush.fill_(i & 255)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(ts)
+
+    # ---- prefill compression, C2 shape (8 rows x 32768 tokens x 8 KV heads)
+    c = synth.config("c2")
+    # 4096 seeded prefill tokens per row, repeated along the context on the device
+    # (the generator's cost stays small; sizes and spectrum are the workload's)
+    kb, vb = synth.prefill_kv(c, 4096)
+    reps = c["T"] // 4096
+    kd = torch.from_numpy(kb.view(np.int16)).to(device).view(torch.bfloat16).repeat(1, 1, reps, 1)
+    vd = torch.from_numpy(vb.view(np.int16)).to(device).view(torch.bfloat16).repeat(1, 1, reps, 1)
+    del kb, vb
+    omk = torch.from_numpy(synth.gaussian_test_matrix(c["Hkv"], 128, 48, 1)).to(device)
+    omv = torch.from_numpy(synth.gaussian_test_matrix(c["Hkv"], 128, 64, 2)).to(device)
+    lay = kvc.Layout(kvc.desc_from_config(c))
+    cache = kvc.Cache(lay, device=device)
+    pos = torch.zeros(c["B"], dtype=torch.int32, device=device)
+
+    def fit():
+        bk, _ = kvc.fit_factors(kd, omk, c["rk"], 2, with_sigma2=False)
+        bv, _ = kvc.fit_factors(vd, omv, c["rv"], 2, with_sigma2=False)
+        cache.bufs["bk"].copy_(bk.view(torch.uint8).reshape(-1))
+        cache.bufs["bv"].copy_(bv.view(torch.uint8).reshape(-1))
+
+    def app():
+        kvc.append(lay, cache, kd, vd, pos, c["T"])
+
+    fit_us = timed(fit)
+    app_us = timed(app)
+    in_bytes = 2 * kd.numel() * 2
+    res["prefill_c2"] = {
+        "what": "factor fit (randomized SVD, rank 32 / 48, sketch 48 / 64, 2 power iterations) "
+                "of K and V, then kvc_append of all 32768 tokens of 8 rows",
+        "fit_us": round(fit_us, 1), "append_us": round(app_us, 1),
+        "tokens": c["B"] * c["T"], "bf16_input_bytes": in_bytes,
+        "fit_GBps": round(in_bytes / fit_us / 1e3, 1),
+        "append_GBps_in": round(in_bytes / app_us / 1e3, 1)}
+    del kd, vd, cache
+    torch.cuda.empty_cache()
+
+    # ---- variable-rate producer, C4 shape (1 row x 131072 tokens)
+    c4 = synth.config("c4")
+    kb, _ = synth.prefill_kv(c4, 8192)
+    kd = torch.from_numpy(kb.view(np.int16)).to(device).view(torch.bfloat16).repeat(
+        1, 1, c4["T"] // 8192, 1)
+    del kb
+    qw = torch.randn(1, 32, 32, 128, device=device).to(torch.bfloat16)
+    T = c4["T"]
+    counts = [int(T * f) for f in (0.05, 0.10, 0.20, 0.25)]
+    out = {}
+
+    def sal():
+        out["s"] = kvc.window_salience(qw, kd)
+        out["r"] = kvc.ranks_by_salience(out["s"], [64, 32, 16, 8, 4], counts)
+
+    sal_us = timed(sal)
+    res["salience_ranks_c4"] = {
+        "what": "window salience (32 query heads x 32 window queries over 131072 keys, "
+                "two tensor-core passes) + ranks by the {5,10,20,25,40} % mix",
+        "us": round(sal_us, 1), "keys_bytes": kd.numel() * 2,
+        "GBps_keys_per_pass": round(2 * kd.numel() * 2 / sal_us / 1e3, 1)}
+    del kd
+    torch.cuda.empty_cache()
+
+    # ---- joint rank / residual-bit allocation (host), 64 cells x 15 options
+    rng = np.random.default_rng(0)
+    spectra = np.exp(-rng.uniform(0.02, 0.08, (64, 1)) * np.arange(128)[None])
+    opts = [(r, b) for r in (8, 16, 32, 48, 64) for b in (0, 2, 4)]
+    t0 = _time.perf_counter()
+    B_, D_ = kvc.rank_bit_tables(spectra, np.full(64, 32768 * 8), np.full(64, 8), opts, 128, 0.006,
+                                 {0: 1.0, 2: 0.12, 4: 0.01})
+    ch, lam = kvc.allocate_rank_bits(B_, D_, B_.min(1).sum() + 0.4 * (B_.max(1).sum() - B_.min(1).sum()))
+    res["allocator_host"] = {"cells": 64, "options": len(opts),
+                             "us": round((_time.perf_counter() - t0) * 1e6, 1)}
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def _oracle_threads():
     """BLAS threads numpy would use (the oracle's matrix products)."""
     try:
@@ -488,6 +591,7 @@ def run_kvc(args, rank, world, torch, dist):
     if not args.no_others:
         others = other_workloads(torch, kvc, synth, device, K, measured_peaks()[0],
                                  measured_peaks()[1])
+        others.update(producer_workloads(torch, kvc, synth, device, K))
 
     if rank != 0:
         return

@@ -252,6 +252,90 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
 
 }  // namespace
 
+// Block-shared latent: one block per (layer, batch row, KV head) merges the
+// G query heads' partials together and applies the layer's W_v slice to all
+// of them, so each W_v element is read once per block rather than once per
+// query head.  Thread (i, half) forms output dim i of every head over half of
+// the latent columns; the two halves are added at the end.
+constexpr int kBGroup = 8;               // query heads per KV head handled (G <= 8)
+
+__global__ void __launch_bounds__(kThreads) combine_block_kernel(Params p) {
+  extern __shared__ float bsm[];
+  const int D = p.D, d = p.d, G = p.G;
+  float* acc = bsm;                      // [G][D]
+  float* ws = acc + G * D;               // [G][S]
+  float* red = ws + G * p.S;             // [kThreads][G]
+  __shared__ float linv[kBGroup];
+  const int blk = blockIdx.x;            // (l * B + b) * Hkv + kvh
+  const int kvh = blk % p.Hkv, lb = blk / p.Hkv;   // lb = l * B + b
+  const int l = lb / p.B;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t rows = (size_t)p.L * p.B * p.Hq;
+  const int pst = p.vdim + 2;
+  const int nS = p.S;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // split weights and softmax sums of the G rows (warp g: row g)
+  for (int g = warp; g < G; g += kThreads / 32) {
+    const float* part = p.part + ((size_t)lb * p.Hq + kvh * G + g) * pst;
+    float mx = -INFINITY;
+    for (int s = lane; s < nS; s += 32) mx = fmaxf(mx, part[(size_t)s * rows * pst + D]);
+    mx = warp_max(mx);
+    float lt = 0.f;
+    for (int s = lane; s < nS; s += 32) {
+      const float* ps = part + (size_t)s * rows * pst;
+      const float w = (mx == -INFINITY) ? 0.f : exp2f(ps[D] - mx);
+      ws[g * nS + s] = w;
+      if (w != 0.f) lt += w * ps[D + 1];
+    }
+    lt = warp_sum(lt);
+    if (lane == 0) linv[g] = lt > 0.f ? 1.f / lt : 0.f;
+  }
+  __syncthreads();
+  // merged accumulators of the G rows
+  for (int e = tid; e < G * D; e += kThreads) {
+    const int g = e / D, c = e % D;
+    const float* part = p.part + ((size_t)lb * p.Hq + kvh * G + g) * pst + c;
+    float a = 0.f;
+    for (int s = 0; s < nS; ++s) {
+      const float w = ws[g * nS + s];
+      if (w != 0.f) a = fmaf(w, part[(size_t)s * rows * pst], a);
+    }
+    acc[e] = a;
+  }
+  __syncthreads();
+  // up-projection o_g = acc_g W_v^l[:, kvh slice] / l_g
+  const __half* w = p.bv + (int64_t)l * D * p.Hkv * d + kvh * d;
+  for (int i0 = 0; i0 < d; i0 += kThreads / 2) {
+    const int i = i0 + tid % (kThreads / 2), half = tid / (kThreads / 2);
+    float o[kBGroup];
+#pragma unroll
+    for (int g = 0; g < kBGroup; ++g) o[g] = 0.f;
+    if (i < d) {
+      const int c0 = half * (D / 2), c1 = c0 + D / 2;
+#pragma unroll 4
+      for (int c = c0; c < c1; ++c) {
+        const float wv = h2f(w[(int64_t)c * p.Hkv * d + i]);
+#pragma unroll
+        for (int g = 0; g < kBGroup; ++g)
+          if (g < G) o[g] = fmaf(acc[g * D + c], wv, o[g]);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kBGroup; ++g)
+      if (g < G) red[tid * G + g] = o[g];
+    __syncthreads();
+    if (tid < kThreads / 2 && i < d) {
+      for (int g = 0; g < G; ++g) {
+        const float t = (red[tid * G + g] + red[(tid + kThreads / 2) * G + g]) * linv[g];
+        const int64_t orow = (int64_t)lb * p.Hq + kvh * G + g;
+        if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[orow * d + i] = __float2bfloat16_rn(t);
+        else reinterpret_cast<float*>(p.out)[orow * d + i] = t;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   if (p.S > kMaxS) return cudaErrorInvalidValue;
   const int rows = p.L * p.B * p.Hq;
@@ -276,6 +360,15 @@ cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (p.kind == KVC_BLOCK_SHARED && p.G <= kBGroup && p.seg_W == 0) {
+    const size_t bb = ((size_t)p.G * p.D + (size_t)p.G * p.S + (size_t)kThreads * p.G) * sizeof(float);
+    e = cudaFuncSetAttribute(combine_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bb);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(p.L * p.B * p.Hkv);
+    cfg.dynamicSmemBytes = bb;
+    return cudaLaunchKernelEx(&cfg, combine_block_kernel, p);
+  }
   if (small) return cudaLaunchKernelEx(&cfg, combine_lowrank_kernel<16, 2>, p);
   if (fast) return cudaLaunchKernelEx(&cfg, combine_lowrank_kernel<40, 5>, p);
   return cudaLaunchKernelEx(&cfg, combine_kernel, p);

@@ -15,8 +15,10 @@
 //      q . R_t k = q_rot . R_delta k) -- no per-token sin/cos,
 //   5. scores S = K'' q_rot^T and accumulates acc^T += L_v^T P with warp-level
 //      mma.sync (m16n8k16): these products have N = 4 query heads, and a
-//      tcgen05 MMA costs the same ~135 SM cycles per K = 16 step whatever its
-//      N, so only the N = 128 reconstruction runs on tcgen05,
+//      tcgen05 MMA with M = 128 keeps the tensor pipe busy for about N / 2
+//      cycles per K = 16 step but no fewer than ~48 (measured: 48 at N = 64,
+//      65 at N = 128, 128 at N = 256), so only the N = 128 reconstruction runs
+//      on tcgen05,
 //   6. keeps an online softmax per warp with a lazily raised reference
 //      maximum (rescaling only when a score exceeds it by 2^8),
 // and writes one partial (acc, m, l) per warp and unit that the split combine
