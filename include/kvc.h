@@ -242,7 +242,8 @@ size_t kvc_step_bytes(const kvc_layout* layout, int32_t n_tokens);
  * pages (split-T partials are this library's design).  0 for NULL. */
 size_t kvc_workspace_bytes(const kvc_layout* layout, int32_t n_tokens);
 
-/* Number of kernel launches one kvc_decode_attn call makes for n_tokens. */
+/* Number of kernel launches one kvc_decode_attn call makes for n_tokens with
+ * uniform lengths (per-row lengths may add the query projection). */
 int32_t kvc_decode_launches(const kvc_layout* layout, int32_t n_tokens);
 
 /* Append n_new tokens to every batch row: project each new pre-RoPE key and
@@ -305,7 +306,8 @@ kvc_status kvc_append(const kvc_layout* layout, const kvc_cache* cache,
  *      call is invalid.  Read it after the stream has completed.
  * Host-detectable errors (NULL, misalignment, n_tokens beyond max_tokens, a
  * small workspace, missing cache buffers) return before anything is enqueued.
- * Launches kvc_decode_launches() kernels: a query projection, the split-T
+ * Launches kvc_decode_launches() kernels: a query projection (where the
+ * layout needs one and the split kernel does not form it itself), the split-T
  * fused decode over the compressed tiles, and the split combine with the
  * up-projection (on some paths a zeroing of the error word precedes them). */
 kvc_status kvc_decode_attn(const kvc_layout* layout, const kvc_cache* cache,

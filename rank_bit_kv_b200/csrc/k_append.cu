@@ -14,6 +14,10 @@
 // between the group's extremes, each value coded by its nearest step, here with
 // the step and the offset stored in fp16.
 //
+// A bulk append of INT4 rows without the residual (prefill) stages the factor
+// once per block of tokens and gives each token to one warp; the arithmetic is
+// the same, term by term.
+//
 // pos and the VARRATE ranks are device arrays, so the kernels validate them:
 // rows with a slot range outside the cache, tokens with a bad rank or page id,
 // and records that would run past their stream are skipped (never written out
@@ -291,13 +295,120 @@ __global__ void append_dense_kernel(AppendParams a) {
   }
 }
 
+// Bulk append (prefill) of INT4 low-rank rows without the residual: one block
+// per (chunk of kBulkTok tokens, batch row, KV head, K or V).  The factor rows
+// are staged once in shared memory as fp32, rows padded to 129 floats so that
+// lane j reading row j is conflict-free; warp w takes tokens w, w + 8, ... of
+// the chunk, lane j forms latent entries j and j + 32 with the summation order
+// of append_lowrank_kernel (so the codes are the same), then the group's
+// minimum and maximum by shuffles and the codes, two per byte.
+constexpr int kBulkTok = 256;
+constexpr int kBulkThreads = 256;
+
+__global__ void __launch_bounds__(kBulkThreads) append_lowrank_bulk_kernel(AppendParams a) {
+  const Params& p = a.p;
+  extern __shared__ float fs[];                  // [r][129] factor rows, then x [8][128]
+  const int chunk = blockIdx.x;
+  int idx = blockIdx.y;                          // (b * Hkv + h) * 2 + comp
+  const int comp = idx & 1;
+  idx >>= 1;
+  const int h = idx % p.Hkv, b = idx / p.Hkv;
+  const int p0 = first_slot(a, b);
+  if (p0 < 0) {
+    if (threadIdx.x == 0 && h == 0 && comp == 0 && chunk == 0) flag(a.status, KVC_DEV_BAD_POS);
+    return;
+  }
+  const int r = comp == 0 ? p.rk : p.rv;
+  const int ng = (r + 31) / 32;
+  const __half* fac = (comp == 0 ? p.bk : p.bv) + (int64_t)h * r * 128;
+  for (int e = threadIdx.x; e < r * 128; e += kBulkThreads) fs[(e >> 7) * 129 + (e & 127)] = h2f(fac[e]);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* xs = fs + r * 129 + warp * 128;
+  __syncthreads();
+  for (int ti = warp; ti < kBulkTok; ti += kBulkThreads / 32) {
+    const int i = chunk * kBulkTok + ti;
+    if (i >= a.n_new) break;
+    const int tok = p0 + i;
+    if (p.page) {
+      const int pp = p.page_table[(int64_t)b * (p.tmax / p.page) + tok / p.page];
+      if (pp < 0 || pp >= p.n_pages) {
+        if (lane == 0 && h == 0 && comp == 0) flag(a.status, KVC_DEV_BAD_PAGE);
+        continue;
+      }
+    }
+    const __nv_bfloat16* src =
+        (comp == 0 ? a.k_new : a.v_new) + (((int64_t)b * p.Hkv + h) * a.n_new + i) * 128;
+    {
+      const uint2 u = *reinterpret_cast<const uint2*>(src + 4 * lane);
+      const __nv_bfloat162 x01 = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+      const __nv_bfloat162 x23 = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+      xs[4 * lane] = __low2float(x01);
+      xs[4 * lane + 1] = __high2float(x01);
+      xs[4 * lane + 2] = __low2float(x23);
+      xs[4 * lane + 3] = __high2float(x23);
+    }
+    __syncwarp();
+    float lat[2] = {0.f, 0.f};
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const int j = lane + 32 * gi;
+      if (j < r) {
+        const float* br = fs + j * 129;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < 128; ++k) acc = fmaf(xs[k], br[k], acc);
+        lat[gi] = acc;
+      }
+    }
+    const int64_t row = lowrank_row(p, b, h, tok);
+    uint8_t* codes = (comp == 0 ? a.lk_w : a.lv_w) + row * (r / 2);
+    __half* sz = (comp == 0 ? a.lksz_w : a.lvsz_w) + row * 2 * ng;
+    for (int gi = 0; gi < ng; ++gi) {
+      const int j = lane + 32 * gi;
+      const bool in = j < r;
+      const float v = gi == 0 ? lat[0] : lat[1];
+      float lo = in ? v : INFINITY, hi = in ? v : -INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      }
+      const __half zh = __float2half_rn(lo);
+      const __half sh = __float2half_rn((hi - lo) / 15.f);
+      const float s = __half2float(sh), z = __half2float(zh);
+      int c = 0;
+      if (in && s > 0.f) c = (int)fminf(fmaxf(rintf((v - z) / s), 0.f), 15.f);
+      const int cn = __shfl_down_sync(0xffffffffu, c, 1);
+      if (in && !(lane & 1)) codes[j >> 1] = (uint8_t)(c | (cn << 4));
+      if (lane == 0) {
+        sz[2 * gi] = sh;
+        sz[2 * gi + 1] = zh;
+      }
+    }
+    __syncwarp();                                // xs is rewritten by the next token
+  }
+}
+
+bool bulk_ok(const AppendParams& a) {
+  const Params& p = a.p;
+  return p.kind == KVC_LOWRANK && p.bits == 4 && p.g == 32 && !p.resid && p.d == 128 &&
+         p.rk <= 64 && p.rv <= 64 && a.n_new >= 64;
+}
+
 }  // namespace
 
 cudaError_t launch_append(const AppendParams& a, cudaStream_t s) {
   const Params& p = a.p;
   switch (p.kind) {
     case KVC_LOWRANK:
-      append_lowrank_kernel<<<p.B * p.Hkv * 2 * a.n_new, kThreads, 0, s>>>(a);
+      if (bulk_ok(a)) {
+        const int rmax = p.rk > p.rv ? p.rk : p.rv;
+        const size_t smem = ((size_t)rmax * 129 + 8 * 128) * sizeof(float);
+        dim3 grid((a.n_new + kBulkTok - 1) / kBulkTok, p.B * p.Hkv * 2);
+        append_lowrank_bulk_kernel<<<grid, kBulkThreads, smem, s>>>(a);
+      } else {
+        append_lowrank_kernel<<<p.B * p.Hkv * 2 * a.n_new, kThreads, 0, s>>>(a);
+      }
       break;
     case KVC_VARRATE:
       varrate_offsets_kernel<<<p.B * 2, 32, 0, s>>>(a);

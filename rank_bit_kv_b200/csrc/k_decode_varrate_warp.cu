@@ -4,10 +4,15 @@
 // A token's rank is shared by all KV heads, so every lane of a warp takes the
 // same rank branch for the same token.  The 8 KV heads x 4 query heads of a
 // batch row fill the 32 lanes; each lane keeps its own online softmax (no
-// shuffles) and its own latent-space accumulator acc[64] in registers:
+// shuffles) and its own latent-space accumulator acc[64] in registers; the
+// projected queries q~ = Bk q are formed by the CTA itself (one thread per
+// (KV head, rank) row of Bk, all four query heads of the group) into shared
+// memory, where each lane reads its own row:
 //   s_t = sum_{i < r_k(t)} q~_i (c_i s_g + z_g),
 //   acc_i += p_t (c_i s_g + z_g) for i < r_v(t).
-// Every warp streams a contiguous token range in chunks of 16 tokens: the byte
+// Keeping q~ out of the registers lets 16 warps share an SM (4 per scheduler)
+// to hide the per-token dependency chain.
+// Every warp streams a contiguous token range in chunks of 8 tokens: the byte
 // range of the chunk's K records and of its V records (contiguous in the
 // per-row streams) is copied with 16-byte cp.async into a double-buffered
 // per-warp area while the previous chunk is processed.  The warps of a CTA
@@ -23,18 +28,23 @@ namespace {
 
 using namespace tc;
 
-constexpr int kVWarps = 8;
+constexpr int kVWarps = 16;
 constexpr int kVThreads = 32 * kVWarps;
-constexpr int kVChunk = 16;                         // tokens per staged chunk
+constexpr int kVChunk = 8;                          // tokens per staged chunk
 constexpr int kVHkv = 8, kVG = 4;                   // lanes = KV heads x query heads
 constexpr int kVRmax = 64;
 constexpr int kVRecMax = kVHkv * (kVRmax / 2 + 8);  // token record bytes at rank 64
 constexpr int kVBuf = kVChunk * kVRecMax + 32;      // one staged stream chunk (+ alignment slack)
 constexpr int kVWarpBytes = 4 * kVBuf;              // K and V, two buffers each
-constexpr int kVSmem = kVWarps * kVWarpBytes;
+constexpr int kVStage = kVWarps * kVWarpBytes;
+constexpr int kVQRow = kVRmax + 4;                  // floats per q~ row (16-byte loads conflict-free)
+constexpr int kVOffQ = kVStage;                     // q~ [32][kVQRow] (softmax scale, log2 e folded)
+constexpr int kVOffX = kVOffQ + 32 * kVQRow * 4;    // the group's queries [32][128] fp32
+constexpr int kVSmem = kVOffX + 32 * 128 * 4;
 constexpr int kVPst = kVRmax + 2;                   // merge slot: acc[64], m, l
 
-static_assert(kVWarps * 32 * kVPst * 4 <= kVSmem, "merge area fits in the staging area");
+static_assert(kVWarps * 32 * kVPst * 4 <= kVStage, "merge area fits in the staging area");
+static_assert(kVThreads == kVHkv * kVRmax, "one thread per (KV head, rank) row of Bk");
 
 __host__ __device__ constexpr int head_bytes(int r) { return r / 2 + 4 * ((r + 31) / 32); }
 
@@ -70,29 +80,35 @@ __device__ __forceinline__ float2 h2f2(uint32_t x) {
 
 // sum_{i < R} q_i (c_i s_g + z_g) over the record at rec (R/2 code bytes, then
 // the groups' (scale, zero) pairs); pre = prefix sums of q
+// (q = this lane's row of q~ in shared memory)
 template <int R>
-__device__ __forceinline__ float score_r(const uint8_t* rec, const float (&q)[kVRmax],
+__device__ __forceinline__ float score_r(const uint8_t* rec, const float* q,
                                          const float (&pre)[5]) {
   if constexpr (R == 4) {
     const uint32_t w = *reinterpret_cast<const uint16_t*>(rec);
     const float s = __half2float(*reinterpret_cast<const __half*>(rec + 2));
     const float z = __half2float(*reinterpret_cast<const __half*>(rec + 4));
+    const float4 q0 = *reinterpret_cast<const float4*>(q);
     float c[8];
     nib8(w, c);
-    float d = c[0] * q[0];
-#pragma unroll
-    for (int k = 1; k < 4; ++k) d = fmaf(c[k], q[k], d);
+    float d = c[0] * q0.x;
+    d = fmaf(c[1], q0.y, d);
+    d = fmaf(c[2], q0.z, d);
+    d = fmaf(c[3], q0.w, d);
     return fmaf(s, d, z * pre[0]);
   } else {
     constexpr int NW = R / 8;
     float dw[NW];                       // one chain per code word (short dependency chains)
 #pragma unroll
     for (int wi = 0; wi < NW; ++wi) {
+      const float4 qa = *reinterpret_cast<const float4*>(q + 8 * wi);
+      const float4 qb = *reinterpret_cast<const float4*>(q + 8 * wi + 4);
+      const float qq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
       float c[8];
       nib8(*reinterpret_cast<const uint32_t*>(rec + 4 * wi), c);
-      float a = c[0] * q[8 * wi];
+      float a = c[0] * qq[0];
 #pragma unroll
-      for (int k = 1; k < 8; ++k) a = fmaf(c[k], q[8 * wi + k], a);
+      for (int k = 1; k < 8; ++k) a = fmaf(c[k], qq[k], a);
       dw[wi] = a;
     }
     float d[2] = {0.f, 0.f};
@@ -156,8 +172,7 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   const int cta_a = s_idx * split_len, cta_b = min(T, cta_a + split_len);
   const int per_warp = (split_len + kVWarps - 1) / kVWarps;
   const int t_a = min(cta_b, cta_a + warp * per_warp), t_b = min(cta_b, t_a + per_warp);
-  const int h = lane >> 2, qi = lane & 3;
-  const size_t row = (size_t)b * p.Hq + h * kVG + qi;
+  const int h = lane >> 2;
 
   uint8_t* const area = vsm + warp * kVWarpBytes;
   const uint32_t area_s = smem_u32(area);
@@ -169,14 +184,42 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   const uint8_t* const rv = p.rank_v + (size_t)b * p.tmax;
   const long long sbytes = (long long)p.stream_bytes;
 
-  // ---- this lane's query (softmax scale and log2 e folded in) and its prefix sums
-  float q[kVRmax], pre[5];
+  // ---- q~ = Bk q for the row's 32 query heads (softmax scale and log2 e
+  // folded in): thread (kvh, j) dots row j of head kvh's Bk with its 4 queries
+  float* const qsm = reinterpret_cast<float*>(vsm + kVOffQ);
   {
-    const float* qt = p.qt + row * p.qdim;
-    float run = 0.f;
+    float* const xs = reinterpret_cast<float*>(vsm + kVOffX);
+    for (int e = threadIdx.x; e < 32 * 128; e += kVThreads)
+      xs[e] = bf2f(p.q[(size_t)b * p.Hq * 128 + e]);
+    __syncthreads();
+    const int kvh = threadIdx.x / kVRmax, j = threadIdx.x % kVRmax;
+    const uint4* br = reinterpret_cast<const uint4*>(p.bk + ((size_t)kvh * kVRmax + j) * 128);
+    float a4[kVG] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+      const uint4 w = __ldg(br + c);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = h2f2(ws[k]);
+#pragma unroll
+        for (int g = 0; g < kVG; ++g) {
+          const float* xg = xs + (kvh * kVG + g) * 128 + 8 * c + 2 * k;
+          a4[g] = fmaf(f.x, xg[0], a4[g]);
+          a4[g] = fmaf(f.y, xg[1], a4[g]);
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kVG; ++g) qsm[(kvh * kVG + g) * kVQRow + j] = a4[g] * p.scale_log2;
+    __syncthreads();
+  }
+  const float* const q = qsm + lane * kVQRow;       // lane = h * 4 + qi
+  float pre[5];
+  {
+    float run = 0.f;
+#pragma unroll 8
     for (int i = 0; i < kVRmax; ++i) {
-      q[i] = qt[i] * p.scale_log2;
       if (i == 32) run = 0.f;
       run += q[i];
       if (i == 3) pre[0] = run;
@@ -289,7 +332,7 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   __syncthreads();
   const size_t rows = (size_t)p.L * p.B * p.Hq;
   const int pst = p.vdim + 2;
-  const int ls = threadIdx.x >> 3, pp = threadIdx.x & 7;    // lane slot, part of its values
+  const int ls = threadIdx.x >> 4, pp = threadIdx.x & 15;   // lane slot, part of its values
   float M = -INFINITY;
 #pragma unroll
   for (int w = 0; w < kVWarps; ++w) M = fmaxf(M, mg[(w * 32 + ls) * kVPst + kVRmax]);
@@ -302,7 +345,7 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   }
   const size_t orow = (size_t)b * p.Hq + (ls >> 2) * kVG + (ls & 3);
   float* dst = p.part + ((size_t)s_idx * rows + orow) * pst;
-  for (int i = pp; i < kVRmax; i += 8) {
+  for (int i = pp; i < kVRmax; i += 16) {
     float a = 0.f;
 #pragma unroll
     for (int w = 0; w < kVWarps; ++w) a = fmaf(wt[w], mg[(w * 32 + ls) * kVPst + i], a);

@@ -155,16 +155,20 @@ __device__ void gemm_G(const double* __restrict__ G, const double* X, double* Y,
 }
 
 // Orthonormalise the k columns of W (d x k) by classical Gram-Schmidt applied
-// twice per column; red = shared scratch of at least k doubles.
+// twice per column; red = shared scratch of at least d + 1 doubles.  The dot
+// products of a pass are spread over the warps (lanes split the d entries).
 __device__ void orthonormalise(double* W, int k, double* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int j = 0; j < k; ++j) {
     double* wj = W + (size_t)j * kFD;
     for (int pass = 0; pass < 2; ++pass) {
-      for (int l = threadIdx.x; l < j; l += blockDim.x) {
+      for (int l = warp; l < j; l += nw) {
         const double* wl = W + (size_t)l * kFD;
         double s = 0.0;
-        for (int i = 0; i < kFD; ++i) s += wl[i] * wj[i];
-        red[l] = s;
+        for (int i = lane; i < kFD; i += 32) s += wl[i] * wj[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) red[l] = s;
       }
       __syncthreads();
       for (int i = threadIdx.x; i < kFD; i += blockDim.x) {
@@ -174,10 +178,12 @@ __device__ void orthonormalise(double* W, int k, double* red) {
       }
       __syncthreads();
     }
-    if (threadIdx.x == 0) {
+    if (warp == 0) {
       double s = 0.0;
-      for (int i = 0; i < kFD; ++i) s += wj[i] * wj[i];
-      red[kFD] = s > 0.0 ? 1.0 / sqrt(s) : 0.0;
+      for (int i = lane; i < kFD; i += 32) s += wj[i] * wj[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) red[kFD] = s > 0.0 ? 1.0 / sqrt(s) : 0.0;
     }
     __syncthreads();
     const double inv = red[kFD];
@@ -271,9 +277,35 @@ __global__ void __launch_bounds__(kSThreads) rsvd_small_kernel(
   }
   __syncthreads();
   // cyclic Jacobi, round-robin pairing (k even): every round rotates k / 2
-  // disjoint pairs; a fixed number of sweeps (quadratic convergence)
+  // disjoint pairs; at most kFitSweeps sweeps (quadratic convergence), fewer
+  // once the off-diagonal mass is negligible against the diagonal
   const int half = k / 2;
   for (int sweep = 0; sweep < kFitSweeps; ++sweep) {
+    {
+      double off = 0.0, dia = 0.0;
+      for (int e = tid; e < k * k; e += nth) {
+        const double v = C[e] * C[e];
+        if (e / k == e % k) dia += v;
+        else off += v;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        off += __shfl_xor_sync(0xffffffffu, off, o);
+        dia += __shfl_xor_sync(0xffffffffu, dia, o);
+      }
+      if ((tid & 31) == 0) {
+        red[2 * (tid >> 5)] = off;
+        red[2 * (tid >> 5) + 1] = dia;
+      }
+      __syncthreads();
+      double offs = 0.0, dias = 0.0;
+      for (int w = 0; w < nth / 32; ++w) {
+        offs += red[2 * w];
+        dias += red[2 * w + 1];
+      }
+      __syncthreads();
+      if (offs <= 1e-30 * dias) break;
+    }
     for (int round = 0; round < k - 1; ++round) {
       auto member = [&](int pos) { return pos == 0 ? 0 : 1 + (pos - 1 + round) % (k - 1); };
       for (int q = tid; q < half; q += nth) {

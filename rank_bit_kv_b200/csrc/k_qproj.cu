@@ -107,11 +107,53 @@ __global__ void __launch_bounds__(kThreads) qproj_group_kernel(Params p) {
   }
 }
 
+// Block-shared latent, head dim 128: one block per (layer, batch row, KV head)
+// forms the absorbed queries of the whole query group, reading each row of the
+// layer's W_k slice once (thread c: latent columns c, c + 256, ...).
+__global__ void __launch_bounds__(256) qproj_block_kernel(Params p) {
+  __shared__ __align__(16) float qs[8][128];
+  const int unit = blockIdx.x;             // (l * B + b) * Hkv + kvh
+  const int kvh = unit % p.Hkv;
+  const int l = unit / (p.B * p.Hkv);
+  const int row0 = (unit / p.Hkv) * p.Hq + kvh * p.G;   // first query row of the group
+  const int tid = threadIdx.x, G = p.G;
+  for (int e = tid; e < G * 128; e += 256)
+    qs[e >> 7][e & 127] = bf2f(p.q[(int64_t)(row0 + (e >> 7)) * 128 + (e & 127)]);
+  __syncthreads();
+  const __half* w = p.bk + (int64_t)l * p.D * p.Hkv * 128 + kvh * 128;
+  for (int c = tid; c < p.D; c += 256) {
+    const uint4* wr = reinterpret_cast<const uint4*>(w + (int64_t)c * p.Hkv * 128);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+    for (int k = 0; k < 16; ++k) {
+      const uint4 u = __ldg(wr + k);
+      const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[j]));
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          if (g < G) {
+            acc[g] = fmaf(f.x, qs[g][8 * k + 2 * j], acc[g]);
+            acc[g] = fmaf(f.y, qs[g][8 * k + 2 * j + 1], acc[g]);
+          }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+      if (g < G) p.qt[(int64_t)(row0 + g) * p.qdim + c] = acc[g];
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_qproj(const Params& p, cudaStream_t s) {
   if ((p.kind == KVC_LOWRANK || p.kind == KVC_VARRATE) && p.d == 128 && p.G <= 8) {
     qproj_group_kernel<<<p.L * p.B * p.Hkv, kThreads, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  if (p.kind == KVC_BLOCK_SHARED && p.d == 128 && p.G <= 8) {
+    qproj_block_kernel<<<p.L * p.B * p.Hkv, 256, 0, s>>>(p);
     return cudaGetLastError();
   }
   const int rows = p.L * p.B * p.Hq;

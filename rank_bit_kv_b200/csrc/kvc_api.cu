@@ -100,6 +100,8 @@ size_t ws_bytes(const kvc_layout* L, int n_tokens) {
   if (L->d.kind == KVC_BLOCK_SHARED) {
     const int Sb = kvc::block_mma_slots(L->d.batch, L->L, L->d.n_q_heads, nt1);
     if (Sb > S) S = Sb;
+    const int St = kvc::block_tc_slots(L->d.batch, nt1);
+    if (St > S) S = St;
   }
   const size_t rows = (size_t)L->L * L->d.batch * L->d.n_q_heads;
   size_t b = kWsHeader + round_up(rows * L->qdim * sizeof(float), 256);
@@ -127,7 +129,7 @@ void kvc_test_skip_tile_copies(int32_t on) { g_test_no_copies = on ? 1 : 0; }
 
 void kvc_select_rope_kernel(int32_t which) { g_rope_kernel = which == 2 ? 2 : 0; }
 
-const char* kvc_version(void) { return "kvc 0.3 (sm_100a; decode kernels rev 12)"; }
+const char* kvc_version(void) { return "kvc 0.3 (sm_100a; decode kernels rev 13)"; }
 
 kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out) {
   if (!desc || !out) return fail(KVC_EINVAL, "kvc_create_layout: NULL argument");
@@ -336,9 +338,14 @@ size_t kvc_workspace_bytes(const kvc_layout* L, int32_t n_tokens) {
 
 int32_t kvc_decode_launches(const kvc_layout* L, int32_t n_tokens) {
   if (!L) return 0;
-  kvc::Params p;
+  kvc::Params p = {};
   p.kind = L->d.kind;
   p.rope = L->d.rope;
+  // uniform lengths: the variable-rate layout of 8 KV heads x 4 query heads
+  // runs the warp kernel, which projects its own queries
+  if (p.kind == KVC_VARRATE && L->d.n_kv_heads == 8 && L->d.n_q_heads == 32 &&
+      L->d.group_size == 32 && n_tokens > 0)
+    p.path = 5;
   return 2 + (kvc::needs_qproj(p) ? 1 : 0);
 }
 
@@ -539,6 +546,9 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
       // fixed token splits per batch row (one partial per CTA)
       kvc::varrate_warp_plan(p, &p.S, &p.split_len);
       p.path = 5;
+    } else if (kvc::block_tc_supported(p)) {
+      kvc::block_tc_plan(p, &p.S, &p.split_len);
+      p.path = 8;
     } else if (kvc::block_mma_supported(p)) {
       kvc::block_mma_plan(p, &p.S, &p.split_len);
       p.path = 6;

@@ -64,7 +64,7 @@ struct Params {
   int seg_W, seg_tpu;
   int seg_parts;         // partials written per CTA and unit on that path
   int path;              // split kernel: 0 generic, 1 rope_tc, 2 dense_tc, 3 latent_tc, 4 rope_mma,
-                         // 5 varrate_warp, 6 block_mma, 7 rope_wg
+                         // 5 varrate_warp, 6 block_mma, 7 rope_wg, 8 block_tc
   uint32_t* err;         // error word of the workspace (bounded waits that gave up)
   int test_no_copies;    // test switch: the tcgen05 producer issues no tile copies
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
@@ -153,6 +153,13 @@ void block_mma_plan(const Params& p, int* splits, int* split_len);
 int block_mma_slots(int batch, int n_layers, int n_q_heads, int n_tokens);
 cudaError_t launch_block_mma(const Params& p, cudaStream_t s);
 
+// block-shared latent on tcgen05: all 128 absorbed queries of a batch row per
+// CTA, one CTA per half of the latent columns
+bool block_tc_supported(const Params& p);
+void block_tc_plan(const Params& p, int* splits, int* split_len);
+int block_tc_slots(int batch, int n_tokens);
+cudaError_t launch_block_tc(const Params& p, cudaStream_t s);
+
 // factor fit by randomized SVD (bulk prefill compression)
 constexpr int kFitChunks = 64;        // Gram partials (CTAs) per KV head
 constexpr int kFitMaxK = 96;          // largest sketch width (rank + oversampling)
@@ -204,15 +211,16 @@ cudaError_t launch_combine(const Params& p, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& a, cudaStream_t s);
 
 // Whether the decode of this layout runs a query projection first.
+// (The variable-rate warp kernel, path 5, projects its queries itself.)
 __host__ __device__ inline bool needs_qproj(const Params& p) {
-  return p.kind == KVC_VARRATE || p.kind == KVC_BLOCK_SHARED ||
+  return (p.kind == KVC_VARRATE && p.path != 5) || p.kind == KVC_BLOCK_SHARED ||
          (p.kind == KVC_LOWRANK && !p.rope);
 }
 
 // Whether the chosen split kernel has bounded waits that can set the
 // workspace error word (the call zeroes the word first only then).
 __host__ __device__ inline bool path_sets_error_word(const Params& p) {
-  return p.path == 1 || p.path == 7;
+  return p.path == 1 || p.path == 7 || p.path == 8;
 }
 
 }  // namespace kvc

@@ -37,8 +37,11 @@ def run_decode(cfg, arrays, n_tokens, capacity=None, out_bf16=0, seq_lens=None, 
     out = torch.empty(qt.shape, device="cuda",
                       dtype=torch.bfloat16 if out_bf16 else torch.float32)
     ws = torch.empty(max(lay.workspace_bytes(n_tokens), 16), dtype=torch.uint8, device="cuda")
+    ws[:16].zero_()
     kvc.decode(lay, cache, qt, out, ws)
     torch.cuda.synchronize()
+    # word 0 of the workspace: a bounded wait of a tensor-core kernel gave up
+    assert int(ws[:4].view(torch.int32).item()) == 0, "decode error word set"
     return out.float().cpu().numpy()
 
 

@@ -120,6 +120,36 @@ def test_lowrank_append_bit_exact(name, n_new):
                     assert not ((gotc != ref["rcodes"]) & eok).any(), f"{name} {comp} residual codes"
 
 
+def test_lowrank_bulk_append_bit_exact():
+    """A prefill-sized append (n_new >= 64) runs the bulk kernel (factor staged
+    once per block, one warp per token); its codes must equal the oracle's
+    quantizer on every appended token, as the per-token kernel's do."""
+    c = synth.config("c2", B=2, T=512)
+    a = synth.lowrank_cache(c, T=512)
+    lay = kvc.Layout(kvc.desc_from_config(c, capacity=512))
+    cache = kvc.Cache(lay, fill=a)
+    n_new, pos = 300, [7, 200]
+    kn, vn = synth.new_tokens(c, n_new)
+    kvc.append(lay, cache, to_dev_bf16(kn), to_dev_bf16(vn), pos, n_new)
+    torch.cuda.synchronize()
+    g = c["g"]
+    rows = a["lk_codes"].shape[:3]
+    for comp, x_bits, r in (("k", kn, c["rk"]), ("v", vn, c["rv"])):
+        codes = fetch(cache, f"l{comp}_codes", np.uint8, rows + (r // 2,))
+        sz = fetch(cache, f"l{comp}_sz", np.float16, rows + (O.n_groups(r, g), 2))
+        fac = a[f"b{comp}"].astype(np.float64)
+        x = O.bf16_bits_to_f64(x_bits)                            # [B, Hkv, n_new, d]
+        for b in range(c["B"]):
+            t = np.arange(pos[b], pos[b] + n_new)
+            lat = np.einsum("hid,hrd->ihr", x[b], fac)            # [n_new, Hkv, r]
+            for i in range(n_new):
+                check_int4(codes[b, :, t[i]], sz[b, :, t[i]], lat[i], g, f"bulk {comp} b{b} i{i}")
+        # slots outside the appended range keep their previous contents
+        before = a[f"l{comp}_codes"]
+        np.testing.assert_array_equal(codes[0, :, :pos[0]], before[0, :, :pos[0]])
+        np.testing.assert_array_equal(codes[1, :, pos[1] + n_new:], before[1, :, pos[1] + n_new:])
+
+
 def test_fp16_latent_append():
     c = synth.config("c1")
     a = synth.lowrank_cache(c, T=16)

@@ -223,19 +223,23 @@ def test_c4_full_size():
     assert_close(run_decode(c, a, c["T"]), oracle(c, a, c["T"]), what="c4 full")
 
 
-def test_c3_full_size_sampled():
+def test_c3_full_size_every_row():
+    """Every batch row at full size (KV heads 0 and 7 of each: the oracle's
+    per-head reconstruction is the cost)."""
     c = synth.config("c3")
     a = synth.block_shared_cache(c)
     got = run_decode(c, a, c["T"])
     T, d = c["T"], c["d"]
-    codes = O.unpack_int4(a["lk_codes"][[1], :T], c["D"])
-    lat = O.dequant_int4_sym(codes, a["lk_sz"][[1], :T].astype(np.float64), c["g"])
-    for kvh in (0, 7):
-        sl = slice(kvh * d, (kvh + 1) * d)
-        q = O.bf16_bits_to_f64(a["q"][:, [1], kvh * 4:(kvh + 1) * 4])     # [L, 1, 4, d]
-        ref = O.decode_block_shared(q, lat, a["wk"][:, :, sl].astype(np.float64),
-                                    a["wv"][:, :, sl].astype(np.float64), 1, 1 / np.sqrt(d))
-        assert_close(got[:, 1:2, kvh * 4:(kvh + 1) * 4], ref, what=f"c3 full kvh={kvh}")
+    for b in range(c["B"]):
+        codes = O.unpack_int4(a["lk_codes"][[b], :T], c["D"])
+        lat = O.dequant_int4_sym(codes, a["lk_sz"][[b], :T].astype(np.float64), c["g"])
+        for kvh in (0, 7):
+            sl = slice(kvh * d, (kvh + 1) * d)
+            q = O.bf16_bits_to_f64(a["q"][:, [b], kvh * 4:(kvh + 1) * 4])     # [L, 1, 4, d]
+            ref = O.decode_block_shared(q, lat, a["wk"][:, :, sl].astype(np.float64),
+                                        a["wv"][:, :, sl].astype(np.float64), 1, 1 / np.sqrt(d))
+            assert_close(got[:, b:b + 1, kvh * 4:(kvh + 1) * 4], ref,
+                         what=f"c3 full b={b} kvh={kvh}")
 
 
 # ------------------------------------------------------------------ tensor-core path
@@ -385,13 +389,15 @@ def test_varrate_warp_single_rank_64():
 # ------------------------------------------------------------------ block-shared latent on warp-level MMAs
 
 
-@pytest.mark.parametrize("B,n", [(1, 1), (2, 300), (1, 2049)])
-def test_block_mma_path(B, n):
-    """The block-shared latent for 4 layers runs on the CTA-cooperative mma.sync
-    kernel (32 absorbed queries per CTA); per-row lengths force the generic
-    kernel.  Both must match the oracle."""
+@pytest.mark.parametrize("B,n", [(1, 1), (2, 63), (2, 64), (1, 65), (2, 300), (1, 2049),
+                                 (3, 8191)])
+def test_block_tc_path(B, n):
+    """The block-shared latent for 4 layers runs on the tcgen05 kernel (128
+    absorbed queries per CTA, 64-token tiles, one CTA per half of the latent
+    columns); per-row lengths force the generic kernel.  Both must match the
+    oracle."""
     c = synth.config("c3", B=B, T=n)
     a = synth.block_shared_cache(c)
     ref = oracle(c, a, n)
-    assert_close(run_decode(c, a, n), ref, what=f"block mma B={B} n={n}")
+    assert_close(run_decode(c, a, n), ref, what=f"block tc B={B} n={n}")
     assert_close(run_decode(c, a, n, seq_lens=[n] * B), ref, what=f"generic B={B} n={n}")
