@@ -297,17 +297,20 @@ __global__ void append_dense_kernel(AppendParams a) {
 
 // Bulk append (prefill) of INT4 low-rank rows without the residual: one block
 // per (chunk of kBulkTok tokens, batch row, KV head, K or V).  The factor rows
-// are staged once in shared memory as fp32, rows padded to 129 floats so that
-// lane j reading row j is conflict-free; warp w takes tokens w, w + 8, ... of
-// the chunk, lane j forms latent entries j and j + 32 with the summation order
-// of append_lowrank_kernel (so the codes are the same), then the group's
-// minimum and maximum by shuffles and the codes, two per byte.
+// are staged once in shared memory as fp32 (rows padded to 132 floats, so the
+// 16-byte loads of 8 lanes reading 8 rows are conflict-free); each warp takes
+// kBulkGroup tokens at a time, lane j forming latent entries j and j + 32 of
+// all of them from one read of its factor rows, each entry summed over d in
+// the order of append_lowrank_kernel (so the codes are the same); then the
+// groups' minimum and maximum by shuffles and the codes, two per byte.
 constexpr int kBulkTok = 256;
 constexpr int kBulkThreads = 256;
+constexpr int kBulkGroup = 8;                    // tokens per warp pass
+constexpr int kBulkRow = 132;                    // floats per staged factor row
 
 __global__ void __launch_bounds__(kBulkThreads) append_lowrank_bulk_kernel(AppendParams a) {
   const Params& p = a.p;
-  extern __shared__ float fs[];                  // [r][129] factor rows, then x [8][128]
+  extern __shared__ __align__(16) float fs[];    // [r][132] factor rows, then x [8 warps][8][128]
   const int chunk = blockIdx.x;
   int idx = blockIdx.y;                          // (b * Hkv + h) * 2 + comp
   const int comp = idx & 1;
@@ -321,71 +324,90 @@ __global__ void __launch_bounds__(kBulkThreads) append_lowrank_bulk_kernel(Appen
   const int r = comp == 0 ? p.rk : p.rv;
   const int ng = (r + 31) / 32;
   const __half* fac = (comp == 0 ? p.bk : p.bv) + (int64_t)h * r * 128;
-  for (int e = threadIdx.x; e < r * 128; e += kBulkThreads) fs[(e >> 7) * 129 + (e & 127)] = h2f(fac[e]);
+  for (int e = threadIdx.x; e < r * 128; e += kBulkThreads) fs[(e >> 7) * kBulkRow + (e & 127)] = h2f(fac[e]);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* xs = fs + r * 129 + warp * 128;
+  const int rmax = p.rk > p.rv ? p.rk : p.rv;
+  float* xs = fs + rmax * kBulkRow + warp * kBulkGroup * 128;
   __syncthreads();
-  for (int ti = warp; ti < kBulkTok; ti += kBulkThreads / 32) {
-    const int i = chunk * kBulkTok + ti;
-    if (i >= a.n_new) break;
-    const int tok = p0 + i;
-    if (p.page) {
-      const int pp = p.page_table[(int64_t)b * (p.tmax / p.page) + tok / p.page];
-      if (pp < 0 || pp >= p.n_pages) {
-        if (lane == 0 && h == 0 && comp == 0) flag(a.status, KVC_DEV_BAD_PAGE);
-        continue;
+  const int i_end = min(a.n_new, (chunk + 1) * kBulkTok);
+  for (int i0 = chunk * kBulkTok + warp * kBulkGroup; i0 < i_end; i0 += (kBulkThreads / 32) * kBulkGroup) {
+    // the group's rows of x (zeros past the end)
+#pragma unroll
+    for (int t = 0; t < kBulkGroup; ++t) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i0 + t < i_end) {
+        const __nv_bfloat16* src = (comp == 0 ? a.k_new : a.v_new) +
+                                   (((int64_t)b * p.Hkv + h) * a.n_new + i0 + t) * 128;
+        const uint2 u = *reinterpret_cast<const uint2*>(src + 4 * lane);
+        const __nv_bfloat162 x01 = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+        const __nv_bfloat162 x23 = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+        v = make_float4(__low2float(x01), __high2float(x01), __low2float(x23), __high2float(x23));
       }
-    }
-    const __nv_bfloat16* src =
-        (comp == 0 ? a.k_new : a.v_new) + (((int64_t)b * p.Hkv + h) * a.n_new + i) * 128;
-    {
-      const uint2 u = *reinterpret_cast<const uint2*>(src + 4 * lane);
-      const __nv_bfloat162 x01 = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-      const __nv_bfloat162 x23 = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-      xs[4 * lane] = __low2float(x01);
-      xs[4 * lane + 1] = __high2float(x01);
-      xs[4 * lane + 2] = __low2float(x23);
-      xs[4 * lane + 3] = __high2float(x23);
+      *reinterpret_cast<float4*>(xs + t * 128 + 4 * lane) = v;
     }
     __syncwarp();
-    float lat[2] = {0.f, 0.f};
+    float lat[2][kBulkGroup];
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi) {
-      const int j = lane + 32 * gi;
-      if (j < r) {
-        const float* br = fs + j * 129;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < 128; ++k) acc = fmaf(xs[k], br[k], acc);
-        lat[gi] = acc;
+    for (int t = 0; t < kBulkGroup; ++t) lat[0][t] = lat[1][t] = 0.f;
+    const bool two = lane + 32 < r;
+    const float* b0 = fs + lane * kBulkRow;
+    const float* b1 = fs + (two ? lane + 32 : lane) * kBulkRow;
+#pragma unroll 2
+    for (int k = 0; k < 128; k += 4) {
+      const float4 w0 = *reinterpret_cast<const float4*>(b0 + k);
+      const float4 w1 = *reinterpret_cast<const float4*>(b1 + k);
+#pragma unroll
+      for (int t = 0; t < kBulkGroup; ++t) {
+        const float4 x = *reinterpret_cast<const float4*>(xs + t * 128 + k);
+        lat[0][t] = fmaf(x.x, w0.x, lat[0][t]);
+        lat[0][t] = fmaf(x.y, w0.y, lat[0][t]);
+        lat[0][t] = fmaf(x.z, w0.z, lat[0][t]);
+        lat[0][t] = fmaf(x.w, w0.w, lat[0][t]);
+        lat[1][t] = fmaf(x.x, w1.x, lat[1][t]);
+        lat[1][t] = fmaf(x.y, w1.y, lat[1][t]);
+        lat[1][t] = fmaf(x.z, w1.z, lat[1][t]);
+        lat[1][t] = fmaf(x.w, w1.w, lat[1][t]);
       }
     }
-    const int64_t row = lowrank_row(p, b, h, tok);
-    uint8_t* codes = (comp == 0 ? a.lk_w : a.lv_w) + row * (r / 2);
-    __half* sz = (comp == 0 ? a.lksz_w : a.lvsz_w) + row * 2 * ng;
-    for (int gi = 0; gi < ng; ++gi) {
-      const int j = lane + 32 * gi;
-      const bool in = j < r;
-      const float v = gi == 0 ? lat[0] : lat[1];
-      float lo = in ? v : INFINITY, hi = in ? v : -INFINITY;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    for (int t = 0; t < kBulkGroup; ++t) {
+      const int i = i0 + t;
+      if (i >= i_end) break;
+      const int tok = p0 + i;
+      if (p.page) {
+        const int pp = p.page_table[(int64_t)b * (p.tmax / p.page) + tok / p.page];
+        if (pp < 0 || pp >= p.n_pages) {
+          if (lane == 0 && h == 0 && comp == 0) flag(a.status, KVC_DEV_BAD_PAGE);
+          continue;
+        }
       }
-      const __half zh = __float2half_rn(lo);
-      const __half sh = __float2half_rn((hi - lo) / 15.f);
-      const float s = __half2float(sh), z = __half2float(zh);
-      int c = 0;
-      if (in && s > 0.f) c = (int)fminf(fmaxf(rintf((v - z) / s), 0.f), 15.f);
-      const int cn = __shfl_down_sync(0xffffffffu, c, 1);
-      if (in && !(lane & 1)) codes[j >> 1] = (uint8_t)(c | (cn << 4));
-      if (lane == 0) {
-        sz[2 * gi] = sh;
-        sz[2 * gi + 1] = zh;
+      const int64_t row = lowrank_row(p, b, h, tok);
+      uint8_t* codes = (comp == 0 ? a.lk_w : a.lv_w) + row * (r / 2);
+      __half* sz = (comp == 0 ? a.lksz_w : a.lvsz_w) + row * 2 * ng;
+      for (int gi = 0; gi < ng; ++gi) {
+        const int j = lane + 32 * gi;
+        const bool in = j < r;
+        const float v = gi == 0 ? lat[0][t] : lat[1][t];
+        float lo = in ? v : INFINITY, hi = in ? v : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+          hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        const __half zh = __float2half_rn(lo);
+        const __half sh = __float2half_rn((hi - lo) / 15.f);
+        const float s = __half2float(sh), z = __half2float(zh);
+        int c = 0;
+        if (in && s > 0.f) c = (int)fminf(fmaxf(rintf((v - z) / s), 0.f), 15.f);
+        const int cn = __shfl_down_sync(0xffffffffu, c, 1);
+        if (in && !(lane & 1)) codes[j >> 1] = (uint8_t)(c | (cn << 4));
+        if (lane == 0) {
+          sz[2 * gi] = sh;
+          sz[2 * gi + 1] = zh;
+        }
       }
     }
-    __syncwarp();                                // xs is rewritten by the next token
+    __syncwarp();                                // xs is rewritten by the next group
   }
 }
 
@@ -403,7 +425,11 @@ cudaError_t launch_append(const AppendParams& a, cudaStream_t s) {
     case KVC_LOWRANK:
       if (bulk_ok(a)) {
         const int rmax = p.rk > p.rv ? p.rk : p.rv;
-        const size_t smem = ((size_t)rmax * 129 + 8 * 128) * sizeof(float);
+        const size_t smem =
+            ((size_t)rmax * kBulkRow + (kBulkThreads / 32) * kBulkGroup * 128) * sizeof(float);
+        cudaError_t e = cudaFuncSetAttribute(append_lowrank_bulk_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
         dim3 grid((a.n_new + kBulkTok - 1) / kBulkTok, p.B * p.Hkv * 2);
         append_lowrank_bulk_kernel<<<grid, kBulkThreads, smem, s>>>(a);
       } else {

@@ -255,16 +255,18 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
 // Block-shared latent: one block per (layer, batch row, KV head) merges the
 // G query heads' partials together and applies the layer's W_v slice to all
 // of them, so each W_v element is read once per block rather than once per
-// query head.  Thread (i, half) forms output dim i of every head over half of
-// the latent columns; the two halves are added at the end.
+// query head.  The slice (D rows x head dim) streams through shared memory in
+// chunks of 64 rows (16-byte cp.async, double-buffered); thread (i, g0) forms
+// output dim i of heads g0, g0 + 2, ... .
 constexpr int kBGroup = 8;               // query heads per KV head handled (G <= 8)
+constexpr int kBRows = 64;               // W_v rows per staged chunk
 
 __global__ void __launch_bounds__(kThreads) combine_block_kernel(Params p) {
-  extern __shared__ float bsm[];
+  extern __shared__ __align__(16) float bsm[];
   const int D = p.D, d = p.d, G = p.G;
   float* acc = bsm;                      // [G][D]
   float* ws = acc + G * D;               // [G][S]
-  float* red = ws + G * p.S;             // [kThreads][G]
+  __half* wv = reinterpret_cast<__half*>(ws + ((G * p.S + 3) & ~3));   // [2][kBRows][d], 16-B aligned
   __shared__ float linv[kBGroup];
   const int blk = blockIdx.x;            // (l * B + b) * Hkv + kvh
   const int kvh = blk % p.Hkv, lb = blk / p.Hkv;   // lb = l * B + b
@@ -273,7 +275,22 @@ __global__ void __launch_bounds__(kThreads) combine_block_kernel(Params p) {
   const size_t rows = (size_t)p.L * p.B * p.Hq;
   const int pst = p.vdim + 2;
   const int nS = p.S;
+  const __half* w = p.bv + (int64_t)l * D * p.Hkv * d + kvh * d;
+  const int n_chunks = (D + kBRows - 1) / kBRows;
+  const int cpr = d / 8;                 // 16-byte chunks per W_v row
+  auto stage = [&](int c, int buf) {
+    for (int e = tid; e < kBRows * cpr; e += kThreads) {
+      const int r = e / cpr, part = e % cpr, row = c * kBRows + r;
+      if (row < D) {
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(wv + ((size_t)buf * kBRows + r) * d + part * 8);
+        const __half* src = w + (int64_t)row * p.Hkv * d + part * 8;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  stage(0, 0);
   // split weights and softmax sums of the G rows (warp g: row g)
   for (int g = warp; g < G; g += kThreads / 32) {
     const float* part = p.part + ((size_t)lb * p.Hq + kvh * G + g) * pst;
@@ -283,9 +300,9 @@ __global__ void __launch_bounds__(kThreads) combine_block_kernel(Params p) {
     float lt = 0.f;
     for (int s = lane; s < nS; s += 32) {
       const float* ps = part + (size_t)s * rows * pst;
-      const float w = (mx == -INFINITY) ? 0.f : exp2f(ps[D] - mx);
-      ws[g * nS + s] = w;
-      if (w != 0.f) lt += w * ps[D + 1];
+      const float wt = (mx == -INFINITY) ? 0.f : exp2f(ps[D] - mx);
+      ws[g * nS + s] = wt;
+      if (wt != 0.f) lt += wt * ps[D + 1];
     }
     lt = warp_sum(lt);
     if (lane == 0) linv[g] = lt > 0.f ? 1.f / lt : 0.f;
@@ -296,43 +313,49 @@ __global__ void __launch_bounds__(kThreads) combine_block_kernel(Params p) {
     const int g = e / D, c = e % D;
     const float* part = p.part + ((size_t)lb * p.Hq + kvh * G + g) * pst + c;
     float a = 0.f;
-    for (int s = 0; s < nS; ++s) {
-      const float w = ws[g * nS + s];
-      if (w != 0.f) a = fmaf(w, part[(size_t)s * rows * pst], a);
-    }
+#pragma unroll 8
+    for (int s = 0; s < nS; ++s) a = fmaf(ws[g * nS + s], part[(size_t)s * rows * pst], a);
     acc[e] = a;
   }
-  __syncthreads();
   // up-projection o_g = acc_g W_v^l[:, kvh slice] / l_g
-  const __half* w = p.bv + (int64_t)l * D * p.Hkv * d + kvh * d;
-  for (int i0 = 0; i0 < d; i0 += kThreads / 2) {
-    const int i = i0 + tid % (kThreads / 2), half = tid / (kThreads / 2);
-    float o[kBGroup];
+  const int gstep = kThreads / d;        // heads handled in parallel (2 for d = 128)
+  const int i = tid % d, g0 = tid / d;
+  float o[kBGroup];
 #pragma unroll
-    for (int g = 0; g < kBGroup; ++g) o[g] = 0.f;
-    if (i < d) {
-      const int c0 = half * (D / 2), c1 = c0 + D / 2;
-#pragma unroll 4
-      for (int c = c0; c < c1; ++c) {
-        const float wv = h2f(w[(int64_t)c * p.Hkv * d + i]);
+  for (int g = 0; g < kBGroup; ++g) o[g] = 0.f;
+  for (int c = 0; c < n_chunks; ++c) {
+    if (c + 1 < n_chunks) {
+      stage(c + 1, (c + 1) & 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const __half* wc = wv + (size_t)(c & 1) * kBRows * d;
+    const int nr = min(kBRows, D - c * kBRows);
+    if (g0 < gstep) {
+      for (int r = 0; r < nr; ++r) {
+        const float wvv = __half2float(wc[r * d + i]);
 #pragma unroll
-        for (int g = 0; g < kBGroup; ++g)
-          if (g < G) o[g] = fmaf(acc[g * D + c], wv, o[g]);
+        for (int gg = 0; gg < kBGroup; ++gg) {
+          const int g = g0 + gstep * gg;
+          if (g < G) o[gg] = fmaf(acc[g * D + c * kBRows + r], wvv, o[gg]);
+        }
       }
     }
+    __syncthreads();                     // buffer c & 1 is restaged for chunk c + 2
+  }
+  if (g0 < gstep) {
 #pragma unroll
-    for (int g = 0; g < kBGroup; ++g)
-      if (g < G) red[tid * G + g] = o[g];
-    __syncthreads();
-    if (tid < kThreads / 2 && i < d) {
-      for (int g = 0; g < G; ++g) {
-        const float t = (red[tid * G + g] + red[(tid + kThreads / 2) * G + g]) * linv[g];
+    for (int gg = 0; gg < kBGroup; ++gg) {
+      const int g = g0 + gstep * gg;
+      if (g < G) {
+        const float t = o[gg] * linv[g];
         const int64_t orow = (int64_t)lb * p.Hq + kvh * G + g;
         if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[orow * d + i] = __float2bfloat16_rn(t);
         else reinterpret_cast<float*>(p.out)[orow * d + i] = t;
       }
     }
-    __syncthreads();
   }
 }
 
@@ -360,8 +383,10 @@ cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (p.kind == KVC_BLOCK_SHARED && p.G <= kBGroup && p.seg_W == 0) {
-    const size_t bb = ((size_t)p.G * p.D + (size_t)p.G * p.S + (size_t)kThreads * p.G) * sizeof(float);
+  if (p.kind == KVC_BLOCK_SHARED && p.G <= kBGroup && p.seg_W == 0 && p.d % 8 == 0 &&
+      p.d <= kThreads) {
+    const size_t bb = ((size_t)p.G * p.D + (size_t)p.G * p.S + 4) * sizeof(float) +
+                      (size_t)2 * kBRows * p.d * sizeof(__half);
     e = cudaFuncSetAttribute(combine_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)bb);
     if (e != cudaSuccess) return e;

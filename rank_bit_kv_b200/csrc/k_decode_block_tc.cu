@@ -13,8 +13,8 @@
 //              with tcgen05.ld, keeps (m, l) with a lazily raised maximum,
 //              writes its probabilities as f16 into TMEM (the A operand of the
 //              O MMA) and rescales its O row in TMEM when the maximum rises;
-//   warps 4-7  producers: load the tile's codes and scales from global memory
-//              into registers one tile ahead and dequantise x = (c - 8) s into
+//   warps 4-7  producers: load the tiles' codes and scales from global memory
+//              into registers two tiles ahead and dequantise x = (c - 8) s into
 //              f16 core matrices in shared memory, the other half (read only
 //              by the score MMAs) into one buffer, this CTA's half (read by
 //              both MMAs) into two;
@@ -248,42 +248,51 @@ __global__ void __launch_bounds__(kThreads, 1) block_tc_kernel(Params p) {
   } else if (warp >= kWarpProd) {
     // ------------------------------------------------------------ producers
     const int pt = tid - 32 * kWarpProd;           // 0..127
-    const int n = pt >> 1, qh = pt & 1;            // token of the tile, quarter of a half
+    // token of the tile and quarter of a half: the 8 lanes of each quarter-warp
+    // take 8 consecutive tokens of one quarter, so every 16-byte shared store
+    // of a quarter-warp fills one 128-byte row of banks
+    const int pl = pt & 31;
+    const int n = (pt >> 5) * 16 + (pl & 7) + ((pl >> 4) << 3);
+    const int qh = (pl >> 3) & 1;
     const uint8_t* codes = p.lk + (size_t)b * p.tmax * (kBD / 2);
     const __half* scales = p.lksz + (size_t)b * p.tmax * (kBD / kBG);
-    auto row_of = [&](int i, const uint8_t** cr, const __half** sr) -> bool {
+    auto load_tile = [&](int i, HalfRegs& ro, HalfRegs& rw) {
       const int tok = t_a + i * kBT + n;
       const bool ok = tok < t_b;
       const int t = ok ? tok : t_a;
-      *cr = codes + (size_t)t * (kBD / 2);
-      *sr = scales + (size_t)t * (kBD / kBG);
-      return ok;
-    };
-    HalfRegs ro, rw;                               // other half, own half
-    if (n_tiles > 0) {
-      const uint8_t* cr;
-      const __half* sr;
-      const bool ok = row_of(0, &cr, &sr);
+      const uint8_t* cr = codes + (size_t)t * (kBD / 2);
+      const __half* sr = scales + (size_t)t * (kBD / kBG);
       load_half(ro, cr, sr, 1 - h, qh, ok);
       load_half(rw, cr, sr, h, qh, ok);
-    }
-    for (int i = 0; i < n_tiles; ++i) {
-      const bool more = i + 1 < n_tiles;
-      const uint8_t* cr = nullptr;
-      const __half* sr = nullptr;
-      const bool ok_next = more ? row_of(i + 1, &cr, &sr) : false;
+    };
+    // codes stay in registers two tiles ahead of the dequantisation
+    auto produce = [&](int i, HalfRegs& ro, HalfRegs& rw) -> bool {
+      const bool ahead = i + 2 < n_tiles;
+      const int tok = t_a + (i + 2) * kBT + n;
+      const bool ok2 = ahead && tok < t_b;
+      const int t2 = ok2 ? tok : t_a;
+      const uint8_t* cr = codes + (size_t)t2 * (kBD / 2);
+      const __half* sr = scales + (size_t)t2 * (kBD / kBG);
       // other half: free once S(i - 1) has read it
-      if (i >= 1 && !mbar_wait(&bars.oth_free, (i - 1) & 1, abort, err)) break;
+      if (i >= 1 && !mbar_wait(&bars.oth_free, (i - 1) & 1, abort, err)) return false;
       store_half(oth_buf, ro, n, qh);
       fence_proxy_async_smem();
       mbar_arrive(&bars.oth_full);
-      if (more) load_half(ro, cr, sr, 1 - h, qh, ok_next);
+      if (ahead) load_half(ro, cr, sr, 1 - h, qh, ok2);
       // own half: buffer i & 1 is free once O(i - 2) has read it
-      if (i >= 2 && !mbar_wait(&bars.own_free[i & 1], ((i - 2) >> 1) & 1, abort, err)) break;
+      if (i >= 2 && !mbar_wait(&bars.own_free[i & 1], ((i - 2) >> 1) & 1, abort, err)) return false;
       store_half(own_buf(i & 1), rw, n, qh);
       fence_proxy_async_smem();
       mbar_arrive(&bars.own_full[i & 1]);
-      if (more) load_half(rw, cr, sr, h, qh, ok_next);
+      if (ahead) load_half(rw, cr, sr, h, qh, ok2);
+      return true;
+    };
+    HalfRegs roA, rwA, roB, rwB;                   // tiles i (even) and i + 1
+    if (n_tiles > 0) load_tile(0, roA, rwA);
+    if (n_tiles > 1) load_tile(1, roB, rwB);
+    for (int i = 0; i < n_tiles; i += 2) {
+      if (!produce(i, roA, rwA)) break;
+      if (i + 1 < n_tiles && !produce(i + 1, roB, rwB)) break;
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-3)

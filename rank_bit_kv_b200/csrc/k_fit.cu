@@ -124,15 +124,18 @@ __global__ void __launch_bounds__(kFThreads) gram_kernel(const __nv_bfloat16* __
   }
 }
 
-// G = sum of the partials of a head, in chunk order, in fp64.
+// G = sum of the partials of a head, in chunk order, in fp64; grid (entry
+// blocks, heads), one entry per thread.
 __global__ void gram_reduce_kernel(const float* __restrict__ part, int n_chunks,
                                    double* __restrict__ G) {
-  const int h = blockIdx.x;
-  for (int e = threadIdx.x; e < kFD * kFD; e += blockDim.x) {
-    double s = 0.0;
-    for (int c = 0; c < n_chunks; ++c) s += (double)part[((size_t)h * n_chunks + c) * kFD * kFD + e];
-    G[(size_t)h * kFD * kFD + e] = s;
-  }
+  const int h = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= kFD * kFD) return;
+  const float* src = part + (size_t)h * n_chunks * kFD * kFD + e;
+  double s = 0.0;
+#pragma unroll 16
+  for (int c = 0; c < n_chunks; ++c) s += (double)src[(size_t)c * kFD * kFD];
+  G[(size_t)h * kFD * kFD + e] = s;
 }
 
 struct SmallWs {          // per-head fp64 scratch in global memory
@@ -192,25 +195,38 @@ __device__ void orthonormalise(double* W, int k, double* red) {
   }
 }
 
+// shared bytes of the small stage without / with W and P
+__host__ __device__ size_t small_smem_base(int k) {
+  return (size_t)(2 * k * k + kFD + 1 + k) * sizeof(double) + (size_t)k * sizeof(int) + 64;
+}
+size_t small_smem_wp(int k) {
+  return ((small_smem_base(k) + 15) & ~(size_t)15) + (size_t)2 * kFD * k * sizeof(double);
+}
+
 // One CTA per head: the small stage in fp64 (see the file comment).
 // Shared: C (k x k), U (k x k), scratch.  k <= kFitMaxK, even.
 __global__ void __launch_bounds__(kSThreads) rsvd_small_kernel(
     const double* __restrict__ Gall, const float* __restrict__ omega, int k, int rank,
-    int power_iters, SmallWs ws_base, __half* __restrict__ factor, float* __restrict__ sigma2) {
+    int power_iters, SmallWs ws_base, __half* __restrict__ factor, float* __restrict__ sigma2,
+    int wp_in_smem) {
   extern __shared__ __align__(16) double ssm[];
   const int h = blockIdx.x;
   const int tid = threadIdx.x, nth = blockDim.x;
   const double* G = Gall + (size_t)h * kFD * kFD;
   const size_t dk = (size_t)kFD * kFitMaxK;
-  double* W = ws_base.W + h * dk;
-  double* P = ws_base.P + h * dk;
-  double* V = ws_base.V + h * dk;
   double* C = ssm;                          // k x k, row-major
   double* U = C + k * k;                    // k x k
   double* red = U + k * k;                  // kFD + 1 + 2k scratch
   double* cs = red + kFD + 1;               // rotation cosines / sines of a round
   double* sn = cs + k / 2;
   int* order = reinterpret_cast<int*>(sn + k / 2);   // k ints
+  // W and P (d x k) live in shared memory when the launch gave room for them
+  // (the Gram-Schmidt passes re-read them column by column), else in global
+  double* const sm_wp = reinterpret_cast<double*>(
+      reinterpret_cast<char*>(ssm) + ((small_smem_base(k) + 15) & ~(size_t)15));
+  double* W = wp_in_smem ? sm_wp : ws_base.W + h * dk;
+  double* P = wp_in_smem ? sm_wp + (size_t)kFD * k : ws_base.P + h * dk;
+  double* V = ws_base.V + h * dk;
 
   // W = Omega (column-major), power iterations
   for (int e = tid; e < kFD * k; e += nth) {
@@ -385,9 +401,6 @@ __global__ void __launch_bounds__(kSThreads) rsvd_small_kernel(
   }
 }
 
-size_t small_smem(int k) {
-  return (size_t)(2 * k * k + kFD + 1 + k) * sizeof(double) + (size_t)k * sizeof(int) + 64;
-}
 
 }  // namespace
 
@@ -416,12 +429,13 @@ cudaError_t launch_fit(const FitParams& f, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   gram_kernel<<<dim3(kFitChunks, f.Hkv), kFThreads, gsm, s>>>(f.x, f.B, f.Hkv, f.cap, f.n_rows,
                                                               kFitChunks, part);
-  gram_reduce_kernel<<<f.Hkv, 256, 0, s>>>(part, kFitChunks, G);
-  const size_t ssm = small_smem(f.k);
+  gram_reduce_kernel<<<dim3(kFD * kFD / 256, f.Hkv), 256, 0, s>>>(part, kFitChunks, G);
+  const int wp = small_smem_wp(f.k) <= 227 * 1024 ? 1 : 0;
+  const size_t ssm = wp ? small_smem_wp(f.k) : small_smem_base(f.k);
   e = cudaFuncSetAttribute(rsvd_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
   if (e != cudaSuccess) return e;
   rsvd_small_kernel<<<f.Hkv, kSThreads, ssm, s>>>(G, f.omega, f.k, f.rank, f.power_iters, sw,
-                                                  f.factor, f.sigma2);
+                                                  f.factor, f.sigma2, wp);
   return cudaGetLastError();
 }
 

@@ -129,7 +129,9 @@ void kvc_test_skip_tile_copies(int32_t on) { g_test_no_copies = on ? 1 : 0; }
 
 void kvc_select_rope_kernel(int32_t which) { g_rope_kernel = which == 2 ? 2 : 0; }
 
-const char* kvc_version(void) { return "kvc 0.3 (sm_100a; decode kernels rev 13)"; }
+const char* kvc_version(void) {
+  return "kvc 0.3 (sm_100a; decode kernels rev 14; rope_mma rev 12)";
+}
 
 kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out) {
   if (!desc || !out) return fail(KVC_EINVAL, "kvc_create_layout: NULL argument");
