@@ -523,6 +523,15 @@ void kvc_test_skip_tile_copies(int32_t on);
  * pages. */
 void kvc_select_rope_kernel(int32_t which);
 
+/* Kernel choice for the variable-rate layout with 8 KV heads x 4 query heads
+ * and uniform lengths (per calling thread): 0 (default) runs the
+ * lane-per-(KV head, query head) kernel on CUDA cores (the faster of the two
+ * as measured), 1 the tensor-core kernel (scores and values on mma.sync at the
+ * full rank, codes beyond a token's rank masked).  Both compute the same
+ * decode (VarRate "Method"); the switch exists so that either can be tested
+ * and timed.  No counterpart on the pages. */
+void kvc_select_varrate_kernel(int32_t which);
+
 /* Thread-local description of the last error on this thread ("" if none). */
 const char* kvc_last_error(void);
 

@@ -370,6 +370,7 @@ cudaError_t launch_split(const Params& p, cudaStream_t s) {
     case 5: return launch_varrate_warp(p, s);
     case 6: return launch_block_mma(p, s);
     case 8: return launch_block_tc(p, s);
+    case 9: return launch_varrate_mma(p, s);
     default: break;
   }
   const Geo g = geometry(p);

@@ -26,6 +26,7 @@ namespace {
 thread_local std::string g_err;
 thread_local int g_test_no_copies = 0;   // kvc_test_skip_tile_copies
 thread_local int g_rope_kernel = 0;      // kvc_select_rope_kernel
+thread_local int g_varrate_kernel = 0;   // 0: lane-per-head warp kernel, 1: tensor-core kernel
 
 kvc_status fail(kvc_status st, const char* fmt, ...) {
   char buf[512];
@@ -128,6 +129,8 @@ const char* kvc_last_error(void) { return g_err.c_str(); }
 void kvc_test_skip_tile_copies(int32_t on) { g_test_no_copies = on ? 1 : 0; }
 
 void kvc_select_rope_kernel(int32_t which) { g_rope_kernel = which == 2 ? 2 : 0; }
+
+void kvc_select_varrate_kernel(int32_t which) { g_varrate_kernel = which == 1 ? 1 : 0; }
 
 const char* kvc_version(void) {
   return "kvc 0.3 (sm_100a; decode kernels rev 14; rope_mma rev 12)";
@@ -347,7 +350,7 @@ int32_t kvc_decode_launches(const kvc_layout* L, int32_t n_tokens) {
   // runs the warp kernel, which projects its own queries
   if (p.kind == KVC_VARRATE && L->d.n_kv_heads == 8 && L->d.n_q_heads == 32 &&
       L->d.group_size == 32 && n_tokens > 0)
-    p.path = 5;
+    p.path = g_varrate_kernel ? 9 : 5;
   return 2 + (kvc::needs_qproj(p) ? 1 : 0);
 }
 
@@ -544,8 +547,11 @@ extern "C" kvc_status kvc_decode_attn_timed(const kvc_layout* L, const kvc_cache
       p.seg_W = W;
       p.seg_tpu = tpu;
       p.seg_parts = parts;
-    } else if (kvc::varrate_warp_supported(p)) {
+    } else if (kvc::varrate_mma_supported(p) && g_varrate_kernel == 1) {
       // fixed token splits per batch row (one partial per CTA)
+      kvc::varrate_mma_plan(p, &p.S, &p.split_len);
+      p.path = 9;
+    } else if (kvc::varrate_warp_supported(p)) {
       kvc::varrate_warp_plan(p, &p.S, &p.split_len);
       p.path = 5;
     } else if (kvc::block_tc_supported(p)) {

@@ -64,7 +64,8 @@ struct Params {
   int seg_W, seg_tpu;
   int seg_parts;         // partials written per CTA and unit on that path
   int path;              // split kernel: 0 generic, 1 rope_tc, 2 dense_tc, 3 latent_tc, 4 rope_mma,
-                         // 5 varrate_warp, 6 block_mma, 7 rope_wg, 8 block_tc
+                         // 5 varrate_warp, 6 block_mma, 7 rope_wg, 8 block_tc,
+                         // 9 varrate_mma
   uint32_t* err;         // error word of the workspace (bounded waits that gave up)
   int test_no_copies;    // test switch: the tcgen05 producer issues no tile copies
   // RoPE: turns per position of frequency pair i, theta^(-2i/d) / (2 pi)
@@ -147,6 +148,12 @@ void varrate_warp_plan(const Params& p, int* splits, int* split_len);
 int varrate_warp_slots(int batch, int n_tokens);
 cudaError_t launch_varrate_warp(const Params& p, cudaStream_t s);
 
+// variable-rate layout on warp-level tensor cores, one warp per (KV head, half
+// of each 32-token chunk); projects its own queries (selectable)
+bool varrate_mma_supported(const Params& p);
+void varrate_mma_plan(const Params& p, int* splits, int* split_len);
+cudaError_t launch_varrate_mma(const Params& p, cudaStream_t s);
+
 // block-shared latent, 32 absorbed queries per CTA on mma.sync
 bool block_mma_supported(const Params& p);
 void block_mma_plan(const Params& p, int* splits, int* split_len);
@@ -211,9 +218,9 @@ cudaError_t launch_combine(const Params& p, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& a, cudaStream_t s);
 
 // Whether the decode of this layout runs a query projection first.
-// (The variable-rate warp kernel, path 5, projects its queries itself.)
+// (The variable-rate kernels, paths 5 and 9, project their queries themselves.)
 __host__ __device__ inline bool needs_qproj(const Params& p) {
-  return (p.kind == KVC_VARRATE && p.path != 5) || p.kind == KVC_BLOCK_SHARED ||
+  return (p.kind == KVC_VARRATE && p.path != 5 && p.path != 9) || p.kind == KVC_BLOCK_SHARED ||
          (p.kind == KVC_LOWRANK && !p.rope);
 }
 

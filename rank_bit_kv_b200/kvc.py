@@ -116,6 +116,8 @@ def lib():
         L.kvc_block_compact.restype = C.c_int
         L.kvc_select_rope_kernel.argtypes = [i32]
         L.kvc_select_rope_kernel.restype = None
+        L.kvc_select_varrate_kernel.argtypes = [i32]
+        L.kvc_select_varrate_kernel.restype = None
         L.kvc_test_skip_tile_copies.argtypes = [i32]
         L.kvc_test_skip_tile_copies.restype = None
         L.kvc_last_error.argtypes = []

@@ -38,6 +38,8 @@ def main(argv=None):
     ap.add_argument("--time", action="store_true")
     ap.add_argument("--rope-kernel", type=int, default=0,
                     help="pre-RoPE layouts: 0 / 1 warp-level mma.sync kernel, 2 tcgen05 warpgroup kernel")
+    ap.add_argument("--varrate-kernel", type=int, default=0,
+                    help="variable-rate layout: 0 lane-per-head kernel, 1 tensor-core kernel")
     args = ap.parse_args(argv)
 
     import numpy as np
@@ -47,6 +49,7 @@ def main(argv=None):
 
     over = {} if args.batch is None else {"B": args.batch}
     kvc.lib().kvc_select_rope_kernel(args.rope_kernel)
+    kvc.lib().kvc_select_varrate_kernel(args.varrate_kernel)
     c = synth.config(args.config, **over)
     lay, cache, fill = _cache(kvc, synth, c)
     q = torch.from_numpy(np.ascontiguousarray(fill["q"]).view(np.int16)).cuda().view(torch.bfloat16)

@@ -102,8 +102,19 @@ def test_paging_shuffled_equals_identity_table():
     np.testing.assert_allclose(g1, g2, rtol=0, atol=1e-6)
 
 
+@pytest.fixture(params=["tensor_core", "lane_per_head"])
+def varrate_kernel(request):
+    """Run a variable-rate test on the lane-per-(KV head, query head) kernel
+    (default) and on the tensor-core kernel."""
+    from rank_bit_kv_b200 import kvc
+
+    kvc.lib().kvc_select_varrate_kernel(1 if request.param == "tensor_core" else 0)
+    yield request.param
+    kvc.lib().kvc_select_varrate_kernel(0)
+
+
 @pytest.mark.parametrize("T", [1, 300, 2000])
-def test_c4_shape_small_varrate(T):
+def test_c4_shape_small_varrate(T, varrate_kernel):
     c = synth.config("c4", T=T)
     a = synth.varrate_cache(c)
     assert_close(run_decode(c, a, T), oracle(c, a, T), what=f"c4 T={T}")
@@ -217,7 +228,7 @@ def test_full_size_every_row(name, variant):
     assert_close(got, ref, what=f"{name} {variant} full, all rows")
 
 
-def test_c4_full_size():
+def test_c4_full_size(varrate_kernel):
     c = synth.config("c4")
     a = synth.varrate_cache(c)
     assert_close(run_decode(c, a, c["T"]), oracle(c, a, c["T"]), what="c4 full")
@@ -367,10 +378,12 @@ def test_rope_kernels_agree_at_full_size():
 # ------------------------------------------------------------------ variable rate, one lane per head pair
 
 
-@pytest.mark.parametrize("B,n", [(1, 1), (1, 17), (2, 2049), (3, 5000)])
-def test_varrate_warp_path(B, n):
-    """Variable-rate records run on the lane-per-(KV head, query head) kernel;
-    per-row lengths force the generic kernel.  Both must match the oracle."""
+@pytest.mark.parametrize("B,n", [(1, 1), (1, 17), (1, 31), (1, 32), (1, 33), (2, 2049),
+                                 (3, 5000)])
+def test_varrate_paths(B, n, varrate_kernel):
+    """Variable-rate records run on the tensor-core kernel or on the
+    lane-per-(KV head, query head) kernel; per-row lengths force the generic
+    kernel.  All must match the oracle."""
     c = synth.config("c4", B=B, T=n)
     a = synth.varrate_cache(c)
     ref = oracle(c, a, n)
@@ -378,12 +391,24 @@ def test_varrate_warp_path(B, n):
     assert_close(run_decode(c, a, n, seq_lens=[n] * B), ref, what=f"generic B={B} n={n}")
 
 
-def test_varrate_warp_single_rank_64():
-    """Every token at the top rank: the ragged layout degenerates to the uniform
-    rank-64 one (the path with two scale groups per record)."""
+@pytest.mark.parametrize("rank", [4, 8, 16, 32, 64])
+def test_varrate_single_rank(rank, varrate_kernel):
+    """Every token at one rank: the ragged layout degenerates to a uniform one
+    (rank 64: two scale groups per record; rank 4: 6-byte head records)."""
     c = synth.config("c4", B=1, T=700)
-    a = synth.varrate_cache(c, ranks={"k": np.full((1, 700), 64), "v": np.full((1, 700), 64)})
-    assert_close(run_decode(c, a, 700), oracle(c, a, 700), what="varrate rank 64")
+    r = np.full((1, 700), rank)
+    a = synth.varrate_cache(c, ranks={"k": r, "v": r})
+    assert_close(run_decode(c, a, 700), oracle(c, a, 700), what=f"varrate rank {rank}")
+
+
+def test_varrate_k_and_v_ranks_differ(varrate_kernel):
+    """K ranks high where V ranks are low and the reverse, so that the score
+    and value sides mask different entries of the same tokens."""
+    c = synth.config("c4", B=1, T=999)
+    rk = np.where(np.arange(999) % 2 == 0, 64, 4)[None, :]
+    rv = np.where(np.arange(999) % 2 == 0, 4, 64)[None, :]
+    a = synth.varrate_cache(c, ranks={"k": rk, "v": rv})
+    assert_close(run_decode(c, a, 999), oracle(c, a, 999), what="varrate k/v ranks differ")
 
 
 # ------------------------------------------------------------------ block-shared latent on warp-level MMAs
