@@ -124,18 +124,23 @@ __global__ void __launch_bounds__(kFThreads) gram_kernel(const __nv_bfloat16* __
   }
 }
 
-// G = sum of the partials of a head, in chunk order, in fp64; grid (entry
-// blocks, heads), one entry per thread.
+// G = sum of the partials of a head, in chunk order, in fp64, symmetrised
+// (the tensor-core partials accumulate the two triangles in different orders):
+// G_ij = (S_ij + S_ji) / 2.  Grid (entry blocks, heads), one entry per thread.
 __global__ void gram_reduce_kernel(const float* __restrict__ part, int n_chunks,
                                    double* __restrict__ G) {
   const int h = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= kFD * kFD) return;
-  const float* src = part + (size_t)h * n_chunks * kFD * kFD + e;
-  double s = 0.0;
+  const int i = e / kFD, j = e % kFD;
+  const float* src = part + (size_t)h * n_chunks * kFD * kFD;
+  double a = 0.0, b = 0.0;
 #pragma unroll 16
-  for (int c = 0; c < n_chunks; ++c) s += (double)src[(size_t)c * kFD * kFD];
-  G[(size_t)h * kFD * kFD + e] = s;
+  for (int c = 0; c < n_chunks; ++c) {
+    a += (double)src[(size_t)c * kFD * kFD + e];
+    b += (double)src[(size_t)c * kFD * kFD + j * kFD + i];
+  }
+  G[(size_t)h * kFD * kFD + e] = 0.5 * (a + b);
 }
 
 struct SmallWs {          // per-head fp64 scratch in global memory
@@ -144,17 +149,71 @@ struct SmallWs {          // per-head fp64 scratch in global memory
   double* V;              // d x k
 };
 
-// Y[:, j] = G X[:, j] for all columns (column-major d x k), one thread per entry.
+// Y[:, j] = G X[:, j] for all columns (column-major d x k).  Thread (row,
+// block of 8 columns) reads G[l][row] (= G[row][l], G is symmetric; the lanes
+// of a warp take consecutive rows, so the loads are coalesced) once for its 8
+// accumulators; the X entries are the same for the whole warp (broadcast).
 __device__ void gemm_G(const double* __restrict__ G, const double* X, double* Y, int k) {
-  for (int e = threadIdx.x; e < kFD * k; e += blockDim.x) {
-    const int row = e % kFD, col = e / kFD;
-    const double* gr = G + (size_t)row * kFD;
-    const double* xc = X + (size_t)col * kFD;
-    double s = 0.0;
-    for (int l = 0; l < kFD; ++l) s += gr[l] * xc[l];
-    Y[(size_t)col * kFD + row] = s;
+  constexpr int CB = 8;
+  const int nblk = (k + CB - 1) / CB;
+  for (int e = threadIdx.x; e < kFD * nblk; e += blockDim.x) {
+    const int row = e % kFD, c0 = (e / kFD) * CB;
+    double acc[CB];
+#pragma unroll
+    for (int j = 0; j < CB; ++j) acc[j] = 0.0;
+#pragma unroll 4
+    for (int l = 0; l < kFD; ++l) {
+      const double gv = G[(size_t)l * kFD + row];
+#pragma unroll
+      for (int j = 0; j < CB; ++j)
+        if (c0 + j < k) acc[j] = fma(gv, X[(size_t)(c0 + j) * kFD + l], acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < CB; ++j)
+      if (c0 + j < k) Y[(size_t)(c0 + j) * kFD + row] = acc[j];
   }
   __syncthreads();
+}
+
+// C = A^T B for column-major d x k matrices A, B (k x k, row-major), in 4 x 4
+// blocks per thread; lane-rotated summation start keeps the column reads of a
+// warp on different banks.
+__device__ void gram_small(const double* A, const double* Bm, double* C, int k) {
+  const int nb = (k + 3) / 4;
+  const int lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < nb * nb; e += blockDim.x) {
+    const int i0 = 4 * (e / nb), j0 = 4 * (e % nb);
+    // columns past k read column k - 1 (in range) and are not stored
+    int ia[4], jb[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      ia[a] = min(i0 + a, k - 1);
+      jb[a] = min(j0 + a, k - 1);
+    }
+    double acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+#pragma unroll 2
+    for (int l0 = 0; l0 < kFD; ++l0) {
+      const int l = (l0 + lane) & (kFD - 1);
+      double x[4], y[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) x[a] = A[(size_t)ia[a] * kFD + l];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) y[b] = Bm[(size_t)jb[b] * kFD + l];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fma(x[a], y[b], acc[a][b]);
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if (i0 + a < k && j0 + b < k) C[(i0 + a) * k + j0 + b] = acc[a][b];
+  }
 }
 
 // Orthonormalise the k columns of W (d x k) by classical Gram-Schmidt applied
@@ -197,7 +256,7 @@ __device__ void orthonormalise(double* W, int k, double* red) {
 
 // shared bytes of the small stage without / with W and P
 __host__ __device__ size_t small_smem_base(int k) {
-  return (size_t)(2 * k * k + kFD + 1 + k) * sizeof(double) + (size_t)k * sizeof(int) + 64;
+  return (size_t)(2 * k * k + kFD + 1 + k) * sizeof(double) + (size_t)2 * k * sizeof(int) + 64;
 }
 size_t small_smem_wp(int k) {
   return ((small_smem_base(k) + 15) & ~(size_t)15) + (size_t)2 * kFD * k * sizeof(double);
@@ -220,6 +279,8 @@ __global__ void __launch_bounds__(kSThreads) rsvd_small_kernel(
   double* cs = red + kFD + 1;               // rotation cosines / sines of a round
   double* sn = cs + k / 2;
   int* order = reinterpret_cast<int*>(sn + k / 2);   // k ints
+  int* pa = order + k;                      // the pairs of a Jacobi round (k / 2 each)
+  int* pb = pa + k / 2;
   // W and P (d x k) live in shared memory when the launch gave room for them
   // (the Gram-Schmidt passes re-read them column by column), else in global
   double* const sm_wp = reinterpret_cast<double*>(
@@ -243,14 +304,7 @@ __global__ void __launch_bounds__(kSThreads) rsvd_small_kernel(
   }
   // P = G W; C = W^T P (k x k)
   gemm_G(G, W, P, k);
-  for (int e = tid; e < k * k; e += nth) {
-    const int i = e / k, j = e % k;
-    const double* wi = W + (size_t)i * kFD;
-    const double* pj = P + (size_t)j * kFD;
-    double s = 0.0;
-    for (int l = 0; l < kFD; ++l) s += wi[l] * pj[l];
-    C[e] = s;
-  }
+  gram_small(W, P, C, k);
   __syncthreads();
   // Cholesky C = R^T R in place (upper triangle holds R); a pivot that has
   // vanished (rank-deficient sketch) makes its column of R and of T zero
@@ -282,15 +336,8 @@ __global__ void __launch_bounds__(kSThreads) rsvd_small_kernel(
     __syncthreads();
   }
   // C = T^T T; U = I
-  for (int e = tid; e < k * k; e += nth) {
-    const int i = e / k, j = e % k;
-    const double* ti = P + (size_t)i * kFD;
-    const double* tj = P + (size_t)j * kFD;
-    double s = 0.0;
-    for (int l = 0; l < kFD; ++l) s += ti[l] * tj[l];
-    C[e] = s;
-    U[e] = i == j ? 1.0 : 0.0;
-  }
+  gram_small(P, P, C, k);
+  for (int e = tid; e < k * k; e += nth) U[e] = (e / k == e % k) ? 1.0 : 0.0;
   __syncthreads();
   // cyclic Jacobi, round-robin pairing (k even): every round rotates k / 2
   // disjoint pairs; at most kFitSweeps sweeps (quadratic convergence), fewer
@@ -336,12 +383,14 @@ __global__ void __launch_bounds__(kSThreads) rsvd_small_kernel(
         }
         cs[q] = c;
         sn[q] = s;
+        pa[q] = a;
+        pb[q] = b;
       }
       __syncthreads();
       // columns: C <- C J, U <- U J
       for (int e = tid; e < k * half; e += nth) {
         const int i = e / half, q = e % half;
-        const int a = member(q), b = member(k - 1 - q);
+        const int a = pa[q], b = pb[q];
         const double c = cs[q], s = sn[q];
         const double x = C[i * k + a], y = C[i * k + b];
         C[i * k + a] = c * x - s * y;
@@ -354,7 +403,7 @@ __global__ void __launch_bounds__(kSThreads) rsvd_small_kernel(
       // rows: C <- J^T C
       for (int e = tid; e < k * half; e += nth) {
         const int j = e / half, q = e % half;
-        const int a = member(q), b = member(k - 1 - q);
+        const int a = pa[q], b = pb[q];
         const double c = cs[q], s = sn[q];
         const double x = C[a * k + j], y = C[b * k + j];
         C[a * k + j] = c * x - s * y;

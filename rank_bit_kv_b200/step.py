@@ -1,6 +1,6 @@
 """Run (and time) the decode step of a named synthetic workload.
 
-    python -m rank_bit_kv_b200.step c5 [--batch B] [--steps N] [--time]
+    python -m rank_bit_kv_b200.step c5 [--batch B] [--steps N] [--time] [--append]
 
 Builds the seeded synthetic cache of the workload (optionally with a smaller
 batch), then calls kvc_decode_attn N times on the current CUDA device.  With
@@ -8,6 +8,8 @@ batch), then calls kvc_decode_attn N times on the current CUDA device.  With
 median, the whole step (query projection, split-T kernel, combine) and the
 split-T kernel alone, both from CUDA events, with the compressed bytes the step
 reads.  Without --time it only runs the calls (the form used under a profiler).
+With --append (low-rank layouts) every step first appends one new token to
+slot T - 1 of every row with kvc_append, as the C5 workload's step does.
 """
 
 from __future__ import annotations
@@ -38,6 +40,8 @@ def main(argv=None):
     ap.add_argument("--time", action="store_true")
     ap.add_argument("--rope-kernel", type=int, default=0,
                     help="pre-RoPE layouts: 0 / 1 warp-level mma.sync kernel, 2 tcgen05 warpgroup kernel")
+    ap.add_argument("--append", action="store_true",
+                    help="low-rank layouts: one kvc_append of a new token per step")
     ap.add_argument("--varrate-kernel", type=int, default=0,
                     help="variable-rate layout: 0 lane-per-head kernel, 1 tensor-core kernel")
     args = ap.parse_args(argv)
@@ -55,9 +59,21 @@ def main(argv=None):
     q = torch.from_numpy(np.ascontiguousarray(fill["q"]).view(np.int16)).cuda().view(torch.bfloat16)
     out = torch.empty(q.shape, device="cuda")
     ws = torch.zeros(lay.workspace_bytes(c["T"]), dtype=torch.uint8, device="cuda")
+    app = None
+    if args.append and c["kind"] == "lowrank":
+        kn, vn = synth.new_tokens(c, 1)
+        app = (torch.from_numpy(kn.view(np.int16)).cuda().view(torch.bfloat16),
+               torch.from_numpy(vn.view(np.int16)).cuda().view(torch.bfloat16),
+               torch.full((c["B"],), c["T"] - 1, dtype=torch.int32, device="cuda"))
+
+    def step(events=None):
+        if app is not None:
+            kvc.append(lay, cache, app[0], app[1], app[2], 1)
+        kvc.decode(lay, cache, q, out, ws, events=events)
+
     if not args.time:
         for _ in range(args.steps):
-            kvc.decode(lay, cache, q, out, ws)
+            step()
         torch.cuda.synchronize()
         print(json.dumps({"config": args.config, "batch": c["B"], "steps": args.steps,
                           "finite": bool(torch.isfinite(out).all().item()),
@@ -65,7 +81,7 @@ def main(argv=None):
         return
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     for _ in range(3):
-        kvc.decode(lay, cache, q, out, ws)
+        step()
     torch.cuda.synchronize()
     step_us, kern_us = [], []
     for _ in range(args.steps):
@@ -73,7 +89,7 @@ def main(argv=None):
         ev = (kvc.RawEvent(), kvc.RawEvent())
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        kvc.decode(lay, cache, q, out, ws, events=ev)
+        step(ev)
         e1.record()
         torch.cuda.synchronize()
         step_us.append(e0.elapsed_time(e1) * 1e3)
