@@ -506,8 +506,9 @@ kvc_status kvc_allocate_rank_bits(int32_t n_cells, int32_t n_options, const doub
                                   double* lambda);
 
 /* Test switch (per calling thread, off by default): while on, decode calls
- * whose split kernel has bounded waits (the tcgen05 pre-RoPE kernel) enqueue
- * that kernel without its tile copies, so its waits run out after their limit
+ * whose split kernel has bounded waits (the tcgen05 pre-RoPE kernel, the
+ * block-shared tcgen05 kernel) enqueue that kernel without its tile copies or
+ * dequantisation, so its waits run out after their limit
  * (0.5 s), it sets KVC_DEV_WAIT_TIMEOUT in the workspace error word and exits
  * cleanly; the output of such a call is invalid.  Used to test that a wait
  * that gives up is reported and leaves the context usable.  No counterpart on

@@ -290,9 +290,11 @@ __global__ void __launch_bounds__(kThreads, 1) block_tc_kernel(Params p) {
     HalfRegs roA, rwA, roB, rwB;                   // tiles i (even) and i + 1
     if (n_tiles > 0) load_tile(0, roA, rwA);
     if (n_tiles > 1) load_tile(1, roB, rwB);
-    for (int i = 0; i < n_tiles; i += 2) {
+    // test switch: no tile is produced, so the other roles' bounded waits run out
+    const int n_prod = p.test_no_copies ? 0 : n_tiles;
+    for (int i = 0; i < n_prod; i += 2) {
       if (!produce(i, roA, rwA)) break;
-      if (i + 1 < n_tiles && !produce(i + 1, roB, rwB)) break;
+      if (i + 1 < n_prod && !produce(i + 1, roB, rwB)) break;
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-3)

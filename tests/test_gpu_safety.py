@@ -88,6 +88,34 @@ def test_bounded_wait_gives_up_reports_and_context_stays_usable():
     assert_close(out.cpu().numpy(), ref, what="decode after a timed-out call")
 
 
+def test_bounded_wait_of_the_block_shared_tensor_core_kernel():
+    """The same on the block-shared tcgen05 kernel: with the switch its
+    producers dequantise nothing, the MMA and softmax warps' waits run out,
+    the word is set, and the next call is correct."""
+    c = synth.config("c3", B=2, T=300)
+    a = synth.block_shared_cache(c)
+    ref = O.decode_from_storage(c, a, 300)
+    lay = kvc.Layout(kvc.desc_from_config(c))
+    cache = kvc.Cache(lay, fill=a)
+    cache.n_tokens = 300
+    q = to_dev_bf16(a["q"])
+    out = torch.empty(q.shape, device="cuda")
+    ws = torch.full((lay.workspace_bytes(300),), 0x5A, dtype=torch.uint8, device="cuda")
+    lib = kvc.lib()
+    lib.kvc_test_skip_tile_copies(1)
+    try:
+        kvc.decode(lay, cache, q, out, ws)
+        torch.cuda.synchronize()
+    finally:
+        lib.kvc_test_skip_tile_copies(0)
+    err = int(ws[:4].view(torch.int32).item())
+    assert err & kvc.DEV_WAIT_TIMEOUT, f"error word {err:#x}: the timeout was not reported"
+    kvc.decode(lay, cache, q, out, ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    assert_close(out.cpu().numpy(), ref, what="block-shared decode after a timed-out call")
+
+
 # ------------------------------------------------------------------ append: device-side checks
 
 
