@@ -78,8 +78,15 @@ __device__ void quant_int4_asym(const float* lat, int r, int g, uint8_t* codes, 
   __syncthreads();
 }
 
+// The factor's r rows are staged in shared memory first (coalesced 4-byte
+// loads, rows padded to kFsRow halves so that lane j reading row j is
+// conflict-free), so the projection and the residual read no global memory in
+// their loops.
+constexpr int kFsRow = 130;
+
 __global__ void __launch_bounds__(kThreads) append_lowrank_kernel(AppendParams a) {
   const Params& p = a.p;
+  __shared__ __align__(16) __half fsm[128 * kFsRow];
   __shared__ float xs[128];
   __shared__ float lat[128];
   __shared__ float lhat[128];
@@ -122,9 +129,14 @@ __global__ void __launch_bounds__(kThreads) append_lowrank_kernel(AppendParams a
     r = comp == 0 ? p.rk : p.rv;
     fac = (comp == 0 ? p.bk : p.bv) + (int64_t)h * r * d;
   }
+  for (int e = tid; e < r * (d / 2); e += kThreads) {
+    const int row = e / (d / 2), c2 = e % (d / 2);
+    *reinterpret_cast<uint32_t*>(fsm + row * kFsRow + 2 * c2) =
+        __ldg(reinterpret_cast<const unsigned int*>(fac + (int64_t)row * d + 2 * c2));
+  }
   __syncthreads();
   for (int j = tid; j < r; j += kThreads) {
-    const __half* br = fac + (int64_t)j * d;
+    const __half* br = fsm + j * kFsRow;
     float acc = 0.f;
     for (int k = 0; k < d; ++k) acc = fmaf(xs[k], h2f(br[k]), acc);
     lat[j] = acc;
@@ -158,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) append_lowrank_kernel(AppendParams a
   const int8_t* sg = comp == 0 ? p.signs_k : p.signs_v;
   for (int j = tid; j < d; j += kThreads) {
     float e = xs[j];
-    for (int k = 0; k < r; ++k) e = fmaf(-lhat[k], h2f(fac[(int64_t)k * d + j]), e);
+    for (int k = 0; k < r; ++k) e = fmaf(-lhat[k], h2f(fsm[k * kFsRow + j]), e);
     ys[j] = (float)sg[j] * e;
   }
   fwht_smem(ys, kResidDim, tid, kThreads);
