@@ -12,10 +12,19 @@
 //   acc_i += p_t (c_i s_g + z_g) for i < r_v(t).
 // Keeping q~ out of the registers lets 16 warps share an SM (4 per scheduler)
 // to hide the per-token dependency chain.
+// The arithmetic is paired: Blackwell's two-wide fp32 instructions
+// (fma/sub/mul .f32x2) take two elements per instruction.  Key codes enter the
+// dot product as f = 1 + c/16 (exact: the nibble is placed in the top mantissa
+// bits), so sum q_i c_i = 16 (sum q_i f_i - sum q_i) needs no per-code
+// subtraction; value codes are centred, c - 8, and the zero terms p (z + 8 s)
+// of the tokens are summed per rank class and added to the accumulator once,
+// at the end, over the indices each class covers.
 // Every warp streams a contiguous token range in chunks of 8 tokens: the byte
 // range of the chunk's K records and of its V records (contiguous in the
 // per-row streams) is copied with 16-byte cp.async into a double-buffered
-// per-warp area while the previous chunk is processed.  The warps of a CTA
+// per-warp area while the previous chunk is processed.  The chunk's records are validated once
+// (offsets on their 16-byte grid and inside the staged area, ranks in the
+// rank set), by the lane that holds the token's metadata.  The warps of a CTA
 // merge their (m, l, acc) in shared memory and write one partial per row; the
 // combine kernel maps acc through Bv.
 #include <math.h>
@@ -45,6 +54,7 @@ constexpr int kVPst = kVRmax + 2;                   // merge slot: acc[64], m, l
 
 static_assert(kVWarps * 32 * kVPst * 4 <= kVStage, "merge area fits in the staging area");
 static_assert(kVThreads == kVHkv * kVRmax, "one thread per (KV head, rank) row of Bk");
+static_assert(kVHkv * kVRmax * 256 <= kVStage, "Bk's copy fits in the staging area");
 
 __host__ __device__ constexpr int head_bytes(int r) { return r / 2 + 4 * ((r + 31) / 32); }
 
@@ -63,24 +73,68 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
-// the 8 nibbles of w as floats (exact): each nibble is moved into the low byte
-// of the bit pattern 0x4B0000xx = 2^23 + c, and 2^23 is subtracted
-__device__ __forceinline__ void nib8(uint32_t w, float (&c)[8]) {
-  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    c[2 * j] = __int_as_float(prmt(lo, 0x4B000000u, 0x7650u + j)) - 8388608.f;
-    c[2 * j + 1] = __int_as_float(prmt(hi, 0x4B000000u, 0x7650u + j)) - 8388608.f;
-  }
+// ---- two-wide fp32 arithmetic (element 0 in the low word)
+__device__ __forceinline__ uint64_t pk2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t pkf(float lo, float hi) {
+  return pk2(__float_as_uint(lo), __float_as_uint(hi));
+}
+__device__ __forceinline__ float2 upk(uint64_t v) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// key codes of word w (nibble 2j = low nibble of byte j, 2j+1 = high nibble) as
+// the pairs (1 + c_2j/16, 1 + c_2j+1/16): each nibble is moved to mantissa bits
+// 19..22 of the bit pattern of 1.0 (exact)
+__device__ __forceinline__ uint64_t key_pair(uint32_t lo, uint32_t hi, int j) {
+  const uint32_t sel = 0x7044u | ((uint32_t)j << 8);
+  return pk2(prmt(lo, 0x3F000000u, sel), prmt(hi, 0x3F000000u, sel));
+}
+__device__ __forceinline__ void key_words(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  lo = ((w << 3) & 0x78787878u) | 0x80808080u;
+  hi = ((w >> 1) & 0x78787878u) | 0x80808080u;
+}
+
+// value codes of word w, centred: the pairs (c_2j - 8, c_2j+1 - 8), formed as
+// (2^23 + c) - (2^23 + 8) (exact)
+__device__ __forceinline__ uint64_t value_pair(uint32_t lo, uint32_t hi, int j) {
+  const uint32_t sel = 0x7650u + (uint32_t)j;
+  return sub2(pk2(prmt(lo, 0x4B000000u, sel), prmt(hi, 0x4B000000u, sel)),
+              pkf(8388616.f, 8388616.f));
 }
 
 __device__ __forceinline__ float2 h2f2(uint32_t x) {
   return __half22float2(*reinterpret_cast<const __half2*>(&x));
 }
+__device__ __forceinline__ float hsum(uint64_t v) {
+  const float2 f = upk(v);
+  return f.x + f.y;
+}
 
 // sum_{i < R} q_i (c_i s_g + z_g) over the record at rec (R/2 code bytes, then
-// the groups' (scale, zero) pairs); pre = prefix sums of q
-// (q = this lane's row of q~ in shared memory)
+// the groups' (scale, zero) pairs); q = this lane's row of q~ in shared memory,
+// pre = its prefix sums: with f_i = 1 + c_i/16,
+//   sum_g [16 s_g sum_{i in g} q_i f_i + (z_g - 16 s_g) sum_{i in g} q_i]
 template <int R>
 __device__ __forceinline__ float score_r(const uint8_t* rec, const float* q,
                                          const float (&pre)[5]) {
@@ -88,80 +142,87 @@ __device__ __forceinline__ float score_r(const uint8_t* rec, const float* q,
     const uint32_t w = *reinterpret_cast<const uint16_t*>(rec);
     const float s = __half2float(*reinterpret_cast<const __half*>(rec + 2));
     const float z = __half2float(*reinterpret_cast<const __half*>(rec + 4));
-    const float4 q0 = *reinterpret_cast<const float4*>(q);
-    float c[8];
-    nib8(w, c);
-    float d = c[0] * q0.x;
-    d = fmaf(c[1], q0.y, d);
-    d = fmaf(c[2], q0.z, d);
-    d = fmaf(c[3], q0.w, d);
-    return fmaf(s, d, z * pre[0]);
+    const ulonglong2 qv = *reinterpret_cast<const ulonglong2*>(q);
+    uint32_t lo, hi;
+    key_words(w, lo, hi);
+    const float d = hsum(fma2(key_pair(lo, hi, 1), qv.y, mul2(key_pair(lo, hi, 0), qv.x)));
+    return fmaf(16.f * s, d, fmaf(-16.f, s, z) * pre[0]);
   } else {
     constexpr int NW = R / 8;
-    float dw[NW];                       // one chain per code word (short dependency chains)
+    uint64_t dw[NW];                    // one chain per code word (short dependency chains)
 #pragma unroll
     for (int wi = 0; wi < NW; ++wi) {
-      const float4 qa = *reinterpret_cast<const float4*>(q + 8 * wi);
-      const float4 qb = *reinterpret_cast<const float4*>(q + 8 * wi + 4);
-      const float qq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-      float c[8];
-      nib8(*reinterpret_cast<const uint32_t*>(rec + 4 * wi), c);
-      float a = c[0] * qq[0];
-#pragma unroll
-      for (int k = 1; k < 8; ++k) a = fmaf(c[k], qq[k], a);
-      dw[wi] = a;
+      const ulonglong2 qa = *reinterpret_cast<const ulonglong2*>(q + 8 * wi);
+      const ulonglong2 qb = *reinterpret_cast<const ulonglong2*>(q + 8 * wi + 4);
+      uint32_t lo, hi;
+      key_words(*reinterpret_cast<const uint32_t*>(rec + 4 * wi), lo, hi);
+      uint64_t a = mul2(key_pair(lo, hi, 0), qa.x);
+      a = fma2(key_pair(lo, hi, 1), qa.y, a);
+      a = fma2(key_pair(lo, hi, 2), qb.x, a);
+      dw[wi] = fma2(key_pair(lo, hi, 3), qb.y, a);
     }
     float d[2] = {0.f, 0.f};
 #pragma unroll
-    for (int wi = 0; wi < NW; ++wi) d[wi / 4] += dw[wi];
+    for (int wi = 0; wi < NW; ++wi) d[wi / 4] += hsum(dw[wi]);
     const float2 sz0 = h2f2(*reinterpret_cast<const uint32_t*>(rec + R / 2));
     constexpr int P = R == 8 ? 1 : R == 16 ? 2 : 3;     // prefix of group 0 up to min(R, 32)
-    float s = fmaf(sz0.x, d[0], sz0.y * pre[P]);
+    float s = fmaf(16.f * sz0.x, d[0], fmaf(-16.f, sz0.x, sz0.y) * pre[P]);
     if constexpr (R == 64) {
       const float2 sz1 = h2f2(*reinterpret_cast<const uint32_t*>(rec + R / 2 + 4));
-      s += fmaf(sz1.x, d[1], sz1.y * pre[4]);
+      s += fmaf(16.f * sz1.x, d[1], fmaf(-16.f, sz1.x, sz1.y) * pre[4]);
     }
     return s;
   }
 }
 
-// acc_i += p (c_i s_g + z_g) for i < R
+// the per-class sums of p (z_g + 8 s_g): index 0..3 for ranks 4..32 (group 0),
+// 4 and 5 for the two groups of rank 64; the accumulator takes
+//   acc_i += p s_g (c_i - 8) for i < R
+// and the class sums are added at the end over the indices each class covers
 template <int R>
-__device__ __forceinline__ void value_r(const uint8_t* rec, float p, float (&acc)[kVRmax]) {
+__device__ __forceinline__ void value_r(const uint8_t* rec, float p, uint64_t (&acc)[kVRmax / 2],
+                                        float (&zc)[6]) {
   if constexpr (R == 4) {
     const uint32_t w = *reinterpret_cast<const uint16_t*>(rec);
-    const float ps = p * __half2float(*reinterpret_cast<const __half*>(rec + 2));
-    const float pz = p * __half2float(*reinterpret_cast<const __half*>(rec + 4));
-    float c[8];
-    nib8(w, c);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = fmaf(ps, c[k], acc[k] + pz);
+    const float s = __half2float(*reinterpret_cast<const __half*>(rec + 2));
+    const float z = __half2float(*reinterpret_cast<const __half*>(rec + 4));
+    const float ps = p * s;
+    zc[0] = fmaf(p, fmaf(8.f, s, z), zc[0]);
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    const uint64_t ps2 = pkf(ps, ps);
+    acc[0] = fma2(ps2, value_pair(lo, hi, 0), acc[0]);
+    acc[1] = fma2(ps2, value_pair(lo, hi, 1), acc[1]);
   } else {
     constexpr int NW = R / 8;
-    float ps[2], pz[2];
+    constexpr int ZC = R == 8 ? 1 : R == 16 ? 2 : R == 32 ? 3 : 4;
+    uint64_t ps2[2];
     {
       const float2 sz0 = h2f2(*reinterpret_cast<const uint32_t*>(rec + R / 2));
-      ps[0] = p * sz0.x;
-      pz[0] = p * sz0.y;
+      const float ps = p * sz0.x;
+      ps2[0] = pkf(ps, ps);
+      zc[ZC] = fmaf(p, fmaf(8.f, sz0.x, sz0.y), zc[ZC]);
       if constexpr (R == 64) {
         const float2 sz1 = h2f2(*reinterpret_cast<const uint32_t*>(rec + R / 2 + 4));
-        ps[1] = p * sz1.x;
-        pz[1] = p * sz1.y;
+        const float ps1 = p * sz1.x;
+        ps2[1] = pkf(ps1, ps1);
+        zc[5] = fmaf(p, fmaf(8.f, sz1.x, sz1.y), zc[5]);
       } else {
-        ps[1] = pz[1] = 0.f;
+        ps2[1] = ps2[0];
       }
     }
 #pragma unroll
     for (int wi = 0; wi < NW; ++wi) {
-      float c[8];
-      nib8(*reinterpret_cast<const uint32_t*>(rec + 4 * wi), c);
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(rec + 4 * wi);
+      const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int i = 8 * wi + k;
-        acc[i] = fmaf(ps[wi / 4], c[k], acc[i] + pz[wi / 4]);
-      }
+      for (int j = 0; j < 4; ++j)
+        acc[4 * wi + j] = fma2(ps2[wi / 4], value_pair(lo, hi, j), acc[4 * wi + j]);
     }
   }
+}
+
+__device__ __forceinline__ bool rank_in_set(int r) {
+  return r == 4 || r == 8 || r == 16 || r == 32 || r == 64;
 }
 
 __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, int split_len) {
@@ -184,36 +245,117 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   const uint8_t* const rv = p.rank_v + (size_t)b * p.tmax;
   const long long sbytes = (long long)p.stream_bytes;
 
+  // ---- chunk staging: the byte ranges [off[t0], off[t0 + n]) of both streams,
+  // from the 16-byte boundary below, clamped to the stream and the buffer.
+  // A chunk's metadata (lane j <= n: offsets, lane j < n: ranks of token
+  // t0 + j) is loaded one chunk before its copies are issued, so the copies of
+  // chunk c + 1 never wait for memory; lane j < n then keeps token t0 + j's
+  // offsets (relative to the staged areas) and ranks, and the chunk's validity
+  // mask is formed once, at issue
+  struct Raw {
+    int ok, ov, rkv;
+  };
+  struct Meta {
+    int ok, ov, rkv;                    // lane j < n: offsets and ranks (rk | rv << 8) of token t0 + j
+    uint32_t valid;                     // bit j: token t0 + j's records lie in the staged areas
+  };
+  auto meta_load = [&](int t0) -> Raw {
+    const int n = min(kVChunk, t_b - t0);
+    Raw r;
+    r.ok = lane <= n ? __ldg(offk + t0 + lane) : 0;
+    r.ov = lane <= n ? __ldg(offv + t0 + lane) : 0;
+    r.rkv = lane < n ? (int)__ldg(rk + t0 + lane) | ((int)__ldg(rv + t0 + lane) << 8) : 0;
+    return r;
+  };
+  auto stage = [&](const Raw& r, int t0, int buf) -> Meta {
+    const int n = min(kVChunk, t_b - t0);
+    Meta mt;
+    mt.rkv = r.rkv;
+    const int k0 = __shfl_sync(0xffffffffu, r.ok, 0), k1 = __shfl_sync(0xffffffffu, r.ok, n);
+    const int v0 = __shfl_sync(0xffffffffu, r.ov, 0), v1 = __shfl_sync(0xffffffffu, r.ov, n);
+    const int base_k = k0 & ~15, base_v = v0 & ~15;
+    const uint32_t dk = area_s + (2 * buf) * kVBuf, dv = area_s + (2 * buf + 1) * kVBuf;
+    const long long ek = min((long long)k1, sbytes), ev = min((long long)v1, sbytes);
+    const int nk = (int)min((ek - base_k + 15) / 16, (long long)(kVBuf / 16));
+    const int nv = (int)min((ev - base_v + 15) / 16, (long long)(kVBuf / 16));
+    for (int c = lane; c < nk; c += 32) cp16(dk + 16 * c, kstream + base_k + 16 * c);
+    for (int c = lane; c < nv; c += 32) cp16(dv + 16 * c, vstream + base_v + 16 * c);
+    // records outside the staged areas or off their 16-byte grid (offsets
+    // inconsistent with the ranks), or ranks outside the set, are skipped
+    mt.ok = r.ok - base_k;
+    mt.ov = r.ov - base_v;
+    const int r_k = mt.rkv & 255, r_v = mt.rkv >> 8;
+    const bool good = lane < n && rank_in_set(r_k) && rank_in_set(r_v) && mt.ok >= 0 &&
+                      !(mt.ok & 15) && mt.ok + kVHkv * head_bytes(r_k) <= 16 * nk &&
+                      mt.ov >= 0 && !(mt.ov & 15) && mt.ov + kVHkv * head_bytes(r_v) <= 16 * nv;
+    mt.valid = __ballot_sync(0xffffffffu, good);
+    return mt;
+  };
+
+  Meta cur{}, nxt{};
+  Raw raw0{}, raw1{};                   // metadata of the current and of the next chunk
+  int t0 = t_a, buf = 0;
+  if (t0 < t_b) raw0 = meta_load(t0);   // in flight during the query projection
+  if (t0 + kVChunk < t_b) raw1 = meta_load(t0 + kVChunk);
+
   // ---- q~ = Bk q for the row's 32 query heads (softmax scale and log2 e
-  // folded in): thread (kvh, j) dots row j of head kvh's Bk with its 4 queries
+  // folded in).  Bk (8 heads x 64 rows x 128, fp16) is first copied into the
+  // staging area with coalesced 16-byte copies, row r's 16-byte piece c at
+  // r * 256 + (c ^ (r & 15)) * 16 (conflict-free row reads); then thread
+  // (kvh, j) dots row j of head kvh's Bk with its 4 queries
   float* const qsm = reinterpret_cast<float*>(vsm + kVOffQ);
   {
-    float* const xs = reinterpret_cast<float*>(vsm + kVOffX);
-    for (int e = threadIdx.x; e < 32 * 128; e += kVThreads)
-      xs[e] = bf2f(p.q[(size_t)b * p.Hq * 128 + e]);
-    __syncthreads();
-    const int kvh = threadIdx.x / kVRmax, j = threadIdx.x % kVRmax;
-    const uint4* br = reinterpret_cast<const uint4*>(p.bk + ((size_t)kvh * kVRmax + j) * 128);
-    float a4[kVG] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+    const uint32_t bks = smem_u32(vsm);
+#pragma unroll
     for (int c = 0; c < 16; ++c) {
-      const uint4 w = __ldg(br + c);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      const int idx = c * kVThreads + threadIdx.x, r = idx >> 4, pc = idx & 15;
+      cp16(bks + r * 256 + ((pc ^ (r & 15)) << 4), p.bk + (size_t)idx * 8);
+    }
+    cp_commit();
+    float* const xs = reinterpret_cast<float*>(vsm + kVOffX);
+    {
+      // the row's 32 x 128 bf16 queries, 8 per thread (one 16-byte load)
+      const uint4 xq = __ldg(reinterpret_cast<const uint4*>(p.q + (size_t)b * p.Hq * 128) +
+                             threadIdx.x);
+      const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+      float4* xd = reinterpret_cast<float4*>(xs + 8 * threadIdx.x);
+      float v[8];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float2 f = h2f2(ws[k]);
+        v[2 * k] = __uint_as_float(xw[k] << 16);
+        v[2 * k + 1] = __uint_as_float(xw[k] & 0xFFFF0000u);
+      }
+      xd[0] = make_float4(v[0], v[1], v[2], v[3]);
+      xd[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    cp_wait<0>();
+    __syncthreads();
+    const int kvh = threadIdx.x / kVRmax, j = threadIdx.x % kVRmax, r = threadIdx.x;
+    const uint8_t* brow = vsm + r * 256;
+    uint64_t a2[kVG] = {0ull, 0ull, 0ull, 0ull};
+    const float* xk = xs + kvh * kVG * 128;
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+      const uint4 w = *reinterpret_cast<const uint4*>(brow + ((c ^ (r & 15)) << 4));
+      const float2 f0 = h2f2(w.x), f1 = h2f2(w.y), f2 = h2f2(w.z), f3 = h2f2(w.w);
+      const uint64_t b0 = pkf(f0.x, f0.y), b1 = pkf(f1.x, f1.y);
+      const uint64_t b2 = pkf(f2.x, f2.y), b3 = pkf(f3.x, f3.y);
 #pragma unroll
-        for (int g = 0; g < kVG; ++g) {
-          const float* xg = xs + (kvh * kVG + g) * 128 + 8 * c + 2 * k;
-          a4[g] = fmaf(f.x, xg[0], a4[g]);
-          a4[g] = fmaf(f.y, xg[1], a4[g]);
-        }
+      for (int g = 0; g < kVG; ++g) {
+        const ulonglong2 xa = *reinterpret_cast<const ulonglong2*>(xk + g * 128 + 8 * c);
+        const ulonglong2 xb = *reinterpret_cast<const ulonglong2*>(xk + g * 128 + 8 * c + 4);
+        a2[g] = fma2(b0, xa.x, a2[g]);
+        a2[g] = fma2(b1, xa.y, a2[g]);
+        a2[g] = fma2(b2, xb.x, a2[g]);
+        a2[g] = fma2(b3, xb.y, a2[g]);
       }
     }
 #pragma unroll
-    for (int g = 0; g < kVG; ++g) qsm[(kvh * kVG + g) * kVQRow + j] = a4[g] * p.scale_log2;
-    __syncthreads();
+    for (int g = 0; g < kVG; ++g) qsm[(kvh * kVG + g) * kVQRow + j] = hsum(a2[g]) * p.scale_log2;
+    __syncthreads();                    // Bk's copy in the staging area is dead from here
   }
+  if (t0 < t_b) cur = stage(raw0, t0, 0);
+  cp_commit();
   const float* const q = qsm + lane * kVQRow;       // lane = h * 4 + qi
   float pre[5];
   {
@@ -229,103 +371,86 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
       if (i == 63) pre[4] = run;
     }
   }
-  float acc[kVRmax];
+  uint64_t acc[kVRmax / 2];
 #pragma unroll
-  for (int i = 0; i < kVRmax; ++i) acc[i] = 0.f;
+  for (int i = 0; i < kVRmax / 2; ++i) acc[i] = 0ull;
+  float zc[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float m = -INFINITY, m_thr = -INFINITY, l = 0.f;
 
-  // ---- chunk staging: the byte ranges [off[t0], off[t0 + n]) of both streams,
-  // from the 16-byte boundary below, clamped to the stream and the buffer
-  struct Meta {
-    int ok, ov, rkv;                    // lane j < n: offsets and ranks (rk | rv << 8) of token t0 + j
-    int base_k, base_v;                 // stream offsets of the staged areas' first byte
-  };
-  auto stage = [&](int t0, int buf) -> Meta {
-    const int n = min(kVChunk, t_b - t0);
-    Meta mt;
-    mt.ok = lane <= n ? __ldg(offk + t0 + lane) : 0;
-    mt.ov = lane <= n ? __ldg(offv + t0 + lane) : 0;
-    mt.rkv = lane < n ? (int)__ldg(rk + t0 + lane) | ((int)__ldg(rv + t0 + lane) << 8) : 0;
-    const int k0 = __shfl_sync(0xffffffffu, mt.ok, 0), k1 = __shfl_sync(0xffffffffu, mt.ok, n);
-    const int v0 = __shfl_sync(0xffffffffu, mt.ov, 0), v1 = __shfl_sync(0xffffffffu, mt.ov, n);
-    mt.base_k = k0 & ~15;
-    mt.base_v = v0 & ~15;
-    const uint32_t dk = area_s + (2 * buf) * kVBuf, dv = area_s + (2 * buf + 1) * kVBuf;
-    const long long ek = min((long long)k1, sbytes), ev = min((long long)v1, sbytes);
-    const int nk = (int)min((ek - mt.base_k + 15) / 16, (long long)(kVBuf / 16));
-    const int nv = (int)min((ev - mt.base_v + 15) / 16, (long long)(kVBuf / 16));
-    for (int c = lane; c < nk; c += 32) cp16(dk + 16 * c, kstream + mt.base_k + 16 * c);
-    for (int c = lane; c < nv; c += 32) cp16(dv + 16 * c, vstream + mt.base_v + 16 * c);
-    return mt;
-  };
-
-  Meta cur{}, nxt{};
-  int t0 = t_a, buf = 0;
-  if (t0 < t_b) cur = stage(t0, 0);
-  cp_commit();
   while (t0 < t_b) {
     const int n = min(kVChunk, t_b - t0);
     const int t1 = t0 + n;
-    if (t1 < t_b) nxt = stage(t1, buf ^ 1);
+    Raw raw2{};
+    if (t1 + kVChunk < t_b) raw2 = meta_load(t1 + kVChunk);
+    if (t1 < t_b) nxt = stage(raw1, t1, buf ^ 1);
     cp_commit();
     cp_wait<1>();
     __syncwarp();
     const uint8_t* kb = area + (2 * buf) * kVBuf;
     const uint8_t* vb = area + (2 * buf + 1) * kVBuf;
     for (int j = 0; j < n; ++j) {
-      const int ok = __shfl_sync(0xffffffffu, cur.ok, j) - cur.base_k;
-      const int ov = __shfl_sync(0xffffffffu, cur.ov, j) - cur.base_v;
+      const int ok = __shfl_sync(0xffffffffu, cur.ok, j);
+      const int ov = __shfl_sync(0xffffffffu, cur.ov, j);
       const int rkv = __shfl_sync(0xffffffffu, cur.rkv, j);
+      if (!((cur.valid >> j) & 1u)) continue;
       const int r_k = rkv & 255, r_v = rkv >> 8;
-      // records outside the staged area or off their 16-byte grid (offsets
-      // inconsistent with the ranks) are skipped
-      if (ok < 0 || (ok & 15) || ok + kVHkv * head_bytes(r_k) > kVBuf || ov < 0 || (ov & 15) ||
-          ov + kVHkv * head_bytes(r_v) > kVBuf)
-        continue;
       float s;
-      const uint8_t* krec = kb + ok + h * head_bytes(r_k);
+      const uint8_t* kr = kb + ok;
       switch (r_k) {
-        case 4: s = score_r<4>(krec, q, pre); break;
-        case 8: s = score_r<8>(krec, q, pre); break;
-        case 16: s = score_r<16>(krec, q, pre); break;
-        case 32: s = score_r<32>(krec, q, pre); break;
-        case 64: s = score_r<64>(krec, q, pre); break;
-        default: continue;
+        case 4: s = score_r<4>(kr + h * head_bytes(4), q, pre); break;
+        case 8: s = score_r<8>(kr + h * head_bytes(8), q, pre); break;
+        case 16: s = score_r<16>(kr + h * head_bytes(16), q, pre); break;
+        case 32: s = score_r<32>(kr + h * head_bytes(32), q, pre); break;
+        default: s = score_r<64>(kr + h * head_bytes(64), q, pre); break;
       }
       if (s > m_thr) {                  // lazily raised maximum (by more than 2^8)
         const float a = ex2_approx(m - s);
         l *= a;
+        const uint64_t a2 = pkf(a, a);
 #pragma unroll
-        for (int i = 0; i < kVRmax; ++i) acc[i] *= a;
+        for (int i = 0; i < kVRmax / 2; ++i) acc[i] = mul2(acc[i], a2);
+#pragma unroll
+        for (int i = 0; i < 6; ++i) zc[i] *= a;
         m = s;
         m_thr = s + 8.f;
       }
       const float pr = ex2_approx(s - m);
       l += pr;
-      const uint8_t* vrec = vb + ov + h * head_bytes(r_v);
+      const uint8_t* vr = vb + ov;
       switch (r_v) {
-        case 4: value_r<4>(vrec, pr, acc); break;
-        case 8: value_r<8>(vrec, pr, acc); break;
-        case 16: value_r<16>(vrec, pr, acc); break;
-        case 32: value_r<32>(vrec, pr, acc); break;
-        case 64: value_r<64>(vrec, pr, acc); break;
-        default: break;
+        case 4: value_r<4>(vr + h * head_bytes(4), pr, acc, zc); break;
+        case 8: value_r<8>(vr + h * head_bytes(8), pr, acc, zc); break;
+        case 16: value_r<16>(vr + h * head_bytes(16), pr, acc, zc); break;
+        case 32: value_r<32>(vr + h * head_bytes(32), pr, acc, zc); break;
+        default: value_r<64>(vr + h * head_bytes(64), pr, acc, zc); break;
       }
     }
     __syncwarp();                       // this buffer is refilled by the next stage
     cur = nxt;
+    raw1 = raw2;
     t0 = t1;
     buf ^= 1;
   }
   cp_wait<0>();
   __syncthreads();
 
-  // ---- merge the warps of this CTA, one partial per row
+  // ---- merge the warps of this CTA, one partial per row; the class sums of
+  // the zero terms join the accumulator first (class of rank R covers i < R)
   float* mg = reinterpret_cast<float*>(vsm);
   {
     float* slot = mg + (warp * 32 + lane) * kVPst;
+    const float z3 = zc[3] + zc[4];     // 16 <= i < 32: ranks 32, 64
+    const float z2 = zc[2] + z3;        // 8 <= i < 16: and 16
+    const float z1 = zc[1] + z2;        // 4 <= i < 8: and 8
+    const float z0 = zc[0] + z1;        // i < 4: and 4
 #pragma unroll
-    for (int i = 0; i < kVRmax; ++i) slot[i] = acc[i];
+    for (int i = 0; i < kVRmax / 2; ++i) {
+      const float2 v = upk(acc[i]);
+      const int e = 2 * i;
+      const float z = e < 4 ? z0 : e < 8 ? z1 : e < 16 ? z2 : e < 32 ? z3 : zc[5];
+      slot[e] = v.x + z;
+      slot[e + 1] = v.y + z;
+    }
     slot[kVRmax] = m;
     slot[kVRmax + 1] = l;
   }
