@@ -22,9 +22,10 @@
 // Every warp streams a contiguous token range in chunks of 8 tokens: the byte
 // range of the chunk's K records and of its V records (contiguous in the
 // per-row streams) is copied with 16-byte cp.async into a double-buffered
-// per-warp area while the previous chunk is processed.  The chunk's records are validated once
-// (offsets on their 16-byte grid and inside the staged area, ranks in the
-// rank set), by the lane that holds the token's metadata.  The warps of a CTA
+// per-warp area while the previous chunk is processed.  The chunk's records are
+// validated once (offsets on their 16-byte grid and inside the staged area,
+// ranks in the rank set), by the lane that holds the token's metadata, which
+// packs offsets, rank classes and the verdict into one word.  The warps of a CTA
 // merge their (m, l, acc) in shared memory and write one partial per row; the
 // combine kernel maps acc through Bv.
 #include <math.h>
@@ -55,6 +56,7 @@ constexpr int kVPst = kVRmax + 2;                   // merge slot: acc[64], m, l
 static_assert(kVWarps * 32 * kVPst * 4 <= kVStage, "merge area fits in the staging area");
 static_assert(kVThreads == kVHkv * kVRmax, "one thread per (KV head, rank) row of Bk");
 static_assert(kVHkv * kVRmax * 256 <= kVStage, "Bk's copy fits in the staging area");
+static_assert(kVBuf <= 4096, "record offsets in a staged chunk fit in 12 bits");
 
 __host__ __device__ constexpr int head_bytes(int r) { return r / 2 + 4 * ((r + 31) / 32); }
 
@@ -256,8 +258,10 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     int ok, ov, rkv;
   };
   struct Meta {
-    int ok, ov, rkv;                    // lane j < n: offsets and ranks (rk | rv << 8) of token t0 + j
-    uint32_t valid;                     // bit j: token t0 + j's records lie in the staged areas
+    // lane j < n: token t0 + j's K and V record offsets in the staged areas
+    // (bits 0-11, 12-23), rank classes (log2 r - 2; bits 24-26, 27-29) and
+    // bit 30 set when its records lie in the staged areas; one shuffle per token
+    uint32_t w;
   };
   auto meta_load = [&](int t0) -> Raw {
     const int n = min(kVChunk, t_b - t0);
@@ -270,7 +274,6 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   auto stage = [&](const Raw& r, int t0, int buf) -> Meta {
     const int n = min(kVChunk, t_b - t0);
     Meta mt;
-    mt.rkv = r.rkv;
     const int k0 = __shfl_sync(0xffffffffu, r.ok, 0), k1 = __shfl_sync(0xffffffffu, r.ok, n);
     const int v0 = __shfl_sync(0xffffffffu, r.ov, 0), v1 = __shfl_sync(0xffffffffu, r.ov, n);
     const int base_k = k0 & ~15, base_v = v0 & ~15;
@@ -282,13 +285,14 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     for (int c = lane; c < nv; c += 32) cp16(dv + 16 * c, vstream + base_v + 16 * c);
     // records outside the staged areas or off their 16-byte grid (offsets
     // inconsistent with the ranks), or ranks outside the set, are skipped
-    mt.ok = r.ok - base_k;
-    mt.ov = r.ov - base_v;
-    const int r_k = mt.rkv & 255, r_v = mt.rkv >> 8;
-    const bool good = lane < n && rank_in_set(r_k) && rank_in_set(r_v) && mt.ok >= 0 &&
-                      !(mt.ok & 15) && mt.ok + kVHkv * head_bytes(r_k) <= 16 * nk &&
-                      mt.ov >= 0 && !(mt.ov & 15) && mt.ov + kVHkv * head_bytes(r_v) <= 16 * nv;
-    mt.valid = __ballot_sync(0xffffffffu, good);
+    const int ok = r.ok - base_k, ov = r.ov - base_v;
+    const int r_k = r.rkv & 255, r_v = r.rkv >> 8;
+    const bool good = lane < n && rank_in_set(r_k) && rank_in_set(r_v) && ok >= 0 &&
+                      !(ok & 15) && ok + kVHkv * head_bytes(r_k) <= 16 * nk &&
+                      ov >= 0 && !(ov & 15) && ov + kVHkv * head_bytes(r_v) <= 16 * nv;
+    mt.w = good ? (uint32_t)ok | ((uint32_t)ov << 12) | ((uint32_t)(__ffs(r_k) - 3) << 24) |
+                      ((uint32_t)(__ffs(r_v) - 3) << 27) | (1u << 30)
+                : 0u;
     return mt;
   };
 
@@ -389,18 +393,15 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     const uint8_t* kb = area + (2 * buf) * kVBuf;
     const uint8_t* vb = area + (2 * buf + 1) * kVBuf;
     for (int j = 0; j < n; ++j) {
-      const int ok = __shfl_sync(0xffffffffu, cur.ok, j);
-      const int ov = __shfl_sync(0xffffffffu, cur.ov, j);
-      const int rkv = __shfl_sync(0xffffffffu, cur.rkv, j);
-      if (!((cur.valid >> j) & 1u)) continue;
-      const int r_k = rkv & 255, r_v = rkv >> 8;
+      const uint32_t w = __shfl_sync(0xffffffffu, cur.w, j);
+      if (!(w >> 30)) continue;
       float s;
-      const uint8_t* kr = kb + ok;
-      switch (r_k) {
-        case 4: s = score_r<4>(kr + h * head_bytes(4), q, pre); break;
-        case 8: s = score_r<8>(kr + h * head_bytes(8), q, pre); break;
-        case 16: s = score_r<16>(kr + h * head_bytes(16), q, pre); break;
-        case 32: s = score_r<32>(kr + h * head_bytes(32), q, pre); break;
+      const uint8_t* kr = kb + (w & 0xFFFu);
+      switch ((w >> 24) & 7u) {
+        case 0: s = score_r<4>(kr + h * head_bytes(4), q, pre); break;
+        case 1: s = score_r<8>(kr + h * head_bytes(8), q, pre); break;
+        case 2: s = score_r<16>(kr + h * head_bytes(16), q, pre); break;
+        case 3: s = score_r<32>(kr + h * head_bytes(32), q, pre); break;
         default: s = score_r<64>(kr + h * head_bytes(64), q, pre); break;
       }
       if (s > m_thr) {                  // lazily raised maximum (by more than 2^8)
@@ -416,12 +417,12 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
       }
       const float pr = ex2_approx(s - m);
       l += pr;
-      const uint8_t* vr = vb + ov;
-      switch (r_v) {
-        case 4: value_r<4>(vr + h * head_bytes(4), pr, acc, zc); break;
-        case 8: value_r<8>(vr + h * head_bytes(8), pr, acc, zc); break;
-        case 16: value_r<16>(vr + h * head_bytes(16), pr, acc, zc); break;
-        case 32: value_r<32>(vr + h * head_bytes(32), pr, acc, zc); break;
+      const uint8_t* vr = vb + ((w >> 12) & 0xFFFu);
+      switch ((w >> 27) & 7u) {
+        case 0: value_r<4>(vr + h * head_bytes(4), pr, acc, zc); break;
+        case 1: value_r<8>(vr + h * head_bytes(8), pr, acc, zc); break;
+        case 2: value_r<16>(vr + h * head_bytes(16), pr, acc, zc); break;
+        case 3: value_r<32>(vr + h * head_bytes(32), pr, acc, zc); break;
         default: value_r<64>(vr + h * head_bytes(64), pr, acc, zc); break;
       }
     }
@@ -480,6 +481,7 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     dst[p.vdim] = M;
     dst[p.vdim + 1] = L;
   }
+
 }
 
 }  // namespace

@@ -263,6 +263,7 @@ class RawEvent:
             rt.cudaEventCreate.argtypes = [C.POINTER(C.c_void_p)]
             rt.cudaEventElapsedTime.argtypes = [C.POINTER(C.c_float), C.c_void_p, C.c_void_p]
             rt.cudaEventDestroy.argtypes = [C.c_void_p]
+            rt.cudaEventRecord.argtypes = [C.c_void_p, C.c_void_p]
             cls._rt = rt
         return cls._rt
 
@@ -280,6 +281,13 @@ class RawEvent:
         if err != 0:
             raise RuntimeError(f"cudaEventElapsedTime failed ({err})")
         return ms.value
+
+    def record(self, stream=None):
+        """Record the event on `stream` (default: torch's current stream)."""
+        st = stream if stream is not None else current_stream_ptr()
+        err = self.rt().cudaEventRecord(C.c_void_p(self.cuda_event), st)
+        if err != 0:
+            raise RuntimeError(f"cudaEventRecord failed ({err})")
 
     def __del__(self):
         if self._rt is not None and getattr(self, "cuda_event", None):

@@ -4,10 +4,13 @@
 
 Builds the seeded synthetic cache of the workload (optionally with a smaller
 batch), then calls kvc_decode_attn N times on the current CUDA device.  With
---time it flushes L2 (a 512 MiB write) before every call and prints, per call
-median, the whole step (query projection, split-T kernel, combine) and the
-split-T kernel alone, both from CUDA events, with the compressed bytes the step
-reads.  Without --time it only runs the calls (the form used under a profiler).
+--time it flushes L2 (a 512 MiB write) before every call and prints medians
+over the calls, from CUDA events: the whole step (query projection, split-T
+kernel, combine) timed without instrumentation, then, in a second pass with
+the library recording events around the split-T kernel, that kernel and the
+parts of the instrumented step before and after it; with the compressed bytes
+the step reads.  Without --time it only runs the calls (the form used under a
+profiler).
 With --append (low-rank layouts) every step first appends one new token to
 slot T - 1 of every row with kvc_append, as the C5 workload's step does.
 """
@@ -83,22 +86,33 @@ def main(argv=None):
     for _ in range(3):
         step()
     torch.cuda.synchronize()
-    step_us, kern_us = [], []
-    for _ in range(args.steps):
+    step_us, kern_us, pre_us, post_us = [], [], [], []
+    for _ in range(args.steps):         # the step, uninstrumented
+        flush.zero_()
+        e0, e1 = kvc.RawEvent(), kvc.RawEvent()
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        step_us.append(e0.elapsed_ms(e1) * 1e3)
+    for _ in range(args.steps):         # the split-T kernel between the library's events
         flush.zero_()
         ev = (kvc.RawEvent(), kvc.RawEvent())
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0, e1 = kvc.RawEvent(), kvc.RawEvent()
         e0.record()
         step(ev)
         e1.record()
         torch.cuda.synchronize()
-        step_us.append(e0.elapsed_time(e1) * 1e3)
         kern_us.append(ev[0].elapsed_ms(ev[1]) * 1e3)
+        pre_us.append(e0.elapsed_ms(ev[0]) * 1e3)
+        post_us.append(ev[1].elapsed_ms(e1) * 1e3)
     nbytes = lay.step_bytes(c["T"])
     st, kt = statistics.median(step_us), statistics.median(kern_us)
     print(json.dumps({"config": args.config, "batch": c["B"], "context": c["T"],
                       "bytes_per_step": nbytes, "step_us": round(st, 2),
                       "split_kernel_us": round(kt, 2), "step_gbs": round(nbytes / st / 1e3, 1),
+                      "before_split_us": round(statistics.median(pre_us), 2),
+                      "after_split_us": round(statistics.median(post_us), 2),
                       "split_kernel_gbs": round(nbytes / kt / 1e3, 1),
                       "finite": bool(torch.isfinite(out).all().item()),
                       "err_word": int(ws[:4].view(torch.int32).item()),

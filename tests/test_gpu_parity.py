@@ -411,6 +411,37 @@ def test_varrate_k_and_v_ranks_differ(varrate_kernel):
     assert_close(run_decode(c, a, 999), oracle(c, a, 999), what="varrate k/v ranks differ")
 
 
+def test_varrate_bf16_output(varrate_kernel):
+    """bf16 output of the variable-rate layout within the stated tolerance."""
+    c = synth.config("c4", B=2, T=3000)
+    a = synth.varrate_cache(c)
+    assert_close(run_decode(c, a, 3000, out_bf16=1), oracle(c, a, 3000), what="varrate bf16 out")
+
+
+def test_varrate_repeated_calls_reuse_the_workspace():
+    """Calls on a workspace full of stale bytes, and repeated calls on one
+    workspace, must all give the oracle's output (nothing in the workspace may
+    carry state from one call to the next)."""
+    import torch
+
+    from rank_bit_kv_b200 import kvc
+
+    kvc.lib().kvc_select_varrate_kernel(0)
+    c = synth.config("c4", B=3, T=5000)
+    a = synth.varrate_cache(c)
+    ref = oracle(c, a, 5000)
+    lay = kvc.Layout(kvc.desc_from_config(c))
+    cache = kvc.Cache(lay, fill=a)
+    cache.n_tokens = 5000
+    qt = torch.from_numpy(np.ascontiguousarray(a["q"]).view(np.int16)).cuda().view(torch.bfloat16)
+    ws = torch.full((lay.workspace_bytes(5000),), 0xA5, dtype=torch.uint8, device="cuda")
+    for i in range(4):
+        out = torch.empty(qt.shape, device="cuda")
+        kvc.decode(lay, cache, qt, out, ws)
+        torch.cuda.synchronize()
+        assert_close(out.cpu().numpy(), ref, what=f"varrate call {i} on a reused workspace")
+
+
 # ------------------------------------------------------------------ block-shared latent on warp-level MMAs
 
 
