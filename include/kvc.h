@@ -104,7 +104,8 @@ typedef struct {
   int32_t rank_v;
   int32_t latent_bits;    /* 16 or 4                                          */
   int32_t group_size;     /* quantization group                               */
-  int32_t latent_dim;     /* BLOCK_SHARED latent width (512)                  */
+  int32_t latent_dim;     /* BLOCK_SHARED latent width (512; 16..512, a
+                             multiple of 16)                                 */
   int32_t rope;           /* 0 or 1 (LOWRANK)                                 */
   int32_t resid_bits;     /* 0 or 2 (LOWRANK, head_dim 128)                   */
   int32_t page_size;      /* 0 (contiguous) or 16 (LOWRANK)                   */

@@ -10,6 +10,7 @@
 #include <math.h>
 
 #include "kvc_device.cuh"
+#include "tc_util.cuh"
 
 namespace kvc {
 namespace {
@@ -359,6 +360,193 @@ __global__ void __launch_bounds__(kThreads) combine_block_kernel(Params p) {
   }
 }
 
+// Block-shared latent, head dim 128, all of a block's partials in shared
+// memory at once (the usual case: few splits per row): one block per (layer,
+// batch row, KV head).  The first rows of the layer's W_v slice are copied
+// before the block waits for the split kernel (they do not depend on it); then
+// the G query heads' partials (every split, accumulators and (m, l)) arrive by
+// cp.async in one round (16-byte pieces: the G rows of a split are one span),
+// are weighted and merged from shared memory,
+// and the rest of the W_v slice lands where the partials were.  The
+// up-projection runs on warp-level MMAs: M = 16 output dims (warp w: dims
+// 16 w ..), N = 8 heads, K = 16 latent rows; the fp32 accumulators enter as
+// the sum of two f16 parts (hi = f16(x), lo = f16(x - hi), after scaling the
+// head by a power of two that puts its largest value below 2^14), so the two
+// MMAs per k-step carry ~22 significant bits of every accumulator; W_v is
+// fp16, products are exact and the sums fp32.
+constexpr int kCbThreads = 256;
+constexpr int kCbRow = 272;             // bytes per staged W_v row (conflict-free ldmatrix)
+
+struct BlockCombinePlan {
+  int rows_a;                           // W_v rows staged before the wait
+  size_t off_acc, off_wts, off_wa, bytes;
+};
+
+__host__ __device__ inline BlockCombinePlan block_combine_plan(int G, int S, int D, int vdim) {
+  BlockCombinePlan pl;
+  const size_t pbytes = (size_t)G * S * (vdim + 2) * sizeof(float);
+  pl.off_acc = (pbytes + 15) & ~(size_t)15;
+  pl.off_wts = pl.off_acc + (size_t)G * D * sizeof(float);
+  pl.off_wa = (pl.off_wts + ((size_t)G * S + 24) * sizeof(float) + 15) & ~(size_t)15;
+  const size_t budget = 227 * 1024;
+  long long ra = pl.off_wa < budget ? (long long)((budget - pl.off_wa) / kCbRow) : 0;
+  ra &= ~15ll;
+  if (ra > D) ra = D;
+  pl.rows_a = (int)ra;
+  pl.bytes = pl.off_wa + (size_t)pl.rows_a * kCbRow;
+  return pl;
+}
+
+__global__ void __launch_bounds__(kCbThreads) combine_block_staged_kernel(Params p) {
+  extern __shared__ __align__(16) uint8_t cbs[];
+  const int D = p.D, G = p.G, nS = p.S, pst = p.vdim + 2;
+  const BlockCombinePlan pl = block_combine_plan(G, nS, D, p.vdim);
+  float* const P = reinterpret_cast<float*>(cbs);                  // [nS][G][pst]
+  float* const acc = reinterpret_cast<float*>(cbs + pl.off_acc);  // [G][D]
+  float* const wts = reinterpret_cast<float*>(cbs + pl.off_wts);  // [G][nS], then 1/l [G]
+  float* const linv = wts + G * nS;
+  const int blk = blockIdx.x;            // (l * B + b) * Hkv + kvh
+  const int kvh = blk % p.Hkv, lb = blk / p.Hkv;
+  const int l = lb / p.B;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t rows = (size_t)p.L * p.B * p.Hq;
+  const __half* w = p.bv + (int64_t)l * D * p.Hkv * 128 + kvh * 128;
+  auto copy_w = [&](int r0, int r1, uint8_t* dst) {
+    for (int e = tid; e < (r1 - r0) * 16; e += kCbThreads) {
+      const int r = e >> 4, part = e & 15;
+      const uint32_t sa = (uint32_t)__cvta_generic_to_shared(dst + r * kCbRow + part * 16);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa),
+                   "l"(w + (int64_t)(r0 + r) * p.Hkv * 128 + part * 8) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  copy_w(0, pl.rows_a, cbs + pl.off_wa);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  {
+    // the G heads' partials of split sp are G consecutive rows of (vdim + 2)
+    // floats: with G even the span starts on a 16-byte boundary and is a
+    // whole number of 16-byte pieces, else it is copied in 8-byte pieces
+    const float* const src0 = p.part + ((size_t)lb * p.Hq + kvh * G) * pst;
+    const uint32_t dst0 = (uint32_t)__cvta_generic_to_shared(P);
+    const int span = G * pst;            // floats
+    if ((G & 1) == 0) {
+      for (int sp = 0; sp < nS; ++sp) {
+        const float* src = src0 + (size_t)sp * rows * pst;
+        const uint32_t dst = dst0 + (uint32_t)sp * span * 4;
+        for (int k = tid; k < span / 4; k += kCbThreads)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * k),
+                       "l"(src + 4 * k) : "memory");
+      }
+    } else {
+      for (int sp = 0; sp < nS; ++sp) {
+        const float* src = src0 + (size_t)sp * rows * pst;
+        const uint32_t dst = dst0 + (uint32_t)sp * span * 4;
+        for (int k = tid; k < span / 2; k += kCbThreads)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst + 8 * k),
+                       "l"(src + 2 * k) : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+  }
+  __syncthreads();
+  // split weights and softmax sums (warp g: head g)
+  for (int g = warp; g < G; g += kCbThreads / 32) {
+    const float* pg = P + (size_t)g * pst;
+    const size_t sstr = (size_t)G * pst;  // between the splits of one head
+    float mx = -INFINITY;
+    for (int sp = lane; sp < nS; sp += 32) mx = fmaxf(mx, pg[sp * sstr + D]);
+    mx = warp_max(mx);
+    float lt = 0.f;
+    for (int sp = lane; sp < nS; sp += 32) {
+      const float m = pg[sp * sstr + D];
+      const float wt = (mx == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - mx);
+      wts[g * nS + sp] = wt;
+      lt = fmaf(wt, pg[sp * sstr + D + 1], lt);
+    }
+    lt = warp_sum(lt);
+    if (lane == 0) linv[g] = lt > 0.f ? 1.f / lt : 0.f;
+  }
+  __syncthreads();
+  for (int g = 0; g < G; ++g) {
+    const float* wg = wts + g * nS;
+    for (int c = tid; c < D; c += kCbThreads) {
+      const float* pg = P + (size_t)g * pst + c;
+      float a = 0.f;
+#pragma unroll 6
+      for (int sp = 0; sp < nS; ++sp) a = fmaf(wg[sp], pg[(size_t)sp * G * pst], a);
+      acc[g * D + c] = a;
+    }
+  }
+  __syncthreads();
+  // per-head scale of the merged accumulators (warp g: head g)
+  float* const down = linv + 8;         // 2^-e_g
+  float* const up = linv + 16;          // 2^e_g / l_g
+  for (int g = warp; g < 8; g += kCbThreads / 32) {
+    float mx = 0.f;
+    if (g < G)
+      for (int c = lane; c < D; c += 32) mx = fmaxf(mx, fabsf(acc[g * D + c]));
+    mx = warp_max(mx);
+    int ex = 0;
+    if (mx > 0.f && mx <= 3.0e38f) {
+      frexpf(mx, &ex);
+      ex = ex > 14 ? ex - 14 : (ex < -100 ? -100 : ex - 14);
+    }
+    if (lane == 0) {
+      down[g] = ldexpf(1.f, -ex);
+      up[g] = g < G ? ldexpf(1.f, ex) * linv[g] : 0.f;
+    }
+  }
+  __syncthreads();                      // the partials are dead: W_v's other rows land there
+  uint8_t* const wb = cbs;
+  if (pl.rows_a < D) copy_w(pl.rows_a, D, wb);
+  // up-projection: warp w forms output dims 16 w .. 16 w + 15 of the 8 heads
+  const int n = lane >> 2, kq = 2 * (lane & 3);
+  const bool live = n < G;
+  const float* const an = acc + (live ? n : 0) * D + kq;
+  const float sn = down[n];
+  const int lj = lane >> 3, lr = lane & 7;
+  const int i_off = 16 * warp + 8 * (lj & 1);
+  float c4[4] = {0.f, 0.f, 0.f, 0.f};
+  auto ksteps = [&](const uint8_t* wr, int k0, int k1, int r_base) {
+    for (int ks = k0; ks < k1; ++ks) {
+      const int row = 16 * ks + lr + 8 * (lj >> 1);
+      uint32_t a[4];
+      tc::ldmatrix_x4_trans(a, wr + (row - r_base) * kCbRow + 2 * i_off);
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      if (live) {
+        const float2 v0 = *reinterpret_cast<const float2*>(an + 16 * ks);
+        const float2 v8 = *reinterpret_cast<const float2*>(an + 16 * ks + 8);
+        x[0] = v0.x * sn; x[1] = v0.y * sn; x[2] = v8.x * sn; x[3] = v8.y * sn;
+      }
+      const __half2 h0 = __floats2half2_rn(x[0], x[1]), h8 = __floats2half2_rn(x[2], x[3]);
+      const float2 f0 = __half22float2(h0), f8 = __half22float2(h8);
+      const __half2 l0 = __floats2half2_rn(x[0] - f0.x, x[1] - f0.y);
+      const __half2 l8 = __floats2half2_rn(x[2] - f8.x, x[3] - f8.y);
+      tc::mma16816(c4, a, *reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h8));
+      tc::mma16816(c4, a, *reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l8));
+    }
+  };
+  asm volatile("cp.async.wait_group 1;" ::: "memory");   // the first rows (the older group)
+  __syncthreads();
+  ksteps(cbs + pl.off_wa, 0, pl.rows_a / 16, 0);
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  if (pl.rows_a < D) ksteps(wb, pl.rows_a / 16, D / 16, pl.rows_a);
+  // C fragment: dims 16 w + lane / 4 (+ 8), heads 2 (lane % 4) (+ 1)
+  const int i0 = 16 * warp + (lane >> 2);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int g = kq + (e & 1), i = i0 + 8 * (e >> 1);
+    if (g < G) {
+      const int64_t orow = (int64_t)lb * p.Hq + kvh * G + g;
+      const float t = c4[e] * up[g];
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[orow * 128 + i] = __float2bfloat16_rn(t);
+      else reinterpret_cast<float*>(p.out)[orow * 128 + i] = t;
+    }
+  }
+}
+
 cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   if (p.S > kMaxS) return cudaErrorInvalidValue;
   const int rows = p.L * p.B * p.Hq;
@@ -383,6 +571,19 @@ cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (p.kind == KVC_BLOCK_SHARED && p.G <= kBGroup && p.seg_W == 0 && p.d == 128 &&
+      p.vdim == p.D && p.D % 8 == 0) {
+    const BlockCombinePlan pl = block_combine_plan(p.G, p.S, p.D, p.vdim);
+    if (pl.rows_a >= 16 && (size_t)(p.D - pl.rows_a) * kCbRow <= pl.off_acc) {
+      e = cudaFuncSetAttribute(combine_block_staged_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.bytes);
+      if (e != cudaSuccess) return e;
+      cfg.gridDim = dim3(p.L * p.B * p.Hkv);
+      cfg.blockDim = dim3(kCbThreads);
+      cfg.dynamicSmemBytes = pl.bytes;
+      return cudaLaunchKernelEx(&cfg, combine_block_staged_kernel, p);
+    }
+  }
   if (p.kind == KVC_BLOCK_SHARED && p.G <= kBGroup && p.seg_W == 0 && p.d % 8 == 0 &&
       p.d <= kThreads) {
     const size_t bb = ((size_t)p.G * p.D + (size_t)p.G * p.S + 4) * sizeof(float) +

@@ -3,6 +3,7 @@
 // residual (q . Q^T y = (Q q) . y), and the absorbed block-shared query
 // q~_l = W_k^l[:, head slice] q_l.
 #include "kvc_device.cuh"
+#include "tc_util.cuh"
 
 namespace kvc {
 namespace {
@@ -183,11 +184,120 @@ __global__ void __launch_bounds__(256) qproj_block_kernel(Params p) {
   }
 }
 
+// The same projection on warp-level MMAs, with the whole W_k slice in flight
+// at once (D <= 768): M = 16 rows of the slice, N = 8 query heads (G of them
+// real), K = 16 head dims.  The group's queries are scaled by a power of two,
+// 2^-e, so that the largest lies below 2^14, and rounded to f16: exact for
+// bf16 inputs (8 significant bits) down to the f16 subnormals, whose spacing
+// is 2^-38 of the largest; W_k is fp16, the products are exact and the sums
+// fp32, and the results are scaled back by 2^e.  The rows of the first and of
+// the second half of the slice are two copy groups, so the MMAs of the first
+// half run while the second lands.
+constexpr int kQsMaxRows = 768;
+constexpr int kQhRow = 136;              // f16 per staged query row (272 bytes)
+
+__global__ void __launch_bounds__(256) qproj_block_mma_kernel(Params p) {
+  extern __shared__ __align__(16) uint8_t qsb[];
+  __half* const qh = reinterpret_cast<__half*>(qsb);              // [8][kQhRow]
+  float* const red = reinterpret_cast<float*>(qsb + 8 * kQhRow * 2);   // [8] warp maxima
+  uint8_t* const wsm = qsb + 8 * kQhRow * 2 + 64;                 // [D][kQbRow]
+  const int unit = blockIdx.x;             // (l * B + b) * Hkv + kvh
+  const int kvh = unit % p.Hkv;
+  const int l = unit / (p.B * p.Hkv);
+  const int row0 = (unit / p.Hkv) * p.Hq + kvh * p.G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, G = p.G, D = p.D;
+  const __half* w = p.bk + (int64_t)l * D * p.Hkv * 128 + kvh * 128;
+  const int mid = min(D, ((D / 16 + 1) / 2) * 16);
+  auto stage = [&](int r0, int r1) {
+    for (int e = tid; e < (r1 - r0) * 16; e += 256) {
+      const int r = r0 + (e >> 4), part = e & 15;
+      const uint32_t dst = (uint32_t)__cvta_generic_to_shared(wsm + r * kQbRow + part * 16);
+      const __half* src = w + (int64_t)r * p.Hkv * 128 + part * 8;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  stage(0, mid);
+  stage(mid, D);
+  // the group's queries (4 per thread) and their largest magnitude
+  float qv[4], mx = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int e = tid + 256 * k, g = e >> 7;
+    qv[k] = g < G ? bf2f(p.q[(int64_t)(row0 + g) * 128 + (e & 127)]) : 0.f;
+    mx = fmaxf(mx, fabsf(qv[k]));
+  }
+  mx = warp_max(mx);
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx = fmaxf(mx, red[k]);
+  int ex = 0;
+  if (mx > 0.f && mx <= 3.0e38f) {
+    frexpf(mx, &ex);                       // mx < 2^ex
+    ex = ex > 14 ? ex - 14 : 0;
+  }
+  const float down = ldexpf(1.f, -ex), up = ldexpf(1.f, ex);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int e = tid + 256 * k;
+    qh[(e >> 7) * kQhRow + (e & 127)] = __float2half_rn(qv[k] * down);
+  }
+  __syncthreads();
+  // B fragments of the 8 k-steps: column n = lane / 4, rows 2 (lane % 4) (+1, +8, +9)
+  uint32_t bf[8][2];
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const __half* qr = qh + (lane >> 2) * kQhRow + 16 * ks + 2 * (lane & 3);
+    bf[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
+    bf[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
+  }
+  const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lk = 8 * (lane >> 4);
+  const int n0 = 2 * (lane & 3);
+  auto tiles = [&](int t0, int t1) {
+    for (int mt = t0 + warp; mt < t1; mt += 8) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint8_t* ar = wsm + (16 * mt + lrow) * kQbRow + lk * 2;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t a[4];
+        tc::ldmatrix_x4(a, ar + 32 * ks);
+        tc::mma16816(c, a, bf[ks][0], bf[ks][1]);
+      }
+      const int ra = 16 * mt + (lane >> 2);
+      if (n0 < G) {
+        p.qt[(int64_t)(row0 + n0) * p.qdim + ra] = c[0] * up;
+        p.qt[(int64_t)(row0 + n0) * p.qdim + ra + 8] = c[2] * up;
+      }
+      if (n0 + 1 < G) {
+        p.qt[(int64_t)(row0 + n0 + 1) * p.qdim + ra] = c[1] * up;
+        p.qt[(int64_t)(row0 + n0 + 1) * p.qdim + ra + 8] = c[3] * up;
+      }
+    }
+  };
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+  __syncthreads();
+  tiles(0, mid / 16);
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  tiles(mid / 16, D / 16);
+}
+
 }  // namespace
 
 cudaError_t launch_qproj(const Params& p, cudaStream_t s) {
   if ((p.kind == KVC_LOWRANK || p.kind == KVC_VARRATE) && p.d == 128 && p.G <= 8) {
     qproj_group_kernel<<<p.L * p.B * p.Hkv, kThreads, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  if (p.kind == KVC_BLOCK_SHARED && p.d == 128 && p.G <= 8 && p.D <= kQsMaxRows &&
+      p.D % 16 == 0) {
+    const int bytes = 8 * kQhRow * 2 + 64 + p.D * kQbRow;
+    cudaError_t e = cudaFuncSetAttribute(qproj_block_mma_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    qproj_block_mma_kernel<<<p.L * p.B * p.Hkv, 256, bytes, s>>>(p);
     return cudaGetLastError();
   }
   if (p.kind == KVC_BLOCK_SHARED && p.d == 128 && p.G <= 8) {

@@ -243,8 +243,10 @@ kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out) {
       break;
     }
     case KVC_BLOCK_SHARED: {
-      if (d.latent_dim < 16 || d.latent_dim > 1024 || d.latent_dim % 16) {
-        st = KVC_EINVAL, why = "latent_dim must be a multiple of 16 in 16..1024";
+      // the decode kernels hold the 32 queries' accumulators of a CTA in
+      // registers (at most 64 per thread): latent widths up to 512
+      if (d.latent_dim < 16 || d.latent_dim > 512 || d.latent_dim % 16) {
+        st = KVC_EINVAL, why = "latent_dim must be a multiple of 16 in 16..512";
         break;
       }
       if (d.group_size < 2 || d.latent_dim % d.group_size || d.group_size % 2) {

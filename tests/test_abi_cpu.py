@@ -97,6 +97,18 @@ def test_invalid_layouts_rejected(lib, bad, status):
     assert lib.kvc_last_error()
 
 
+@pytest.mark.parametrize("D", [640, 768, 1024])
+def test_block_shared_latent_wider_than_512_rejected(lib, D):
+    """The decode kernels keep at most 64 accumulators per thread for the 32
+    queries of a CTA, i.e. latent widths up to 512; wider ones are refused at
+    layout creation rather than decoded wrongly."""
+    with pytest.raises(kvc.KvcError) as ei:
+        kvc.Layout(kvc.make_desc("block_shared", batch=1, n_q_heads=32, n_kv_heads=8,
+                                 head_dim=128, max_tokens=16, n_layers=4, latent_dim=D,
+                                 group_size=64))
+    assert kvc.STATUS[ei.value.status] == "KVC_EINVAL" and b"latent_dim" in lib.kvc_last_error()
+
+
 def test_kind_flag_conflicts(lib):
     with pytest.raises(kvc.KvcError):
         kvc.Layout(kvc.make_desc("varrate", batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128,

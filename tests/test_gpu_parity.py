@@ -120,6 +120,15 @@ def test_c4_shape_small_varrate(T, varrate_kernel):
     assert_close(run_decode(c, a, T), oracle(c, a, T), what=f"c4 T={T}")
 
 
+@pytest.mark.parametrize("D,B,n", [(128, 2, 300), (256, 3, 1000), (384, 4, 640)])
+def test_block_shared_latent_widths(D, B, n):
+    """Latent widths other than 512: the query projection's MMA tiles and the
+    staged combine's split of the W_v rows change with D."""
+    c = synth.config("c3", B=B, T=n, D=D)
+    a = synth.block_shared_cache(c)
+    assert_close(run_decode(c, a, n), oracle(c, a, n), what=f"block-shared D={D} B={B} n={n}")
+
+
 def test_c3_shape_small_block_shared():
     c = synth.config("c3", B=2, T=300)
     a = synth.block_shared_cache(c)
