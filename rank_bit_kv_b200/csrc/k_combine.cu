@@ -361,12 +361,13 @@ __global__ void __launch_bounds__(kThreads) combine_block_kernel(Params p) {
 }
 
 // Block-shared latent, head dim 128, all of a block's partials in shared
-// memory at once (the usual case: few splits per row): one block per (layer,
-// batch row, KV head).  The first rows of the layer's W_v slice are copied
+// memory at once (the usual case: few splits per row, an even group): one
+// block per (layer, batch row, KV head).  The first rows of the layer's W_v
+// slice are copied
 // before the block waits for the split kernel (they do not depend on it); then
-// the G query heads' partials (every split, accumulators and (m, l)) arrive by
-// cp.async in one round (16-byte pieces: the G rows of a split are one span),
-// are weighted and merged from shared memory,
+// the G query heads' partials (every split, accumulators and (m, l); the G
+// rows of a split are one span) arrive by 1-D bulk copies counted on an
+// mbarrier (bounded wait), are weighted and merged from shared memory,
 // and the rest of the W_v slice lands where the partials were.  The
 // up-projection runs on warp-level MMAs: M = 16 output dims (warp w: dims
 // 16 w ..), N = 8 heads, K = 16 latent rows; the fp32 accumulators enter as
@@ -388,7 +389,7 @@ __host__ __device__ inline BlockCombinePlan block_combine_plan(int G, int S, int
   pl.off_acc = (pbytes + 15) & ~(size_t)15;
   pl.off_wts = pl.off_acc + (size_t)G * D * sizeof(float);
   pl.off_wa = (pl.off_wts + ((size_t)G * S + 24) * sizeof(float) + 15) & ~(size_t)15;
-  const size_t budget = 227 * 1024;
+  const size_t budget = 227 * 1024 - 256;   // the kernel's static barriers and flag
   long long ra = pl.off_wa < budget ? (long long)((budget - pl.off_wa) / kCbRow) : 0;
   ra &= ~15ll;
   if (ra > D) ra = D;
@@ -399,6 +400,8 @@ __host__ __device__ inline BlockCombinePlan block_combine_plan(int G, int S, int
 
 __global__ void __launch_bounds__(kCbThreads) combine_block_staged_kernel(Params p) {
   extern __shared__ __align__(16) uint8_t cbs[];
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
   const int D = p.D, G = p.G, nS = p.S, pst = p.vdim + 2;
   const BlockCombinePlan pl = block_combine_plan(G, nS, D, p.vdim);
   float* const P = reinterpret_cast<float*>(cbs);                  // [nS][G][pst]
@@ -411,44 +414,34 @@ __global__ void __launch_bounds__(kCbThreads) combine_block_staged_kernel(Params
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t rows = (size_t)p.L * p.B * p.Hq;
   const __half* w = p.bv + (int64_t)l * D * p.Hkv * 128 + kvh * 128;
-  auto copy_w = [&](int r0, int r1, uint8_t* dst) {
-    for (int e = tid; e < (r1 - r0) * 16; e += kCbThreads) {
-      const int r = e >> 4, part = e & 15;
-      const uint32_t sa = (uint32_t)__cvta_generic_to_shared(dst + r * kCbRow + part * 16);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa),
-                   "l"(w + (int64_t)(r0 + r) * p.Hkv * 128 + part * 8) : "memory");
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
+  const int span = G * pst;              // floats: the G heads' partials of one split
+  if (tid == 0) {
+    tc::mbar_init(&bars[0], 1);
+    tc::mbar_init(&bars[1], 1);
+    tc::fence_mbar_init();
+    abort_flag = 0;
+    // the first W_v rows and every split's span on barrier 0, the other rows on 1
+    tc::mbar_arrive_expect_tx(&bars[0], (uint32_t)(pl.rows_a * 256 + nS * span * 4));
+    tc::mbar_arrive_expect_tx(&bars[1], (uint32_t)((D - pl.rows_a) * 256));
+  }
+  __syncthreads();
+  // 1-D bulk copies: W_v rows (256 bytes) into rows of kCbRow bytes
+  auto copy_w = [&](int r0, int r1, uint8_t* dst, uint64_t* bar) {
+    for (int r = r0 + tid; r < r1; r += kCbThreads)
+      tc::bulk_g2s(dst + (r - r0) * kCbRow, w + (int64_t)r * p.Hkv * 128, 256, bar);
   };
-  copy_w(0, pl.rows_a, cbs + pl.off_wa);
+  copy_w(0, pl.rows_a, cbs + pl.off_wa, &bars[0]);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   {
     // the G heads' partials of split sp are G consecutive rows of (vdim + 2)
-    // floats: with G even the span starts on a 16-byte boundary and is a
-    // whole number of 16-byte pieces, else it is copied in 8-byte pieces
+    // floats; with G even the span starts on a 16-byte boundary and is a whole
+    // number of 16-byte pieces (the launch requires G even)
     const float* const src0 = p.part + ((size_t)lb * p.Hq + kvh * G) * pst;
-    const uint32_t dst0 = (uint32_t)__cvta_generic_to_shared(P);
-    const int span = G * pst;            // floats
-    if ((G & 1) == 0) {
-      for (int sp = 0; sp < nS; ++sp) {
-        const float* src = src0 + (size_t)sp * rows * pst;
-        const uint32_t dst = dst0 + (uint32_t)sp * span * 4;
-        for (int k = tid; k < span / 4; k += kCbThreads)
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * k),
-                       "l"(src + 4 * k) : "memory");
-      }
-    } else {
-      for (int sp = 0; sp < nS; ++sp) {
-        const float* src = src0 + (size_t)sp * rows * pst;
-        const uint32_t dst = dst0 + (uint32_t)sp * span * 4;
-        for (int k = tid; k < span / 2; k += kCbThreads)
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst + 8 * k),
-                       "l"(src + 2 * k) : "memory");
-      }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    for (int sp = tid; sp < nS; sp += kCbThreads)
+      tc::bulk_g2s(P + (size_t)sp * span, src0 + (size_t)sp * rows * pst, (uint32_t)span * 4,
+                   &bars[0]);
   }
+  if (!tc::mbar_wait(&bars[0], 0, &abort_flag, p.err)) return;
   __syncthreads();
   // split weights and softmax sums (warp g: head g)
   for (int g = warp; g < G; g += kCbThreads / 32) {
@@ -468,15 +461,28 @@ __global__ void __launch_bounds__(kCbThreads) combine_block_staged_kernel(Params
     if (lane == 0) linv[g] = lt > 0.f ? 1.f / lt : 0.f;
   }
   __syncthreads();
-  for (int g = 0; g < G; ++g) {
-    const float* wg = wts + g * nS;
-    for (int c = tid; c < D; c += kCbThreads) {
-      const float* pg = P + (size_t)g * pst + c;
-      float a = 0.f;
-#pragma unroll 6
-      for (int sp = 0; sp < nS; ++sp) a = fmaf(wg[sp], pg[(size_t)sp * G * pst], a);
-      acc[g * D + c] = a;
+  // merged accumulators: thread t forms dims 2 t, 2 t + 1 (+ 512 k) of every
+  // head, one independent chain per (head, dim)
+  for (int c2 = 2 * tid; c2 < D; c2 += 2 * kCbThreads) {
+    float2 a[kBGroup];
+#pragma unroll
+    for (int g = 0; g < kBGroup; ++g) a[g] = make_float2(0.f, 0.f);
+#pragma unroll 2
+    for (int sp = 0; sp < nS; ++sp) {
+      const float* ps = P + (size_t)sp * G * pst + c2;
+#pragma unroll
+      for (int g = 0; g < kBGroup; ++g) {
+        if (g < G) {
+          const float wgt = wts[g * nS + sp];
+          const float2 v = *reinterpret_cast<const float2*>(ps + (size_t)g * pst);
+          a[g].x = fmaf(wgt, v.x, a[g].x);
+          a[g].y = fmaf(wgt, v.y, a[g].y);
+        }
+      }
     }
+#pragma unroll
+    for (int g = 0; g < kBGroup; ++g)
+      if (g < G) *reinterpret_cast<float2*>(acc + g * D + c2) = a[g];
   }
   __syncthreads();
   // per-head scale of the merged accumulators (warp g: head g)
@@ -499,7 +505,7 @@ __global__ void __launch_bounds__(kCbThreads) combine_block_staged_kernel(Params
   }
   __syncthreads();                      // the partials are dead: W_v's other rows land there
   uint8_t* const wb = cbs;
-  if (pl.rows_a < D) copy_w(pl.rows_a, D, wb);
+  copy_w(pl.rows_a, D, wb, &bars[1]);
   // up-projection: warp w forms output dims 16 w .. 16 w + 15 of the 8 heads
   const int n = lane >> 2, kq = 2 * (lane & 3);
   const bool live = n < G;
@@ -527,11 +533,8 @@ __global__ void __launch_bounds__(kCbThreads) combine_block_staged_kernel(Params
       tc::mma16816(c4, a, *reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l8));
     }
   };
-  asm volatile("cp.async.wait_group 1;" ::: "memory");   // the first rows (the older group)
-  __syncthreads();
   ksteps(cbs + pl.off_wa, 0, pl.rows_a / 16, 0);
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
+  if (!tc::mbar_wait(&bars[1], 0, &abort_flag, p.err)) return;
   if (pl.rows_a < D) ksteps(wb, pl.rows_a / 16, D / 16, pl.rows_a);
   // C fragment: dims 16 w + lane / 4 (+ 8), heads 2 (lane % 4) (+ 1)
   const int i0 = 16 * warp + (lane >> 2);
@@ -574,7 +577,7 @@ cudaError_t launch_combine(const Params& p, cudaStream_t s) {
   if (p.kind == KVC_BLOCK_SHARED && p.G <= kBGroup && p.seg_W == 0 && p.d == 128 &&
       p.vdim == p.D && p.D % 8 == 0) {
     const BlockCombinePlan pl = block_combine_plan(p.G, p.S, p.D, p.vdim);
-    if (pl.rows_a >= 16 && (size_t)(p.D - pl.rows_a) * kCbRow <= pl.off_acc) {
+    if (p.G % 2 == 0 && pl.rows_a >= 16 && (size_t)(p.D - pl.rows_a) * kCbRow <= pl.off_acc) {
       e = cudaFuncSetAttribute(combine_block_staged_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.bytes);
       if (e != cudaSuccess) return e;

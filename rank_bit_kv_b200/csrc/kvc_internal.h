@@ -227,7 +227,8 @@ __host__ __device__ inline bool needs_qproj(const Params& p) {
 // Whether the chosen split kernel has bounded waits that can set the
 // workspace error word (the call zeroes the word first only then).
 __host__ __device__ inline bool path_sets_error_word(const Params& p) {
-  return p.path == 1 || p.path == 7 || p.path == 8;
+  // tcgen05 split kernels, and the block-shared combine (bounded mbarrier waits)
+  return p.path == 1 || p.path == 7 || p.path == 8 || p.kind == KVC_BLOCK_SHARED;
 }
 
 }  // namespace kvc
