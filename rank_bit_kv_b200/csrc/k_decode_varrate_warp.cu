@@ -7,7 +7,7 @@
 // shuffles) and its own latent-space accumulator acc[64] in registers; the
 // projected queries q~ = Bk q are formed by the CTA itself (one thread per
 // (KV head, rank) row of Bk, all four query heads of the group) into shared
-// memory, where each lane reads its own row:
+// memory (on warp-level MMAs), where each lane reads its own row:
 //   s_t = sum_{i < r_k(t)} q~_i (c_i s_g + z_g),
 //   acc_i += p_t (c_i s_g + z_g) for i < r_v(t).
 // Keeping q~ out of the registers lets 16 warps share an SM (4 per scheduler)
@@ -49,7 +49,8 @@ constexpr int kVWarpBytes = 4 * kVBuf;              // K and V, two buffers each
 constexpr int kVStage = kVWarps * kVWarpBytes;
 constexpr int kVQRow = kVRmax + 4;                  // floats per q~ row (16-byte loads conflict-free)
 constexpr int kVOffQ = kVStage;                     // q~ [32][kVQRow] (softmax scale, log2 e folded)
-constexpr int kVOffX = kVOffQ + 32 * kVQRow * 4;    // the group's queries [32][128] fp32
+constexpr int kVOffX = kVOffQ + 32 * kVQRow * 4;    // the queries [32][kVQhRow] f16, then 16 maxima
+constexpr int kVQhRow = 136;                        // f16 per staged query row (272 bytes)
 constexpr int kVSmem = kVOffX + 32 * 128 * 4;
 constexpr int kVPst = kVRmax + 2;                   // merge slot: acc[64], m, l
 
@@ -57,6 +58,7 @@ static_assert(kVWarps * 32 * kVPst * 4 <= kVStage, "merge area fits in the stagi
 static_assert(kVThreads == kVHkv * kVRmax, "one thread per (KV head, rank) row of Bk");
 static_assert(kVHkv * kVRmax * 256 <= kVStage, "Bk's copy fits in the staging area");
 static_assert(kVBuf <= 4096, "record offsets in a staged chunk fit in 12 bits");
+static_assert(32 * kVQhRow * 2 + kVWarps * 4 <= 32 * 128 * 4, "f16 queries and maxima fit");
 
 __host__ __device__ constexpr int head_bytes(int r) { return r / 2 + 4 * ((r + 31) / 32); }
 
@@ -303,10 +305,14 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   if (t0 + kVChunk < t_b) raw1 = meta_load(t0 + kVChunk);
 
   // ---- q~ = Bk q for the row's 32 query heads (softmax scale and log2 e
-  // folded in).  Bk (8 heads x 64 rows x 128, fp16) is first copied into the
-  // staging area with coalesced 16-byte copies, row r's 16-byte piece c at
-  // r * 256 + (c ^ (r & 15)) * 16 (conflict-free row reads); then thread
-  // (kvh, j) dots row j of head kvh's Bk with its 4 queries
+  // folded in), on warp-level MMAs.  Bk (8 heads x 64 rows x 128, fp16) is first
+  // copied into the staging area with coalesced 16-byte copies, row r's 16-byte
+  // piece c at r * 256 + (c ^ (r & 15)) * 16 (conflict-free ldmatrix rows).  The
+  // queries are scaled by a power of two, 2^-e, so that the largest lies below
+  // 2^14, and rounded to f16: exact for bf16 values down to the f16
+  // subnormals, whose spacing is 2^-38 of the largest.  Warp w forms rows
+  // 32 (w % 2) .. + 31 of head w / 2: M = 16 rows, N = the head's 4 queries (of
+  // 8), K = 16 dims; products exact, sums fp32, scaled back by 2^e.
   float* const qsm = reinterpret_cast<float*>(vsm + kVOffQ);
   {
     const uint32_t bks = smem_u32(vsm);
@@ -316,46 +322,72 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
       cp16(bks + r * 256 + ((pc ^ (r & 15)) << 4), p.bk + (size_t)idx * 8);
     }
     cp_commit();
-    float* const xs = reinterpret_cast<float*>(vsm + kVOffX);
+    __half* const qh = reinterpret_cast<__half*>(vsm + kVOffX);             // [32][kVQhRow]
+    float* const red = reinterpret_cast<float*>(vsm + kVOffX + 32 * kVQhRow * 2);
+    // the row's 32 x 128 bf16 queries, 8 per thread (one 16-byte load)
+    const uint4 xq = __ldg(reinterpret_cast<const uint4*>(p.q + (size_t)b * p.Hq * 128) +
+                           threadIdx.x);
+    const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+    float v[8], mx = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = __uint_as_float(xw[k] << 16);
+      v[2 * k + 1] = __uint_as_float(xw[k] & 0xFFFF0000u);
+      mx = fmaxf(mx, fmaxf(fabsf(v[2 * k]), fabsf(v[2 * k + 1])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    mx = 0.f;
+#pragma unroll
+    for (int k = 0; k < kVWarps; ++k) mx = fmaxf(mx, red[k]);
+    int ex = 0;
+    if (mx > 0.f && mx <= 3.0e38f) {
+      frexpf(mx, &ex);                  // mx < 2^ex
+      ex = ex > 14 ? ex - 14 : 0;
+    }
+    const float down = ldexpf(1.f, -ex), up = ldexpf(1.f, ex) * p.scale_log2;
     {
-      // the row's 32 x 128 bf16 queries, 8 per thread (one 16-byte load)
-      const uint4 xq = __ldg(reinterpret_cast<const uint4*>(p.q + (size_t)b * p.Hq * 128) +
-                             threadIdx.x);
-      const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
-      float4* xd = reinterpret_cast<float4*>(xs + 8 * threadIdx.x);
-      float v[8];
+      uint32_t hw[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        v[2 * k] = __uint_as_float(xw[k] << 16);
-        v[2 * k + 1] = __uint_as_float(xw[k] & 0xFFFF0000u);
+        const __half2 h2 = __floats2half2_rn(v[2 * k] * down, v[2 * k + 1] * down);
+        hw[k] = *reinterpret_cast<const uint32_t*>(&h2);
       }
-      xd[0] = make_float4(v[0], v[1], v[2], v[3]);
-      xd[1] = make_float4(v[4], v[5], v[6], v[7]);
+      *reinterpret_cast<uint4*>(qh + (threadIdx.x >> 4) * kVQhRow + 8 * (threadIdx.x & 15)) =
+          make_uint4(hw[0], hw[1], hw[2], hw[3]);
     }
     cp_wait<0>();
     __syncthreads();
-    const int kvh = threadIdx.x / kVRmax, j = threadIdx.x % kVRmax, r = threadIdx.x;
-    const uint8_t* brow = vsm + r * 256;
-    uint64_t a2[kVG] = {0ull, 0ull, 0ull, 0ull};
-    const float* xk = xs + kvh * kVG * 128;
-#pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
-      const uint4 w = *reinterpret_cast<const uint4*>(brow + ((c ^ (r & 15)) << 4));
-      const float2 f0 = h2f2(w.x), f1 = h2f2(w.y), f2 = h2f2(w.z), f3 = h2f2(w.w);
-      const uint64_t b0 = pkf(f0.x, f0.y), b1 = pkf(f1.x, f1.y);
-      const uint64_t b2 = pkf(f2.x, f2.y), b3 = pkf(f3.x, f3.y);
+    const int kvh = warp >> 1, n = lane >> 2, kq = 2 * (lane & 3);
+    uint32_t bf[8][2];
 #pragma unroll
-      for (int g = 0; g < kVG; ++g) {
-        const ulonglong2 xa = *reinterpret_cast<const ulonglong2*>(xk + g * 128 + 8 * c);
-        const ulonglong2 xb = *reinterpret_cast<const ulonglong2*>(xk + g * 128 + 8 * c + 4);
-        a2[g] = fma2(b0, xa.x, a2[g]);
-        a2[g] = fma2(b1, xa.y, a2[g]);
-        a2[g] = fma2(b2, xb.x, a2[g]);
-        a2[g] = fma2(b3, xb.y, a2[g]);
+    for (int ks = 0; ks < 8; ++ks) {
+      const __half* qr = qh + (kvh * kVG + (n & 3)) * kVQhRow + 16 * ks + kq;
+      bf[ks][0] = n < kVG ? *reinterpret_cast<const uint32_t*>(qr) : 0u;
+      bf[ks][1] = n < kVG ? *reinterpret_cast<const uint32_t*>(qr + 8) : 0u;
+    }
+    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lpc = lane >> 4;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const int j0 = 32 * (warp & 1) + 16 * mt;          // first row of the tile in the head
+      const int r = kvh * kVRmax + j0 + lrow;             // this lane's ldmatrix row
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t a[4];
+        ldmatrix_x4(a, vsm + r * 256 + (((2 * ks + lpc) ^ (r & 15)) << 4));
+        mma16816(c, a, bf[ks][0], bf[ks][1]);
+      }
+      if (kq < kVG) {                   // C: rows lane / 4 (+ 8), queries kq, kq + 1
+        const int jr = j0 + (lane >> 2);
+        qsm[(kvh * kVG + kq) * kVQRow + jr] = c[0] * up;
+        qsm[(kvh * kVG + kq + 1) * kVQRow + jr] = c[1] * up;
+        qsm[(kvh * kVG + kq) * kVQRow + jr + 8] = c[2] * up;
+        qsm[(kvh * kVG + kq + 1) * kVQRow + jr + 8] = c[3] * up;
       }
     }
-#pragma unroll
-    for (int g = 0; g < kVG; ++g) qsm[(kvh * kVG + g) * kVQRow + j] = hsum(a2[g]) * p.scale_log2;
     __syncthreads();                    // Bk's copy in the staging area is dead from here
   }
   if (t0 < t_b) cur = stage(raw0, t0, 0);
