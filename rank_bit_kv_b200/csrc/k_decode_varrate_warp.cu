@@ -2,7 +2,11 @@
 // one lane per (KV head, query head) pair.
 //
 // A token's rank is shared by all KV heads, so every lane of a warp takes the
-// same rank branch for the same token.  The 8 KV heads x 4 query heads of a
+// same rank branch for the same token; a staged chunk of 8 tokens is taken
+// class by class (all its key-rank-4 tokens, then rank 8, ...: one loop per
+// class instead of a dispatch per token), with one maximum update and eight
+// independent exp2 for the chunk, the weights kept in per-warp slots, and the
+// value updates again class by class.  The 8 KV heads x 4 query heads of a
 // batch row fill the 32 lanes; each lane keeps its own online softmax (no
 // shuffles) and its own latent-space accumulator acc[64] in registers; the
 // projected queries q~ = Bk q are formed by the CTA itself (one thread per
@@ -59,6 +63,7 @@ static_assert(kVThreads == kVHkv * kVRmax, "one thread per (KV head, rank) row o
 static_assert(kVHkv * kVRmax * 256 <= kVStage, "Bk's copy fits in the staging area");
 static_assert(kVBuf <= 4096, "record offsets in a staged chunk fit in 12 bits");
 static_assert(32 * kVQhRow * 2 + kVWarps * 4 <= 32 * 128 * 4, "f16 queries and maxima fit");
+static_assert(kVWarps * kVChunk * 32 * 4 <= 32 * 128 * 4, "the warps' score slots fit");
 
 __host__ __device__ constexpr int head_bytes(int r) { return r / 2 + 4 * ((r + 31) / 32); }
 
@@ -222,6 +227,35 @@ __device__ __forceinline__ void value_r(const uint8_t* rec, float p, uint64_t (&
       for (int j = 0; j < 4; ++j)
         acc[4 * wi + j] = fma2(ps2[wi / 4], value_pair(lo, hi, j), acc[4 * wi + j]);
     }
+  }
+}
+
+// the scores of the chunk's tokens of key rank R (bit j of m: token j), into
+// this lane's column of the warp's score slots sc[j][lane]; lane j holds token
+// j's metadata word mw
+template <int R>
+__device__ __forceinline__ void scores_of_class(uint32_t m, uint32_t mw, const uint8_t* kb, int h,
+                                                const float* q, const float (&pre)[5], float* sc,
+                                                int lane) {
+  while (m) {
+    const int j = __ffs(m) - 1;
+    m &= m - 1;
+    const uint32_t w = __shfl_sync(0xffffffffu, mw, j);
+    sc[j * 32 + lane] = score_r<R>(kb + (w & 0xFFFu) + h * head_bytes(R), q, pre);
+  }
+}
+
+// the value updates of the chunk's tokens of value rank R, with the weights p
+// in the score slots
+template <int R>
+__device__ __forceinline__ void values_of_class(uint32_t m, uint32_t mw, const uint8_t* vb, int h,
+                                                const float* sc, int lane,
+                                                uint64_t (&acc)[kVRmax / 2], float (&zc)[6]) {
+  while (m) {
+    const int j = __ffs(m) - 1;
+    m &= m - 1;
+    const uint32_t w = __shfl_sync(0xffffffffu, mw, j);
+    value_r<R>(vb + ((w >> 12) & 0xFFFu) + h * head_bytes(R), sc[j * 32 + lane], acc, zc);
   }
 }
 
@@ -393,6 +427,8 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   if (t0 < t_b) cur = stage(raw0, t0, 0);
   cp_commit();
   const float* const q = qsm + lane * kVQRow;       // lane = h * 4 + qi
+  // this warp's score slots [kVChunk][32] (the staged queries' region, dead here)
+  float* const sc = reinterpret_cast<float*>(vsm + kVOffX) + warp * (kVChunk * 32);
   float pre[5];
   {
     float run = 0.f;
@@ -424,39 +460,48 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     __syncwarp();
     const uint8_t* kb = area + (2 * buf) * kVBuf;
     const uint8_t* vb = area + (2 * buf + 1) * kVBuf;
-    for (int j = 0; j < n; ++j) {
-      const uint32_t w = __shfl_sync(0xffffffffu, cur.w, j);
-      if (!(w >> 30)) continue;
-      float s;
-      const uint8_t* kr = kb + (w & 0xFFFu);
-      switch ((w >> 24) & 7u) {
-        case 0: s = score_r<4>(kr + h * head_bytes(4), q, pre); break;
-        case 1: s = score_r<8>(kr + h * head_bytes(8), q, pre); break;
-        case 2: s = score_r<16>(kr + h * head_bytes(16), q, pre); break;
-        case 3: s = score_r<32>(kr + h * head_bytes(32), q, pre); break;
-        default: s = score_r<64>(kr + h * head_bytes(64), q, pre); break;
-      }
-      if (s > m_thr) {                  // lazily raised maximum (by more than 2^8)
-        const float a = ex2_approx(m - s);
+    // the chunk by rank class: the scores of all its tokens (one loop per key
+    // rank class), one maximum update and the weights of all of them, then the
+    // value updates (one loop per value rank class); lanes >= n hold word 0
+    {
+      const uint32_t mw = cur.w;
+      const bool live = (mw >> 30) != 0;
+      const uint32_t ck = (mw >> 24) & 7u;
+      const uint32_t valid = __ballot_sync(0xffffffffu, live);
+      scores_of_class<4>(__ballot_sync(0xffffffffu, live && ck == 0u), mw, kb, h, q, pre, sc, lane);
+      scores_of_class<8>(__ballot_sync(0xffffffffu, live && ck == 1u), mw, kb, h, q, pre, sc, lane);
+      scores_of_class<16>(__ballot_sync(0xffffffffu, live && ck == 2u), mw, kb, h, q, pre, sc, lane);
+      scores_of_class<32>(__ballot_sync(0xffffffffu, live && ck == 3u), mw, kb, h, q, pre, sc, lane);
+      scores_of_class<64>(__ballot_sync(0xffffffffu, live && ck == 4u), mw, kb, h, q, pre, sc, lane);
+      float smax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kVChunk; ++j)
+        if ((valid >> j) & 1u) smax = fmaxf(smax, sc[j * 32 + lane]);
+      if (smax > m_thr) {               // lazily raised maximum (by more than 2^8)
+        const float a = ex2_approx(m - smax);
         l *= a;
         const uint64_t a2 = pkf(a, a);
 #pragma unroll
         for (int i = 0; i < kVRmax / 2; ++i) acc[i] = mul2(acc[i], a2);
 #pragma unroll
         for (int i = 0; i < 6; ++i) zc[i] *= a;
-        m = s;
-        m_thr = s + 8.f;
+        m = smax;
+        m_thr = smax + 8.f;
       }
-      const float pr = ex2_approx(s - m);
-      l += pr;
-      const uint8_t* vr = vb + ((w >> 12) & 0xFFFu);
-      switch ((w >> 27) & 7u) {
-        case 0: value_r<4>(vr + h * head_bytes(4), pr, acc, zc); break;
-        case 1: value_r<8>(vr + h * head_bytes(8), pr, acc, zc); break;
-        case 2: value_r<16>(vr + h * head_bytes(16), pr, acc, zc); break;
-        case 3: value_r<32>(vr + h * head_bytes(32), pr, acc, zc); break;
-        default: value_r<64>(vr + h * head_bytes(64), pr, acc, zc); break;
+#pragma unroll
+      for (int j = 0; j < kVChunk; ++j) {
+        if ((valid >> j) & 1u) {
+          const float pr = ex2_approx(sc[j * 32 + lane] - m);
+          l += pr;
+          sc[j * 32 + lane] = pr;
+        }
       }
+      const uint32_t cv = (mw >> 27) & 7u;
+      values_of_class<4>(__ballot_sync(0xffffffffu, live && cv == 0u), mw, vb, h, sc, lane, acc, zc);
+      values_of_class<8>(__ballot_sync(0xffffffffu, live && cv == 1u), mw, vb, h, sc, lane, acc, zc);
+      values_of_class<16>(__ballot_sync(0xffffffffu, live && cv == 2u), mw, vb, h, sc, lane, acc, zc);
+      values_of_class<32>(__ballot_sync(0xffffffffu, live && cv == 3u), mw, vb, h, sc, lane, acc, zc);
+      values_of_class<64>(__ballot_sync(0xffffffffu, live && cv == 4u), mw, vb, h, sc, lane, acc, zc);
     }
     __syncwarp();                       // this buffer is refilled by the next stage
     cur = nxt;
