@@ -2,9 +2,9 @@
 // one lane per (KV head, query head) pair.
 //
 // A token's rank is shared by all KV heads, so every lane of a warp takes the
-// same rank branch for the same token; a staged chunk of 8 tokens is taken
-// class by class (all its key-rank-4 tokens, then rank 8, ...: one loop per
-// class instead of a dispatch per token), with one maximum update and eight
+// same rank branch for the same token; a staged chunk of up to 16 tokens is
+// taken class by class (all its key-rank-4 tokens, then rank 8, ...: one loop
+// per class instead of a dispatch per token), with one maximum update and
 // independent exp2 for the chunk, the weights kept in per-warp slots, and the
 // value updates again class by class.  The 8 KV heads x 4 query heads of a
 // batch row fill the 32 lanes; each lane keeps its own online softmax (no
@@ -23,9 +23,10 @@
 // subtraction; value codes are centred, c - 8, and the zero terms p (z + 8 s)
 // of the tokens are summed per rank class and added to the accumulator once,
 // at the end, over the indices each class covers.
-// Every warp streams a contiguous token range in chunks of 8 tokens: the byte
-// range of the chunk's K records and of its V records (contiguous in the
-// per-row streams) is copied with 16-byte cp.async into a double-buffered
+// Every warp streams a contiguous token range in chunks of up to 16 tokens
+// (as many as fit a buffer sized for 8 tokens of rank 64; ~86 bytes per token
+// and stream on average): the byte range of the chunk's K records and of its V
+// records (contiguous in the per-row streams) is copied with 16-byte cp.async into a double-buffered
 // per-warp area while the previous chunk is processed.  The chunk's records are
 // validated once (offsets on their 16-byte grid and inside the staged area,
 // ranks in the rank set), by the lane that holds the token's metadata, which
@@ -44,18 +45,20 @@ using namespace tc;
 
 constexpr int kVWarps = 16;
 constexpr int kVThreads = 32 * kVWarps;
-constexpr int kVChunk = 8;                          // tokens per staged chunk
+constexpr int kVChunk = 16;                         // tokens per staged chunk at most
+constexpr int kVBufTok = 8;                         // tokens of rank 64 a chunk buffer holds
 constexpr int kVHkv = 8, kVG = 4;                   // lanes = KV heads x query heads
 constexpr int kVRmax = 64;
 constexpr int kVRecMax = kVHkv * (kVRmax / 2 + 8);  // token record bytes at rank 64
-constexpr int kVBuf = kVChunk * kVRecMax + 32;      // one staged stream chunk (+ alignment slack)
+constexpr int kVBuf = kVBufTok * kVRecMax + 32;     // one staged stream chunk (+ alignment slack)
 constexpr int kVWarpBytes = 4 * kVBuf;              // K and V, two buffers each
 constexpr int kVStage = kVWarps * kVWarpBytes;
 constexpr int kVQRow = kVRmax + 4;                  // floats per q~ row (16-byte loads conflict-free)
 constexpr int kVOffQ = kVStage;                     // q~ [32][kVQRow] (softmax scale, log2 e folded)
 constexpr int kVOffX = kVOffQ + 32 * kVQRow * 4;    // the queries [32][kVQhRow] f16, then 16 maxima
 constexpr int kVQhRow = 136;                        // f16 per staged query row (272 bytes)
-constexpr int kVSmem = kVOffX + 32 * 128 * 4;
+constexpr int kVOffS = kVOffX + 32 * 128 * 4;       // the warps' score slots [kVChunk][32]
+constexpr int kVSmem = kVOffS + kVWarps * kVChunk * 32 * 4;
 constexpr int kVPst = kVRmax + 2;                   // merge slot: acc[64], m, l
 
 static_assert(kVWarps * 32 * kVPst * 4 <= kVStage, "merge area fits in the staging area");
@@ -63,7 +66,7 @@ static_assert(kVThreads == kVHkv * kVRmax, "one thread per (KV head, rank) row o
 static_assert(kVHkv * kVRmax * 256 <= kVStage, "Bk's copy fits in the staging area");
 static_assert(kVBuf <= 4096, "record offsets in a staged chunk fit in 12 bits");
 static_assert(32 * kVQhRow * 2 + kVWarps * 4 <= 32 * 128 * 4, "f16 queries and maxima fit");
-static_assert(kVWarps * kVChunk * 32 * 4 <= 32 * 128 * 4, "the warps' score slots fit");
+static_assert(kVSmem <= 227 * 1024, "shared memory of a CTA");
 
 __host__ __device__ constexpr int head_bytes(int r) { return r / 2 + 4 * ((r + 31) / 32); }
 
@@ -298,9 +301,10 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     // (bits 0-11, 12-23), rank classes (log2 r - 2; bits 24-26, 27-29) and
     // bit 30 set when its records lie in the staged areas; one shuffle per token
     uint32_t w;
+    int n;                              // tokens in the chunk (the same in every lane)
   };
   auto meta_load = [&](int t0) -> Raw {
-    const int n = min(kVChunk, t_b - t0);
+    const int n = min(kVChunk, t_b - t0);   // at most; the chunk may end sooner
     Raw r;
     r.ok = lane <= n ? __ldg(offk + t0 + lane) : 0;
     r.ov = lane <= n ? __ldg(offv + t0 + lane) : 0;
@@ -308,11 +312,18 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     return r;
   };
   auto stage = [&](const Raw& r, int t0, int buf) -> Meta {
-    const int n = min(kVChunk, t_b - t0);
+    const int nmax = min(kVChunk, t_b - t0);
     Meta mt;
-    const int k0 = __shfl_sync(0xffffffffu, r.ok, 0), k1 = __shfl_sync(0xffffffffu, r.ok, n);
-    const int v0 = __shfl_sync(0xffffffffu, r.ov, 0), v1 = __shfl_sync(0xffffffffu, r.ov, n);
+    const int k0 = __shfl_sync(0xffffffffu, r.ok, 0), v0 = __shfl_sync(0xffffffffu, r.ov, 0);
     const int base_k = k0 & ~15, base_v = v0 & ~15;
+    // the chunk: the longest run of tokens (at most nmax, at least one) whose
+    // K and V records both fit a buffer; lane j holds the end of token j - 1
+    const bool over = lane >= 1 && lane <= nmax &&
+                      (r.ok - base_k > kVBuf || r.ov - base_v > kVBuf || r.ok < k0 || r.ov < v0);
+    const uint32_t ov_mask = __ballot_sync(0xffffffffu, over);
+    const int n = ov_mask ? max(__ffs(ov_mask) - 2, 1) : nmax;
+    mt.n = n;
+    const int k1 = __shfl_sync(0xffffffffu, r.ok, n), v1 = __shfl_sync(0xffffffffu, r.ov, n);
     const uint32_t dk = area_s + (2 * buf) * kVBuf, dv = area_s + (2 * buf + 1) * kVBuf;
     const long long ek = min((long long)k1, sbytes), ev = min((long long)v1, sbytes);
     const int nk = (int)min((ek - base_k + 15) / 16, (long long)(kVBuf / 16));
@@ -332,11 +343,10 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     return mt;
   };
 
-  Meta cur{}, nxt{};
+  Meta cur{0u, 0}, nxt{0u, 0};
   Raw raw0{}, raw1{};                   // metadata of the current and of the next chunk
   int t0 = t_a, buf = 0;
   if (t0 < t_b) raw0 = meta_load(t0);   // in flight during the query projection
-  if (t0 + kVChunk < t_b) raw1 = meta_load(t0 + kVChunk);
 
   // ---- q~ = Bk q for the row's 32 query heads (softmax scale and log2 e
   // folded in), on warp-level MMAs.  Bk (8 heads x 64 rows x 128, fp16) is first
@@ -424,11 +434,14 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
     }
     __syncthreads();                    // Bk's copy in the staging area is dead from here
   }
-  if (t0 < t_b) cur = stage(raw0, t0, 0);
+  if (t0 < t_b) {
+    cur = stage(raw0, t0, 0);
+    if (t0 + cur.n < t_b) raw1 = meta_load(t0 + cur.n);
+  }
   cp_commit();
   const float* const q = qsm + lane * kVQRow;       // lane = h * 4 + qi
-  // this warp's score slots [kVChunk][32] (the staged queries' region, dead here)
-  float* const sc = reinterpret_cast<float*>(vsm + kVOffX) + warp * (kVChunk * 32);
+  // this warp's score slots [kVChunk][32]
+  float* const sc = reinterpret_cast<float*>(vsm + kVOffS) + warp * (kVChunk * 32);
   float pre[5];
   {
     float run = 0.f;
@@ -450,11 +463,12 @@ __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, in
   float m = -INFINITY, m_thr = -INFINITY, l = 0.f;
 
   while (t0 < t_b) {
-    const int n = min(kVChunk, t_b - t0);
-    const int t1 = t0 + n;
+    const int t1 = t0 + cur.n;
     Raw raw2{};
-    if (t1 + kVChunk < t_b) raw2 = meta_load(t1 + kVChunk);
-    if (t1 < t_b) nxt = stage(raw1, t1, buf ^ 1);
+    if (t1 < t_b) {
+      nxt = stage(raw1, t1, buf ^ 1);
+      if (t1 + nxt.n < t_b) raw2 = meta_load(t1 + nxt.n);
+    }
     cp_commit();
     cp_wait<1>();
     __syncwarp();
