@@ -573,7 +573,9 @@ def run_kvc(args, rank, world, torch, dist):
     ms_per_step = ms / K
     value = job_rate(world, step_bytes, K, ms)
 
-    # end to end through the C ABI with host buffers: q in, output out, each step
+    # end to end through the C ABI with host buffers: every step copies its q in
+    # from pinned host memory, decodes, and copies its output out to pinned host
+    # memory, one after the other on the decode's stream
     q_host = q.cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     q_dev = torch.empty_like(q)
@@ -596,7 +598,61 @@ def run_kvc(args, rank, world, torch, dist):
     e2e = {"value": round(job_rate(world, step_bytes, K, ems), 1), "unit": "GB/s",
            "us_per_step": round(ems * 1e3 / K, 2),
            "h2d_bytes_per_step": int(q.numel() * q.element_size()),
-           "d2h_bytes_per_step": int(out.numel() * out.element_size())}
+           "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+           "copies": "serial: q in, decode, output out, every step on one stream"}
+
+    # the same copies on a second stream with two device buffers each, as a
+    # serving loop would run them: step i + 1's q arrives and step i's output
+    # leaves while the neighbouring step decodes (all inside the timed region;
+    # the last output is waited for before the end event)
+    cs = torch.cuda.Stream(device=device)
+    q_hp = [q.cpu().pin_memory() for _ in range(2)]
+    out_hp = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    q_dv = [torch.empty_like(q) for _ in range(2)]
+    out_dv = [torch.empty_like(out) for _ in range(2)]
+    ev_h2d = [torch.cuda.Event() for _ in range(2)]
+    ev_dec = [torch.cuda.Event() for _ in range(2)]
+    ev_d2h = [torch.cuda.Event() for _ in range(2)]
+
+    def pipelined_steps(steps, start_event=None):
+        with torch.cuda.stream(cs):
+            if start_event is not None:
+                cs.wait_event(start_event)
+            q_dv[0].copy_(q_hp[0], non_blocking=True)
+            ev_h2d[0].record(cs)
+        for i in range(steps):
+            k = i & 1
+            if i + 1 < steps:   # the next q; its buffer's last reader (decode i - 1) precedes on cs
+                with torch.cuda.stream(cs):
+                    q_dv[k ^ 1].copy_(q_hp[k ^ 1], non_blocking=True)
+                    ev_h2d[k ^ 1].record(cs)
+            stream.wait_event(ev_h2d[k])
+            if i >= 2:
+                stream.wait_event(ev_d2h[k])   # out_dv[k] copied out by step i - 2
+            kvc.decode(lay, caches[i % n], q_dv[k], out_dv[k], ws)
+            ev_dec[k].record(stream)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev_dec[k])
+                out_hp[k].copy_(out_dv[k], non_blocking=True)
+                ev_d2h[k].record(cs)
+        for k in range(min(steps, 2)):
+            stream.wait_event(ev_d2h[k])
+
+    pipelined_steps(W)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    t0.record(stream)
+    pipelined_steps(K, t0)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    pms = max_over_ranks(torch, dist, t0.elapsed_time(t1), device)
+    e2e_pipelined = {"value": round(job_rate(world, step_bytes, K, pms), 1), "unit": "GB/s",
+                     "us_per_step": round(pms * 1e3 / K, 2),
+                     "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                     "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
+                     "copies": "a second stream, two device buffers each: step i+1's q in and "
+                               "step i's output out overlap the neighbouring decodes"}
 
     dense = None
     if not args.no_dense:
@@ -629,6 +685,7 @@ def run_kvc(args, rank, world, torch, dist):
             "cache_copies": {"n": n, "bytes_each": step_bytes, "total": n * step_bytes},
             "bytes_per_step": step_bytes, "gpu_launches": K * launches,
             "kernel_version": version, "clocks": clocks, "roofline": roof, "e2e": e2e,
+            "e2e_pipelined": e2e_pipelined,
             "dense_bf16_same_step": dense, "workloads": others, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
 
