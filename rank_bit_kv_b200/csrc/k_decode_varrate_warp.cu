@@ -30,7 +30,7 @@
 // per-warp area while the previous chunk is processed.  The chunk's records are
 // validated once (offsets on their 16-byte grid and inside the staged area,
 // ranks in the rank set), by the lane that holds the token's metadata, which
-// packs offsets, rank classes and the verdict into one word.  The warps of a CTA
+// packs offsets, rank classes and the validity bit into one word.  The warps of a CTA
 // merge their (m, l, acc) in shared memory and write one partial per row; the
 // combine kernel maps acc through Bv.
 #include <math.h>
