@@ -151,6 +151,17 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
   const size_t rows = (size_t)p.B * p.Hq;
   const int pst = p.vdim + 2, rv = p.rv, vdim = p.vdim;
   const float* part = p.part + (size_t)row * pst;
+  // the Bv column slice and the signs are not written by the split kernel:
+  // loaded before waiting for it (this block may start during its last CTAs)
+  const int oi = tid & 127, half = tid >> 7;          // output dim, half of the ranks
+  const __half* bv = p.bv + (size_t)kvh * rv * 128 + oi;
+  float bw[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int r = half + 2 * i;
+    bw[i] = r < rv ? h2f(bv[(size_t)r * 128]) : 0.f;
+  }
+  const float sgn = p.resid ? (float)p.signs_v[oi] * rsqrtf((float)kResidDim) : 0.f;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int nS = p.S;
   if (p.seg_W > 0) {
@@ -177,15 +188,6 @@ __global__ void __launch_bounds__(kThreads) combine_lowrank_kernel(Params p) {
     const int sidx = k + i * K;
     pv[i] = (k < K && sidx < nS) ? part[(size_t)sidx * rows * pst + j] : 0.f;
   }
-  const int oi = tid & 127, half = tid >> 7;          // output dim, half of the ranks
-  const __half* bv = p.bv + (size_t)kvh * rv * 128 + oi;
-  float bw[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int r = half + 2 * i;
-    bw[i] = r < rv ? h2f(bv[(size_t)r * 128]) : 0.f;
-  }
-  const float sgn = p.resid ? (float)p.signs_v[oi] * rsqrtf((float)kResidDim) : 0.f;
   // ---- weights
   if (tid < 32) {
     float mx = -INFINITY;

@@ -138,6 +138,9 @@ __device__ __forceinline__ void store_half(uint8_t* buf, const HalfRegs& r, int 
 }
 
 __global__ void __launch_bounds__(kThreads, 1) block_tc_kernel(Params p) {
+  // the combine may launch now: its blocks take SMs as this grid's CTAs exit and
+  // wait (griddepcontrol.wait) for the whole grid before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(1024) uint8_t sm[];
   Bars& bars = *reinterpret_cast<Bars*>(sm + OFF_BAR);
   volatile int* abort = &bars.abort;

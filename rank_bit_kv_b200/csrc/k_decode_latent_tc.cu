@@ -140,6 +140,9 @@ __device__ __forceinline__ uint32_t hsub_u32(uint32_t x, uint32_t c) {
 
 template <int RV, bool RES>
 __global__ void __launch_bounds__(kLThreads, 1) latent_tc_kernel(Params p, LWork wk) {
+  // the combine may launch now: its blocks take SMs as this grid's CTAs exit and
+  // wait (griddepcontrol.wait) for the whole grid before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   using L = Stage<RV, RES>;
   constexpr int NVG = L::NVG, VT = L::VT;
   constexpr int RVB = RV / 2;                   // latent value row bytes

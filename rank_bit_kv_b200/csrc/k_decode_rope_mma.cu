@@ -124,6 +124,9 @@ __host__ __device__ constexpr int recon_rank(int ks, int kappa) {
 
 template <int RV>
 __global__ void __launch_bounds__(kPThreads, 1) rope_mma_kernel(Params p, PWork wk) {
+  // the combine may launch now: its blocks take SMs as this grid's CTAs exit and
+  // wait (griddepcontrol.wait) for the whole grid before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   using L = PStage<RV>;
   constexpr int NVG = L::NVG, VT = L::VT;
   constexpr int RVB = RV / 2;

@@ -267,6 +267,9 @@ __device__ __forceinline__ bool rank_in_set(int r) {
 }
 
 __global__ void __launch_bounds__(kVThreads, 1) varrate_warp_kernel(Params p, int split_len) {
+  // the combine may launch now: its blocks take SMs as this grid's CTAs exit and
+  // wait (griddepcontrol.wait) for the whole grid before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(128) uint8_t vsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s_idx = blockIdx.x, b = blockIdx.y;
