@@ -109,82 +109,12 @@ __global__ void __launch_bounds__(kThreads) qproj_group_kernel(Params p) {
 }
 
 // Block-shared latent, head dim 128: one block per (layer, batch row, KV head)
-// forms the absorbed queries of the whole query group.  The layer's W_k slice
-// (D rows x 128) streams through shared memory in chunks of 64 rows (16-byte
-// cp.async, double-buffered, rows padded to 272 bytes so that 32 lanes reading
-// 32 rows are conflict-free); thread (r, g0) dots row r of the chunk with the
-// group's queries g0, g0 + 4.
-constexpr int kQbRows = 64;
+// forms the absorbed queries of the whole query group from the layer's W_k
+// slice (D rows x 128, staged in shared memory with rows padded to 272 bytes
+// so that ldmatrix reads are conflict-free).
 constexpr int kQbRow = 272;
 
-__global__ void __launch_bounds__(256) qproj_block_kernel(Params p) {
-  __shared__ __align__(16) float qs[8][128];
-  __shared__ __align__(16) uint8_t wsm[2][kQbRows * kQbRow];
-  const int unit = blockIdx.x;             // (l * B + b) * Hkv + kvh
-  const int kvh = unit % p.Hkv;
-  const int l = unit / (p.B * p.Hkv);
-  const int row0 = (unit / p.Hkv) * p.Hq + kvh * p.G;   // first query row of the group
-  const int tid = threadIdx.x, G = p.G;
-  const __half* w = p.bk + (int64_t)l * p.D * p.Hkv * 128 + kvh * 128;
-  const int n_chunks = (p.D + kQbRows - 1) / kQbRows;
-  auto stage = [&](int c, int buf) {
-    for (int e = tid; e < kQbRows * 16; e += 256) {
-      const int r = e >> 4, part = e & 15, row = c * kQbRows + r;
-      if (row < p.D) {
-        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(&wsm[buf][r * kQbRow + part * 16]);
-        const __half* src = w + (int64_t)row * p.Hkv * 128 + part * 8;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-      }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-  stage(0, 0);
-  for (int e = tid; e < G * 128; e += 256)
-    qs[e >> 7][e & 127] = bf2f(p.q[(int64_t)(row0 + (e >> 7)) * 128 + (e & 127)]);
-  const int r = tid & (kQbRows - 1), g0 = tid >> 6;
-  for (int c = 0; c < n_chunks; ++c) {
-    if (c + 1 < n_chunks) {
-      stage(c + 1, (c + 1) & 1);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    }
-    __syncthreads();
-    const int row = c * kQbRows + r;
-    const uint4* wr = reinterpret_cast<const uint4*>(&wsm[c & 1][r * kQbRow]);
-    float acc[2] = {0.f, 0.f};
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-      const uint4 u = wr[k];
-      const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        const int g = g0 + 4 * gi;
-        if (g < G) {
-          const float4 qa = *reinterpret_cast<const float4*>(&qs[g][8 * k]);
-          const float4 qb = *reinterpret_cast<const float4*>(&qs[g][8 * k + 4]);
-          const float qq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[j]));
-            acc[gi] = fmaf(f.x, qq[2 * j], acc[gi]);
-            acc[gi] = fmaf(f.y, qq[2 * j + 1], acc[gi]);
-          }
-        }
-      }
-    }
-    if (row < p.D) {
-#pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        const int g = g0 + 4 * gi;
-        if (g < G) p.qt[(int64_t)(row0 + g) * p.qdim + row] = acc[gi];
-      }
-    }
-    __syncthreads();                       // buffer c & 1 is restaged for chunk c + 2
-  }
-}
-
-// The same projection on warp-level MMAs, with the whole W_k slice in flight
+// The projection runs on warp-level MMAs, with the whole W_k slice in flight
 // at once (D <= 768): M = 16 rows of the slice, N = 8 query heads (G of them
 // real), K = 16 head dims.  The group's queries are scaled by a power of two,
 // 2^-e, so that the largest lies below 2^14, and rounded to f16: exact for
@@ -298,10 +228,6 @@ cudaError_t launch_qproj(const Params& p, cudaStream_t s) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     qproj_block_mma_kernel<<<p.L * p.B * p.Hkv, 256, bytes, s>>>(p);
-    return cudaGetLastError();
-  }
-  if (p.kind == KVC_BLOCK_SHARED && p.d == 128 && p.G <= 8) {
-    qproj_block_kernel<<<p.L * p.B * p.Hkv, 256, 0, s>>>(p);
     return cudaGetLastError();
   }
   const int rows = p.L * p.B * p.Hq;
