@@ -133,7 +133,7 @@ void kvc_select_rope_kernel(int32_t which) { g_rope_kernel = which == 2 ? 2 : 0;
 void kvc_select_varrate_kernel(int32_t which) { g_varrate_kernel = which == 1 ? 1 : 0; }
 
 const char* kvc_version(void) {
-  return "kvc 0.3 (sm_100a; decode kernels rev 15; rope_mma rev 12)";
+  return "kvc 0.3 (sm_100a; decode kernels rev 16; rope_mma rev 13)";
 }
 
 kvc_status kvc_create_layout(const kvc_layout_desc* desc, kvc_layout** out) {
