@@ -9,9 +9,9 @@
 // value updates again class by class.  The 8 KV heads x 4 query heads of a
 // batch row fill the 32 lanes; each lane keeps its own online softmax (no
 // shuffles) and its own latent-space accumulator acc[64] in registers; the
-// projected queries q~ = Bk q are formed by the CTA itself (one thread per
-// (KV head, rank) row of Bk, all four query heads of the group) into shared
-// memory (on warp-level MMAs), where each lane reads its own row:
+// projected queries q~ = Bk q are formed by the CTA itself on warp-level MMAs
+// (warp w: 32 rows of head w / 2) into shared memory, where each lane reads
+// its own row:
 //   s_t = sum_{i < r_k(t)} q~_i (c_i s_g + z_g),
 //   acc_i += p_t (c_i s_g + z_g) for i < r_v(t).
 // Keeping q~ out of the registers lets 16 warps share an SM (4 per scheduler)
@@ -25,14 +25,15 @@
 // at the end, over the indices each class covers.
 // Every warp streams a contiguous token range in chunks of up to 16 tokens
 // (as many as fit a buffer sized for 8 tokens of rank 64; ~86 bytes per token
-// and stream on average): the byte range of the chunk's K records and of its V
-// records (contiguous in the per-row streams) is copied with 16-byte cp.async into a double-buffered
-// per-warp area while the previous chunk is processed.  The chunk's records are
-// validated once (offsets on their 16-byte grid and inside the staged area,
-// ranks in the rank set), by the lane that holds the token's metadata, which
-// packs offsets, rank classes and the validity bit into one word.  The warps of a CTA
-// merge their (m, l, acc) in shared memory and write one partial per row; the
-// combine kernel maps acc through Bv.
+// and stream on average): the byte range of the chunk's K records and of its
+// V records (contiguous in the per-row streams) is copied with 16-byte
+// cp.async into a double-buffered per-warp area while the previous chunk is
+// processed.  The chunk's records are validated once (offsets on their
+// 16-byte grid and inside the staged area, ranks in the rank set), by the
+// lane that holds the token's metadata, which packs offsets, rank classes and
+// the validity bit into one word.  The warps of a CTA merge their (m, l, acc)
+// in shared memory and write one partial per row; the combine kernel maps acc
+// through Bv.
 #include <math.h>
 
 #include "kvc_device.cuh"
@@ -62,7 +63,7 @@ constexpr int kVSmem = kVOffS + kVWarps * kVChunk * 32 * 4;
 constexpr int kVPst = kVRmax + 2;                   // merge slot: acc[64], m, l
 
 static_assert(kVWarps * 32 * kVPst * 4 <= kVStage, "merge area fits in the staging area");
-static_assert(kVThreads == kVHkv * kVRmax, "one thread per (KV head, rank) row of Bk");
+static_assert(kVThreads * 16 == kVHkv * kVRmax * 16, "16 Bk copy pieces per thread");
 static_assert(kVHkv * kVRmax * 256 <= kVStage, "Bk's copy fits in the staging area");
 static_assert(kVBuf <= 4096, "record offsets in a staged chunk fit in 12 bits");
 static_assert(32 * kVQhRow * 2 + kVWarps * 4 <= 32 * 128 * 4, "f16 queries and maxima fit");
